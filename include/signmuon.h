@@ -1,0 +1,205 @@
+/*
+ * signmuon.h -- C ABI of libsignmuon.so, the B200 (sm_100a) Sign-Muon step.
+ *
+ * The method is the one described in the technical summary of "SignMuon:
+ * Communication-Efficient Distributed Muon Optimization" (arXiv 2605.16311),
+ * section 2, "Algorithmic flow (distributed)", steps 1-5:
+ *   1. every worker m updates its momentum M^(m) from its gradient G^(m) and
+ *      computes the polar factor U^(m) with Newton-Schulz iterations;
+ *   2. it takes the entrywise sign S^(m) = sign(U^(m));
+ *   3. the signs are exchanged as an integer sum (int8) or as 1-bit packed
+ *      buffers;
+ *   4. the majority vote sign(sum_m S^(m)) updates W <- W - eta * vote;
+ *   5. optionally, a local polar step on the voted matrix.
+ * Here the M workers are M buffers on one GPU, so step 3's collective is the
+ * local M-way reduction inside signmuon_vote_update.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All pointers named "device" point to device memory of the current CUDA
+ *   device; arrays of pointers (type `const void* const*` etc.) are HOST
+ *   arrays whose elements are device pointers.  The library copies what it
+ *   needs into the caller's device workspace.
+ * - Ownership: the caller owns every buffer, including the workspace.  The
+ *   library allocates no memory and keeps no state between calls.
+ * - Units: a "unit" is one (matrix i, worker m) pair; per-unit arrays have
+ *   n_mats * n_workers entries, indexed i * n_workers + m.
+ * - Matrices are row-major.  Dense fp32/bf16/int8 buffers have row stride
+ *   `cols`.  bf16 Newton-Schulz buffers (the "X" buffers and the vote matrix)
+ *   have row stride signmuon_x_ld(cols) elements (cols rounded up to 8).
+ * - Packed sign buffers: row-major uint32 words, ceil(cols/32) words per row;
+ *   bit j of word w in row r is entry (r, 32w + j); a set bit is +1; bits
+ *   past the last column are 0.  A buffer holds signmuon_packed_words(shape)
+ *   words (the row-major words, rounded up to a multiple of 4).
+ * - int8 sign buffers: row-major int8 in {-1, +1}, row stride cols.
+ * - sign(0) = sign(-0) = +1 and a NaN maps to +1 (the test is "u < 0").
+ * - Every buffer pointer must be 16-byte aligned (SIGNMUON_ERR_ALIGNMENT).
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *   enqueued asynchronously; no entry point synchronises the host except
+ *   signmuon_device_error.
+ * - Errors: arguments are validated before anything is enqueued and a
+ *   status is returned; nothing is launched when validation fails.  Launch
+ *   failures return SIGNMUON_ERR_CUDA.  Kernels never trap: a kernel that
+ *   gives up waiting (a bounded wait ran out) records a nonzero code in the
+ *   first word of the workspace it was given, readable with
+ *   signmuon_device_error.
+ */
+#ifndef SIGNMUON_H_
+#define SIGNMUON_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum signmuon_status {
+  SIGNMUON_OK = 0,
+  SIGNMUON_ERR_INVALID_ARG = 1,  /* null pointer, size <= 0, count out of range */
+  SIGNMUON_ERR_ALIGNMENT = 2,    /* a buffer is not 16-byte aligned             */
+  SIGNMUON_ERR_UNSUPPORTED = 3,  /* valid request this build cannot run        */
+  SIGNMUON_ERR_WORKSPACE = 4,    /* workspace null or smaller than required     */
+  SIGNMUON_ERR_CUDA = 5          /* a CUDA call or kernel launch failed        */
+} signmuon_status;
+
+typedef enum signmuon_dtype { SIGNMUON_F32 = 0, SIGNMUON_BF16 = 1 } signmuon_dtype;
+
+/* What the last Newton-Schulz iteration writes. */
+typedef enum signmuon_ns_out {
+  SIGNMUON_OUT_PACK1 = 0,     /* 1-bit packed signs, one buffer per unit        */
+  SIGNMUON_OUT_INT8 = 1,      /* int8 +-1 signs, one buffer per unit             */
+  SIGNMUON_OUT_UPDATE_W = 2,  /* W <- W - eta * U in place (n_workers must be 1) */
+  SIGNMUON_OUT_U_F32 = 3      /* the polar estimate U itself, fp32 [rows, cols]  */
+} signmuon_ns_out;
+
+typedef struct signmuon_shape {
+  int32_t rows;
+  int32_t cols;
+} signmuon_shape;
+
+#define SIGNMUON_MAX_WORKERS 127
+
+/* Human-readable name of a status code (static storage). */
+const char* signmuon_status_string(int status);
+
+/* Library ABI version (incremented on any signature change). */
+int signmuon_abi_version(void);
+
+/* Row stride, in elements, of a bf16 Newton-Schulz buffer with `cols` columns:
+ * cols rounded up to a multiple of 8 (16 bytes, the TMA stride granule). */
+int32_t signmuon_x_ld(int32_t cols);
+
+/* Words (uint32) of one packed sign buffer of this shape: rows*ceil(cols/32)
+ * rounded up to a multiple of 4.  Returns -1 for an invalid shape. */
+int64_t signmuon_packed_words(signmuon_shape shape);
+
+/* Reads (synchronously: waits for the device) the error word a kernel left
+ * in `workspace` (device pointer given to an earlier call) and clears it.
+ * *code = 0 means no kernel gave up.  Returns SIGNMUON_ERR_CUDA if the copy
+ * fails. */
+signmuon_status signmuon_device_error(void* workspace, uint32_t* code, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Step 1a: momentum and Frobenius normalisation.
+ * Source: SignMuon summary, section 2 "Algorithmic flow", step 1 (each
+ * worker updates its local momentum) and section 4 "nanoGPT" (Frobenius
+ * scaling of the Newton-Schulz input).
+ *
+ * For every unit u = i*n_workers + m (matrix i has shapes[i]):
+ *   mom[u]    <- beta * mom[u] + (1 - beta) * grad[u]          (fp32, in place)
+ *   x_bf16[u] <- bf16(mom[u])  (row stride signmuon_x_ld(cols); pad columns
+ *                               are not written)
+ *   inv_norm[u] <- 1 / (||mom[u]||_F + 1e-7)                   (fp32)
+ * so that the Newton-Schulz input is X0 = inv_norm[u] * x_bf16[u].
+ * The norm is reduced in a fixed order (bit-reproducible run to run).
+ *
+ * grad: per-unit device pointers, dtype grad_dtype, [rows, cols].
+ * mom: per-unit device fp32 [rows, cols], updated in place.
+ * x_bf16: per-unit device bf16 [rows, x_ld].
+ * inv_norm: device fp32 [n_mats * n_workers].
+ * workspace: device, >= signmuon_momentum_workspace_bytes(...) bytes.
+ * ---------------------------------------------------------------------- */
+size_t signmuon_momentum_workspace_bytes(const signmuon_shape* shapes, int n_mats,
+                                         int n_workers);
+signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                       signmuon_dtype grad_dtype, const void* const* grad,
+                                       float* const* mom, float beta, void* const* x_bf16,
+                                       float* inv_norm, void* workspace, size_t ws_bytes,
+                                       void* stream);
+
+/* ------------------------------------------------------------------------
+ * Step 1b-2: k Newton-Schulz iterations, then the entrywise sign.
+ * Source: SignMuon summary, section 2 "Core mechanism" item 1 and
+ * "Algorithmic flow" steps 1-2 (and step 5 for SIGNMUON_OUT_UPDATE_W).
+ *
+ * For every unit, starting from X = inv_norm[u] * x_bf16[u], k times:
+ *   rows <= cols:  A = X X^T,  B = b A + c A^2,  X <- a X + B X
+ *   rows >  cols:  A = X^T X,  B = b A + c A^2,  X <- a X + X B
+ * on the tensor cores (bf16 operands, fp32 accumulation, bf16 between
+ * iterations).  The last iteration's epilogue writes, per out_mode:
+ *   PACK1:    out[u] = packed sign(U)   (uint32, signmuon_packed_words words)
+ *   INT8:     out[u] = int8 sign(U)     ([rows, cols])
+ *   U_F32:    out[u] = U                (fp32 [rows, cols])
+ *   UPDATE_W: w[i] <- w[i] - eta * U    (w_dtype [rows, cols], in place;
+ *             requires n_workers == 1; `out` is ignored and may be NULL)
+ * k = 0 writes the same outputs from U = X0.
+ *
+ * x_bf16 buffers are CLOBBERED (used as one of the two iterate buffers).
+ * Coefficients a, b, c are the caller's (the build uses 3.4445, -4.7750,
+ * 2.0315).  k must be in [0, 64].
+ * workspace: device; signmuon_newton_schulz_workspace_bytes(..., 0) bytes
+ * run all units at once, any size >= the value for minimal=1 runs them in
+ * successive waves.
+ * ---------------------------------------------------------------------- */
+size_t signmuon_newton_schulz_workspace_bytes(const signmuon_shape* shapes, int n_mats,
+                                              int n_workers, int minimal);
+signmuon_status signmuon_newton_schulz_batched(
+    const signmuon_shape* shapes, int n_mats, int n_workers, void* const* x_bf16,
+    const float* inv_norm, int k, float a, float b, float c, signmuon_ns_out out_mode,
+    void* const* out, signmuon_dtype w_dtype, void* const* w, float eta, void* workspace,
+    size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Step 2-3 standalone: entrywise sign of a matrix, packed or int8.
+ * Source: SignMuon summary, section 2 "Algorithmic flow", steps 2-3 and
+ * "Communication efficiency" (1 bit per entry, or 8 bits with int8).
+ *
+ * u: device [rows, ld_u] of u_dtype (ld_u >= cols, in elements).
+ * out: device; packed (signmuon_packed_words words, pad bits 0 and trailing
+ * pad words 0) when int8_out == 0, else int8 [rows, cols].
+ * ---------------------------------------------------------------------- */
+signmuon_status signmuon_sign_pack(signmuon_shape shape, signmuon_dtype u_dtype, const void* u,
+                                   int64_t ld_u, int int8_out, void* out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Steps 3-4: majority vote over the M workers' signs and the update.
+ * Source: SignMuon summary, section 2 "Core mechanism" item 3 (integer sum
+ * then sign) and "Algorithmic flow" step 4 (W <- W - eta * vote).
+ *
+ * For every matrix i, with c = number of workers whose sign is +1:
+ *   vote = +1 if 2c > M, -1 if 2c < M, 0 on a tie (even M).
+ * signs: per-unit device buffers, packed (int8_in == 0) or int8.
+ * Update mode (vote_bf16 == NULL):  w[i] <- w[i] - eta * vote, computed
+ *   exactly and rounded once to w_dtype (round to nearest even).
+ * Vote-out mode (vote_bf16 != NULL): w is not touched; writes the vote as
+ *   bf16 {-1, 0, +1} to vote_bf16[i] ([rows, signmuon_x_ld(cols)]), its
+ *   number of non-zeros to nnz[i] (device int64) and 1/sqrt(nnz) (0 when
+ *   nnz = 0) to vote_inv_norm[i] (device fp32): the input of the optional
+ *   local polar step (signmuon_newton_schulz_batched with n_workers = 1,
+ *   k = 1, out_mode = SIGNMUON_OUT_UPDATE_W).
+ * 1 <= n_workers <= SIGNMUON_MAX_WORKERS.
+ * workspace: device, >= signmuon_vote_workspace_bytes(...) bytes.
+ * ---------------------------------------------------------------------- */
+size_t signmuon_vote_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers);
+signmuon_status signmuon_vote_update(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                     int int8_in, const void* const* signs,
+                                     signmuon_dtype w_dtype, void* const* w, float eta,
+                                     void* const* vote_bf16, int64_t* nnz, float* vote_inv_norm,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIGNMUON_H_ */

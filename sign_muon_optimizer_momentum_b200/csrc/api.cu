@@ -1,0 +1,415 @@
+// C ABI of libsignmuon.so: argument validation, workspace layout, descriptor
+// planning (tensor maps, unit tables) and kernel launches.  The declarations
+// and their contracts are in include/signmuon.h.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+using namespace signmuon;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int32_t x_ld_of(int32_t cols) { return (cols + 7) / 8 * 8; }
+inline int64_t wpr_of(int32_t cols) { return (cols + 31) / 32; }
+inline int64_t packed_words_of(signmuon_shape s) { return ((int64_t)s.rows * wpr_of(s.cols) + 3) / 4 * 4; }
+
+signmuon_status validate_shapes(const signmuon_shape* shapes, int n_mats) {
+  if (!shapes || n_mats <= 0) return SIGNMUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n_mats; ++i)
+    if (shapes[i].rows <= 0 || shapes[i].cols <= 0) return SIGNMUON_ERR_INVALID_ARG;
+  return SIGNMUON_OK;
+}
+
+signmuon_status validate_ptrs(const void* const* p, int n, bool allow_null = false) {
+  if (!p) return SIGNMUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (!p[i]) {
+      if (allow_null) continue;
+      return SIGNMUON_ERR_INVALID_ARG;
+    }
+    if (!aligned16(p[i])) return SIGNMUON_ERR_ALIGNMENT;
+  }
+  return SIGNMUON_OK;
+}
+
+signmuon_status check_workspace(void* ws, size_t have, size_t need) {
+  if (!ws) return SIGNMUON_ERR_WORKSPACE;
+  if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SIGNMUON_ERR_ALIGNMENT;
+  if (have < need) return SIGNMUON_ERR_WORKSPACE;
+  return SIGNMUON_OK;
+}
+
+inline signmuon_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SIGNMUON_OK : SIGNMUON_ERR_CUDA; }
+
+// ----------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] with row stride ld elements; 64x64 boxes,
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_bf16_2d(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- NS planning
+struct UnitBytes {
+  size_t a, b, xalt, total;
+};
+
+UnitBytes ns_unit_bytes(signmuon_shape sh) {
+  const int64_t s = std::min(sh.rows, sh.cols);
+  const int64_t ld_s = x_ld_of((int32_t)s);
+  UnitBytes u;
+  u.a = align_up((size_t)(s * ld_s * 2), 1024);
+  u.b = u.a;
+  u.xalt = align_up((size_t)sh.rows * x_ld_of(sh.cols) * 2, 1024);
+  u.total = u.a + u.b + u.xalt;
+  return u;
+}
+
+int ns_tiles(int rows, int cols, int stage) {
+  const bool tall = rows > cols;
+  const int s = tall ? cols : rows;
+  if (stage == kStageApply) {
+    return ((rows + kBM - 1) / kBM) * ((cols + kBN - 1) / kBN);
+  }
+  const int tm = (s + kBM - 1) / kBM, tn = (s + kBN - 1) / kBN;
+  int n = 0;
+  for (int i = 0; i < tm; ++i) n += tn - (i >> 1);
+  return n;
+}
+
+size_t ns_desc_bytes(int n_units) { return align_up((size_t)n_units * sizeof(NsUnit), 1024); }
+
+}  // namespace
+
+extern "C" {
+
+const char* signmuon_status_string(int status) {
+  switch (status) {
+    case SIGNMUON_OK: return "SIGNMUON_OK";
+    case SIGNMUON_ERR_INVALID_ARG: return "SIGNMUON_ERR_INVALID_ARG";
+    case SIGNMUON_ERR_ALIGNMENT: return "SIGNMUON_ERR_ALIGNMENT";
+    case SIGNMUON_ERR_UNSUPPORTED: return "SIGNMUON_ERR_UNSUPPORTED";
+    case SIGNMUON_ERR_WORKSPACE: return "SIGNMUON_ERR_WORKSPACE";
+    case SIGNMUON_ERR_CUDA: return "SIGNMUON_ERR_CUDA";
+    default: return "SIGNMUON_UNKNOWN_STATUS";
+  }
+}
+
+int signmuon_abi_version(void) { return kAbiVersion; }
+
+int32_t signmuon_x_ld(int32_t cols) { return cols <= 0 ? -1 : x_ld_of(cols); }
+
+int64_t signmuon_packed_words(signmuon_shape shape) {
+  if (shape.rows <= 0 || shape.cols <= 0) return -1;
+  return packed_words_of(shape);
+}
+
+signmuon_status signmuon_device_error(void* workspace, uint32_t* code, void* stream) {
+  if (!workspace || !code) return SIGNMUON_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SIGNMUON_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SIGNMUON_ERR_CUDA;
+  *code = v;
+  if (v != 0 && cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return SIGNMUON_ERR_CUDA;
+  return SIGNMUON_OK;
+}
+
+// ------------------------------------------------------------------ momentum
+static int mom_blocks(signmuon_shape s) {
+  const int64_t n = (int64_t)s.rows * s.cols;
+  return (int)((n + kMomElemsPerBlock - 1) / kMomElemsPerBlock);
+}
+
+size_t signmuon_momentum_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers) {
+  if (validate_shapes(shapes, n_mats) != SIGNMUON_OK || n_workers <= 0) return 0;
+  int64_t blocks = 0;
+  for (int i = 0; i < n_mats; ++i) blocks += (int64_t)mom_blocks(shapes[i]) * n_workers;
+  const int64_t units = (int64_t)n_mats * n_workers;
+  return kWsHeaderBytes + align_up((size_t)units * sizeof(MomUnit), 256) + align_up((size_t)blocks * 4, 256);
+}
+
+signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                       signmuon_dtype grad_dtype, const void* const* grad, float* const* mom,
+                                       float beta, void* const* x_bf16, float* inv_norm, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+  signmuon_status st = validate_shapes(shapes, n_mats);
+  if (st) return st;
+  if (n_workers <= 0 || n_workers > SIGNMUON_MAX_WORKERS) return SIGNMUON_ERR_INVALID_ARG;
+  if (grad_dtype != SIGNMUON_F32 && grad_dtype != SIGNMUON_BF16) return SIGNMUON_ERR_INVALID_ARG;
+  const int units = n_mats * n_workers;
+  if ((st = validate_ptrs(grad, units))) return st;
+  if ((st = validate_ptrs(reinterpret_cast<const void* const*>(mom), units))) return st;
+  if ((st = validate_ptrs(reinterpret_cast<const void* const*>(x_bf16), units))) return st;
+  if (!inv_norm) return SIGNMUON_ERR_INVALID_ARG;
+  if (!aligned16(inv_norm)) return SIGNMUON_ERR_ALIGNMENT;
+  if ((st = check_workspace(workspace, ws_bytes, signmuon_momentum_workspace_bytes(shapes, n_mats, n_workers))))
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  std::vector<MomUnit> mu(units);
+  int blocks = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    for (int m = 0; m < n_workers; ++m) {
+      MomUnit& u = mu[i * n_workers + m];
+      u.grad = grad[i * n_workers + m];
+      u.mom = mom[i * n_workers + m];
+      u.x = static_cast<__nv_bfloat16*>(x_bf16[i * n_workers + m]);
+      u.rows = shapes[i].rows;
+      u.cols = shapes[i].cols;
+      u.n = (int64_t)u.rows * u.cols;
+      u.ld_x = x_ld_of(u.cols);
+      u.block_begin = blocks;
+      u.block_count = mom_blocks(shapes[i]);
+      u.pad_ = 0;
+      blocks += u.block_count;
+    }
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  MomUnit* d_units = reinterpret_cast<MomUnit*>(ws + kWsHeaderBytes);
+  float* partials = reinterpret_cast<float*>(ws + kWsHeaderBytes + align_up((size_t)units * sizeof(MomUnit), 256));
+  cudaError_t e = upload_bytes(d_units, mu.data(), mu.size() * sizeof(MomUnit), s);
+  if (e == cudaSuccess) e = launch_momentum(d_units, units, blocks, grad_dtype == SIGNMUON_BF16, beta, partials, s);
+  if (e == cudaSuccess) e = launch_momentum_finalize(d_units, units, partials, inv_norm, s);
+  return cuda_status(e);
+}
+
+// ------------------------------------------------------------ Newton-Schulz
+size_t signmuon_newton_schulz_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                              int minimal) {
+  if (validate_shapes(shapes, n_mats) != SIGNMUON_OK || n_workers <= 0) return 0;
+  const int units = n_mats * n_workers;
+  size_t arena = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const size_t b = ns_unit_bytes(shapes[i]).total;
+    arena = minimal ? std::max(arena, b) : arena + b * n_workers;
+  }
+  return kWsHeaderBytes + ns_desc_bytes(units) + arena;
+}
+
+signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                               void* const* x_bf16, const float* inv_norm, int k, float a,
+                                               float b, float c, signmuon_ns_out out_mode, void* const* out,
+                                               signmuon_dtype w_dtype, void* const* w, float eta,
+                                               void* workspace, size_t ws_bytes, void* stream) {
+  signmuon_status st = validate_shapes(shapes, n_mats);
+  if (st) return st;
+  if (n_workers <= 0 || n_workers > SIGNMUON_MAX_WORKERS) return SIGNMUON_ERR_INVALID_ARG;
+  if (k < 0 || k > 64) return SIGNMUON_ERR_INVALID_ARG;
+  if (out_mode != SIGNMUON_OUT_PACK1 && out_mode != SIGNMUON_OUT_INT8 && out_mode != SIGNMUON_OUT_UPDATE_W &&
+      out_mode != SIGNMUON_OUT_U_F32)
+    return SIGNMUON_ERR_INVALID_ARG;
+  const int units = n_mats * n_workers;
+  if ((st = validate_ptrs(x_bf16, units))) return st;
+  if (!inv_norm) return SIGNMUON_ERR_INVALID_ARG;
+  if (!aligned16(inv_norm)) return SIGNMUON_ERR_ALIGNMENT;
+  if (out_mode == SIGNMUON_OUT_UPDATE_W) {
+    if (n_workers != 1) return SIGNMUON_ERR_INVALID_ARG;
+    if (w_dtype != SIGNMUON_F32 && w_dtype != SIGNMUON_BF16) return SIGNMUON_ERR_INVALID_ARG;
+    if ((st = validate_ptrs(w, n_mats))) return st;
+  } else {
+    if ((st = validate_ptrs(out, units))) return st;
+  }
+  const size_t need_min = signmuon_newton_schulz_workspace_bytes(shapes, n_mats, n_workers, 1);
+  if ((st = check_workspace(workspace, ws_bytes, need_min))) return st;
+  if (!encode_fn()) return SIGNMUON_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  NsUnit* d_units = reinterpret_cast<NsUnit*>(ws + kWsHeaderBytes);
+  uint8_t* arena = ws + kWsHeaderBytes + ns_desc_bytes(units);
+  const size_t arena_bytes = ws_bytes - kWsHeaderBytes - ns_desc_bytes(units);
+
+  // Plan waves: consecutive units whose buffers fit the arena together.
+  std::vector<NsUnit> hu(units);
+  std::vector<int> wave_begin;
+  size_t used = arena_bytes;  // forces a new wave at unit 0
+  int64_t max_elems = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const UnitBytes ub = ns_unit_bytes(shapes[i]);
+    const int rows = shapes[i].rows, cols = shapes[i].cols;
+    const int32_t sdim = std::min(rows, cols);
+    max_elems = std::max(max_elems, (int64_t)rows * cols);
+    for (int m = 0; m < n_workers; ++m) {
+      const int ui = i * n_workers + m;
+      if (used + ub.total > arena_bytes) {
+        wave_begin.push_back(ui);
+        used = 0;
+      }
+      NsUnit& u = hu[ui];
+      memset(&u, 0, sizeof(NsUnit));
+      u.rows = rows;
+      u.cols = cols;
+      u.ld_x = x_ld_of(cols);
+      u.ld_s = x_ld_of(sdim);
+      u.x = static_cast<__nv_bfloat16*>(x_bf16[ui]);
+      u.a = reinterpret_cast<__nv_bfloat16*>(arena + used);
+      u.b = reinterpret_cast<__nv_bfloat16*>(arena + used + ub.a);
+      u.xalt = reinterpret_cast<__nv_bfloat16*>(arena + used + ub.a + ub.b);
+      used += ub.total;
+      u.out = out_mode == SIGNMUON_OUT_UPDATE_W ? w[i] : out[ui];
+      u.scale = inv_norm + ui;
+      if (!encode_bf16_2d(&u.map_x, u.x, cols, rows, u.ld_x) ||
+          !encode_bf16_2d(&u.map_xalt, u.xalt, cols, rows, u.ld_x) ||
+          !encode_bf16_2d(&u.map_a, u.a, sdim, sdim, u.ld_s) ||
+          !encode_bf16_2d(&u.map_b, u.b, sdim, sdim, u.ld_s))
+        return SIGNMUON_ERR_UNSUPPORTED;
+    }
+  }
+  wave_begin.push_back(units);
+  // Tile prefixes restart at each wave (a launch covers one wave).
+  for (size_t wv = 0; wv + 1 < wave_begin.size(); ++wv) {
+    int pre[3] = {0, 0, 0};
+    for (int ui = wave_begin[wv]; ui < wave_begin[wv + 1]; ++ui) {
+      for (int stg = 0; stg < 3; ++stg) {
+        hu[ui].tile_begin[stg] = pre[stg];
+        hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg);
+        pre[stg] += hu[ui].tile_count[stg];
+      }
+    }
+  }
+  cudaError_t e = upload_bytes(d_units, hu.data(), hu.size() * sizeof(NsUnit), s);
+  if (e != cudaSuccess) return SIGNMUON_ERR_CUDA;
+
+  for (size_t wv = 0; wv + 1 < wave_begin.size(); ++wv) {
+    const int u0 = wave_begin[wv], nu = wave_begin[wv + 1] - u0;
+    if (k == 0) {
+      e = launch_ns_identity(d_units + u0, nu, max_elems, (int)out_mode, (int)w_dtype, eta, s);
+      if (e != cudaSuccess) return SIGNMUON_ERR_CUDA;
+      continue;
+    }
+    int total[3] = {0, 0, 0};
+    for (int stg = 0; stg < 3; ++stg) {
+      const NsUnit& lastu = hu[u0 + nu - 1];
+      total[stg] = lastu.tile_begin[stg] + lastu.tile_count[stg];
+    }
+    for (int it = 0; it < k; ++it) {
+      NsLaunch L;
+      memset(&L, 0, sizeof(L));
+      L.units = d_units + u0;
+      L.n_units = nu;
+      L.parity = it & 1;
+      L.first = it == 0;
+      L.a = a;
+      L.b = b;
+      L.c = c;
+      L.eta = eta;
+      L.w_dtype = (int)w_dtype;
+      L.err = reinterpret_cast<uint32_t*>(ws);
+      for (int stg = 0; stg < 3; ++stg) {
+        L.stage = stg;
+        L.total_tiles = total[stg];
+        L.out_kind = (stg == kStageApply && it == k - 1) ? (int)out_mode : (int)kOutIterate;
+        e = launch_ns_gemm(L, s);
+        if (e != cudaSuccess) return SIGNMUON_ERR_CUDA;
+      }
+    }
+  }
+  return SIGNMUON_OK;
+}
+
+// ------------------------------------------------------------------ sign pack
+signmuon_status signmuon_sign_pack(signmuon_shape shape, signmuon_dtype u_dtype, const void* u, int64_t ld_u,
+                                   int int8_out, void* out, void* stream) {
+  if (shape.rows <= 0 || shape.cols <= 0 || !u || !out || ld_u < shape.cols) return SIGNMUON_ERR_INVALID_ARG;
+  if (u_dtype != SIGNMUON_F32 && u_dtype != SIGNMUON_BF16) return SIGNMUON_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(out)) return SIGNMUON_ERR_ALIGNMENT;
+  return cuda_status(launch_sign_pack(shape, u_dtype == SIGNMUON_BF16, u, ld_u, int8_out != 0, out,
+                                      packed_words_of(shape), static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------------------ vote
+size_t signmuon_vote_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers) {
+  if (validate_shapes(shapes, n_mats) != SIGNMUON_OK || n_workers <= 0) return 0;
+  return kWsHeaderBytes + align_up((size_t)n_mats * sizeof(VoteMat), 256) +
+         align_up((size_t)n_mats * n_workers * sizeof(void*), 256);
+}
+
+signmuon_status signmuon_vote_update(const signmuon_shape* shapes, int n_mats, int n_workers, int int8_in,
+                                     const void* const* signs, signmuon_dtype w_dtype, void* const* w, float eta,
+                                     void* const* vote_bf16, int64_t* nnz, float* vote_inv_norm, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  signmuon_status st = validate_shapes(shapes, n_mats);
+  if (st) return st;
+  if (n_workers <= 0 || n_workers > SIGNMUON_MAX_WORKERS) return SIGNMUON_ERR_INVALID_ARG;
+  if (w_dtype != SIGNMUON_F32 && w_dtype != SIGNMUON_BF16) return SIGNMUON_ERR_INVALID_ARG;
+  const int units = n_mats * n_workers;
+  if ((st = validate_ptrs(signs, units))) return st;
+  const bool vote_out = vote_bf16 != nullptr;
+  if (vote_out) {
+    if ((st = validate_ptrs(vote_bf16, n_mats))) return st;
+    if (!nnz || !vote_inv_norm) return SIGNMUON_ERR_INVALID_ARG;
+    if (!aligned16(nnz) || !aligned16(vote_inv_norm)) return SIGNMUON_ERR_ALIGNMENT;
+  } else {
+    if ((st = validate_ptrs(w, n_mats))) return st;
+  }
+  if ((st = check_workspace(workspace, ws_bytes, signmuon_vote_workspace_bytes(shapes, n_mats, n_workers))))
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  std::vector<VoteMat> hm(n_mats);
+  int blocks = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    VoteMat& v = hm[i];
+    memset(&v, 0, sizeof(v));
+    v.w = vote_out ? nullptr : w[i];
+    v.vote = vote_out ? vote_bf16[i] : nullptr;
+    v.rows = shapes[i].rows;
+    v.cols = shapes[i].cols;
+    v.n = (int64_t)v.rows * v.cols;
+    v.wpr = (int32_t)wpr_of(v.cols);
+    v.n_words = (int64_t)v.rows * v.wpr;
+    v.ld_x = x_ld_of(v.cols);
+    v.block_begin = blocks;
+    v.block_count = vote_blocks_for(int8_in != 0, v.cols, v.n, v.n_words);
+    v.sign_ptr_offset = i * n_workers;
+    blocks += v.block_count;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  VoteMat* d_mats = reinterpret_cast<VoteMat*>(ws + kWsHeaderBytes);
+  const void** d_table =
+      reinterpret_cast<const void**>(ws + kWsHeaderBytes + align_up((size_t)n_mats * sizeof(VoteMat), 256));
+  cudaError_t e = upload_bytes(d_mats, hm.data(), hm.size() * sizeof(VoteMat), s);
+  if (e == cudaSuccess) e = upload_bytes(d_table, signs, (size_t)units * sizeof(void*), s);
+  if (e == cudaSuccess && vote_out) e = cudaMemsetAsync(nnz, 0, (size_t)n_mats * sizeof(int64_t), s);
+  if (e == cudaSuccess)
+    e = launch_vote(d_mats, n_mats, blocks, d_table, n_workers, int8_in != 0, w_dtype == SIGNMUON_BF16, eta,
+                    vote_out, reinterpret_cast<unsigned long long*>(nnz), s);
+  if (e == cudaSuccess && vote_out) e = launch_vote_inv(nnz, vote_inv_norm, n_mats, s);
+  return cuda_status(e);
+}
+
+}  // extern "C"

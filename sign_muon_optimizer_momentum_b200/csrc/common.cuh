@@ -1,0 +1,147 @@
+// Internal definitions shared by the kernels and the C-ABI layer of
+// libsignmuon.so.  Not part of the public interface (see include/signmuon.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "signmuon.h"
+
+namespace signmuon {
+
+// ---------------------------------------------------------------------------
+// Device error codes recorded in the first word of a workspace.
+// ---------------------------------------------------------------------------
+enum DeviceError : uint32_t {
+  kErrNone = 0,
+  kErrWaitTimeoutProducer = 0x101,  // TMA producer gave up waiting for a free stage
+  kErrWaitTimeoutMma = 0x102,       // MMA issuer gave up waiting for data / accumulator
+  kErrWaitTimeoutEpilogue = 0x103,  // epilogue gave up waiting for an accumulator
+  kErrWaitTimeoutDrain = 0x104,     // exit-time wait for in-flight copies ran out
+};
+
+// Workspace header: error word + padding.  Every workspace starts with it.
+constexpr size_t kWsHeaderBytes = 256;
+
+// Bounded waits: give up after this many nanoseconds of device time.
+constexpr uint64_t kWaitTimeoutNs = 2000ull * 1000ull * 1000ull;  // 2 s
+
+// ---------------------------------------------------------------------------
+// Newton-Schulz GEMM tiling (tcgen05, one CTA per tile, cta_group::1).
+// ---------------------------------------------------------------------------
+constexpr int kBM = 128;          // MMA M (TMEM lanes)
+constexpr int kBN = 256;          // MMA N (TMEM fp32 columns per accumulator)
+constexpr int kBK = 64;           // K per stage: 64 bf16 = 128 B = one swizzle row
+constexpr int kUmmaK = 16;        // K per tcgen05.mma for kind::f16
+constexpr int kStages = 4;
+constexpr int kBoxRows = 64;      // every TMA box is 64 x 64 bf16 (8 KB)
+constexpr int kBoxBytes = 64 * 64 * 2;
+constexpr int kAStageBytes = kBM * kBK * 2;               // 16 KB
+constexpr int kBStageBytes = kBN * kBK * 2;               // 32 KB
+constexpr int kStageBytes = kAStageBytes + kBStageBytes;  // 48 KB
+constexpr int kAccCols = kBN;                             // fp32 columns per accumulator
+constexpr int kTmemCols = 2 * kAccCols;                   // double-buffered: 512
+constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+enum NsStage : int { kStageGram = 0, kStageSquare = 1, kStageApply = 2 };
+
+// Final-iteration output kinds (mirror signmuon_ns_out) and the bf16 iterate.
+enum NsOut : int {
+  kOutPack1 = SIGNMUON_OUT_PACK1,
+  kOutInt8 = SIGNMUON_OUT_INT8,
+  kOutUpdateW = SIGNMUON_OUT_UPDATE_W,
+  kOutUF32 = SIGNMUON_OUT_U_F32,
+  kOutIterate = 100,
+};
+
+// One (matrix, worker) unit of a Newton-Schulz launch.  Tensor maps first so
+// they stay 64-byte aligned (the struct is 64-byte aligned and a multiple
+// of 64 bytes long).
+struct alignas(64) NsUnit {
+  CUtensorMap map_x;     // caller's bf16 X buffer  [rows, ld_x]
+  CUtensorMap map_xalt;  // workspace bf16 X buffer [rows, ld_x]
+  CUtensorMap map_a;     // workspace Gram A        [s, ld_s]
+  CUtensorMap map_b;     // workspace polynomial B  [s, ld_s]
+  __nv_bfloat16* x;
+  __nv_bfloat16* xalt;
+  __nv_bfloat16* a;
+  __nv_bfloat16* b;
+  void* out;             // final output (packed / int8 / fp32 U / W)
+  const float* scale;    // &inv_norm[u]
+  int32_t rows, cols, ld_x, ld_s;
+  int32_t tile_begin[3];  // prefix of tiles over the launch's units, per stage
+  int32_t tile_count[3];
+  int32_t pad_[4];
+};
+static_assert(sizeof(NsUnit) % 64 == 0, "NsUnit must keep 64-byte alignment");
+
+struct NsLaunch {
+  const NsUnit* units;
+  int n_units;
+  int stage;        // NsStage
+  int parity;       // 0: X_in = x, X_out = xalt; 1: the reverse
+  int first;        // scale X by *unit.scale (iteration 0)
+  int out_kind;     // NsOut: kOutIterate for non-final APPLY
+  int w_dtype;      // for kOutUpdateW
+  int total_tiles;
+  float a, b, c, eta;
+  uint32_t* err;
+};
+
+// Momentum units.
+struct MomUnit {
+  const void* grad;
+  float* mom;
+  __nv_bfloat16* x;
+  int64_t n;          // rows * cols
+  int32_t rows, cols, ld_x;
+  int32_t block_begin;  // first block of this unit in the flattened grid
+  int32_t block_count;
+  int32_t pad_;
+};
+
+// Vote matrices.
+struct VoteMat {
+  void* w;
+  void* vote;          // bf16 vote-out buffer or null
+  int64_t n;           // rows * cols
+  int64_t n_words;     // rows * ceil(cols/32) (packed) -- logical words
+  int32_t rows, cols, wpr, ld_x;
+  int32_t block_begin, block_count;
+  int32_t sign_ptr_offset;  // index into the sign pointer table (i * n_workers)
+  int32_t pad_;
+};
+
+static_assert(sizeof(NsUnit) == 640, "descriptor size is part of the launch-count bookkeeping");
+static_assert(sizeof(MomUnit) == 56, "descriptor size is part of the launch-count bookkeeping");
+static_assert(sizeof(VoteMat) == 64, "descriptor size is part of the launch-count bookkeeping");
+
+// ---------------------------------------------------------------------------
+// Launch helpers implemented in the .cu files (all enqueue on `stream`).
+// ---------------------------------------------------------------------------
+cudaError_t upload_bytes(void* dst_device, const void* src_host, size_t bytes, cudaStream_t stream);
+cudaError_t launch_momentum(const MomUnit* units, int n_units, int total_blocks, int grad_bf16,
+                            float beta, float* partials, cudaStream_t stream);
+cudaError_t launch_momentum_finalize(const MomUnit* units, int n_units, const float* partials,
+                                     float* inv_norm, cudaStream_t stream);
+cudaError_t launch_sign_pack(signmuon_shape shape, int u_bf16, const void* u, int64_t ld_u,
+                             int int8_out, void* out, int64_t out_words, cudaStream_t stream);
+cudaError_t launch_vote(const VoteMat* mats, int n_mats, int total_blocks, const void* const* sign_table,
+                        int n_workers, int int8_in, int w_bf16, float eta, int vote_out,
+                        unsigned long long* nnz, cudaStream_t stream);
+cudaError_t launch_vote_inv(const int64_t* nnz, float* inv, int n_mats, cudaStream_t stream);
+int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words);
+cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream);
+cudaError_t launch_ns_identity(const NsUnit* units, int n_units, int64_t max_elems, int out_kind,
+                               int w_dtype, float eta, cudaStream_t stream);
+
+// Block-count helpers shared by host planning and kernels.
+constexpr int kMomThreads = 256;
+constexpr int kMomElemsPerThread = 16;
+constexpr int kMomElemsPerBlock = kMomThreads * kMomElemsPerThread;  // 4096
+constexpr int kVoteThreads = 256;
+
+}  // namespace signmuon

@@ -1,0 +1,636 @@
+// HBM-bound kernels of the Sign-Muon step on sm_100a:
+//   * descriptor upload (kernel-parameter copy, fully asynchronous);
+//   * momentum + bf16 cast + Frobenius sum of squares (step 1 of the
+//     SignMuon summary's "Algorithmic flow"), with a fixed-order reduction;
+//   * standalone sign / 1-bit pack (steps 2-3);
+//   * majority vote over M sign buffers fused with W <- W - eta * vote
+//     (steps 3-4), or writing the vote matrix for the local polar step (5);
+//   * the k = 0 Newton-Schulz output path (U = X0).
+#include <cstring>
+
+#include "common.cuh"
+
+namespace signmuon {
+
+// ---------------------------------------------------------------------------
+// Descriptor upload: the host's descriptor blob travels as a kernel
+// parameter (up to ~32 KB per launch), so no pinned staging buffer and no
+// host synchronisation are needed.
+// ---------------------------------------------------------------------------
+constexpr int kUploadChunk = 32768 - 512;
+struct UploadChunk {
+  uint8_t* dst;
+  uint32_t n;
+  uint32_t pad_;
+  alignas(16) uint8_t data[kUploadChunk];
+};
+
+__global__ void __launch_bounds__(256) upload_kernel(const __grid_constant__ UploadChunk c) {
+  const uint32_t n16 = c.n / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(c.data);
+  uint4* dst = reinterpret_cast<uint4*>(c.dst);
+  for (uint32_t i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
+  for (uint32_t i = n16 * 16 + threadIdx.x; i < c.n; i += blockDim.x) c.dst[i] = c.data[i];
+}
+
+cudaError_t upload_bytes(void* dst_device, const void* src_host, size_t bytes,
+                         cudaStream_t stream) {
+  // dst must be 16-byte aligned (all workspace regions are 256-byte aligned).
+  static thread_local UploadChunk chunk;
+  const uint8_t* src = static_cast<const uint8_t*>(src_host);
+  uint8_t* dst = static_cast<uint8_t*>(dst_device);
+  for (size_t off = 0; off < bytes; off += kUploadChunk) {
+    const size_t n = bytes - off < (size_t)kUploadChunk ? bytes - off : (size_t)kUploadChunk;
+    chunk.dst = dst + off;
+    chunk.n = (uint32_t)n;
+    memcpy(chunk.data, src + off, n);
+    upload_kernel<<<1, 256, 0, stream>>>(chunk);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// Momentum
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int find_block_unit(const MomUnit* units, int n_units, int b) {
+  int lo = 0, hi = n_units - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (units[mid].block_begin <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ float load_grad(const void* g, int64_t i, int bf16) {
+  if (bf16) return __bfloat162float(static_cast<const __nv_bfloat16*>(g)[i]);
+  return static_cast<const float*>(g)[i];
+}
+
+// M <- beta*M + (1-beta)*G.  Both products are exact in fp64 (24-bit x 24-bit
+// significands), so the fp64 sum is rounded once and then once more to fp32.
+__device__ __forceinline__ float momentum_one(float m, float g, double beta, double omb) {
+  return (float)fma(beta, (double)m, omb * (double)g);
+}
+
+__global__ void __launch_bounds__(kMomThreads)
+momentum_kernel(const MomUnit* __restrict__ units, int n_units, int grad_bf16, float beta_f,
+                float* __restrict__ partials) {
+  const int b = blockIdx.x;
+  const int ui = find_block_unit(units, n_units, b);
+  const MomUnit u = units[ui];
+  const int lb = b - u.block_begin;
+  const double beta = (double)beta_f;
+  const double omb = 1.0 - beta;
+  const int64_t base = (int64_t)lb * kMomElemsPerBlock;
+  float ssq = 0.f;
+  const bool dense = (u.cols % 8) == 0;  // then ld_x == cols
+#pragma unroll
+  for (int it = 0; it < kMomElemsPerThread / 8; ++it) {
+    const int64_t e0 = base + (int64_t)it * (kMomThreads * 8) + threadIdx.x * 8;
+    if (e0 >= u.n) break;
+    float g[8], m[8];
+    if (e0 + 8 <= u.n) {
+      if (grad_bf16) {
+        const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(u.grad) + e0);
+        const __nv_bfloat162* gp = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(gp[j]);
+          g[2 * j] = f.x;
+          g[2 * j + 1] = f.y;
+        }
+      } else {
+        const float4 g0 = *reinterpret_cast<const float4*>(static_cast<const float*>(u.grad) + e0);
+        const float4 g1 = *reinterpret_cast<const float4*>(static_cast<const float*>(u.grad) + e0 + 4);
+        g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
+        g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+      }
+      const float4 m0 = *reinterpret_cast<const float4*>(u.mom + e0);
+      const float4 m1 = *reinterpret_cast<const float4*>(u.mom + e0 + 4);
+      m[0] = m0.x; m[1] = m0.y; m[2] = m0.z; m[3] = m0.w;
+      m[4] = m1.x; m[5] = m1.y; m[6] = m1.z; m[7] = m1.w;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        m[j] = momentum_one(m[j], g[j], beta, omb);
+        ssq = fmaf(m[j], m[j], ssq);
+      }
+      *reinterpret_cast<float4*>(u.mom + e0) = make_float4(m[0], m[1], m[2], m[3]);
+      *reinterpret_cast<float4*>(u.mom + e0 + 4) = make_float4(m[4], m[5], m[6], m[7]);
+      if (dense) {
+        __nv_bfloat162 xb[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xb[j] = __floats2bfloat162_rn(m[2 * j], m[2 * j + 1]);
+        *reinterpret_cast<uint4*>(u.x + e0) = *reinterpret_cast<const uint4*>(xb);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int64_t e = e0 + j;
+          const int64_t r = e / u.cols, c = e - r * u.cols;
+          u.x[r * u.ld_x + c] = __float2bfloat16_rn(m[j]);
+        }
+      }
+    } else {
+      for (int j = 0; j < 8; ++j) {
+        const int64_t e = e0 + j;
+        if (e >= u.n) break;
+        const float mj = momentum_one(u.mom[e], load_grad(u.grad, e, grad_bf16), beta, omb);
+        u.mom[e] = mj;
+        ssq = fmaf(mj, mj, ssq);
+        const int64_t r = e / u.cols, c = e - r * u.cols;
+        u.x[r * u.ld_x + c] = __float2bfloat16_rn(mj);
+      }
+    }
+  }
+  // Fixed-order block reduction: warp shuffles, then warp 0 over the warps.
+  __shared__ float red[kMomThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ssq;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < kMomThreads / 32 ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) partials[b] = v;
+  }
+}
+
+// inv_norm[u] = 1 / (sqrt(sum of the unit's partials) + 1e-7), partials summed
+// in fp64 in a fixed order.
+__global__ void __launch_bounds__(256)
+momentum_finalize_kernel(const MomUnit* __restrict__ units, const float* __restrict__ partials,
+                         float* __restrict__ inv_norm) {
+  const MomUnit u = units[blockIdx.x];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < u.block_count; i += blockDim.x) s += (double)partials[u.block_begin + i];
+  __shared__ double red[256];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) inv_norm[blockIdx.x] = (float)(1.0 / (sqrt(red[0]) + 1e-7));
+}
+
+cudaError_t launch_momentum(const MomUnit* units, int n_units, int total_blocks, int grad_bf16,
+                            float beta, float* partials, cudaStream_t stream) {
+  if (total_blocks <= 0) return cudaSuccess;
+  momentum_kernel<<<total_blocks, kMomThreads, 0, stream>>>(units, n_units, grad_bf16, beta, partials);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_momentum_finalize(const MomUnit* units, int n_units, const float* partials,
+                                     float* inv_norm, cudaStream_t stream) {
+  momentum_finalize_kernel<<<n_units, 256, 0, stream>>>(units, partials, inv_norm);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Standalone sign + pack
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float load_u(const void* u, int64_t i, int bf16) {
+  if (bf16) return __bfloat162float(static_cast<const __nv_bfloat16*>(u)[i]);
+  return static_cast<const float*>(u)[i];
+}
+
+// One warp per 32-column word: lane j tests entry (r, 32w + j); the ballot is
+// the packed word (bit j <-> column 32w + j, set bit <-> +1, pad bits 0).
+__global__ void __launch_bounds__(256)
+sign_pack_kernel(int rows, int cols, int u_bf16, const void* __restrict__ u, int64_t ld_u,
+                 uint32_t* __restrict__ out, int64_t out_words) {
+  const int wpr = (cols + 31) >> 5;
+  const int64_t n_words = (int64_t)rows * wpr;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t w = warp; w < out_words; w += n_warps) {
+    uint32_t word = 0;
+    if (w < n_words) {
+      const int64_t r = w / wpr;
+      const int c = (int)(w - r * wpr) * 32 + lane;
+      bool bit = false;
+      if (c < cols) bit = !(load_u(u, r * ld_u + c, u_bf16) < 0.f);
+      word = __ballot_sync(0xffffffffu, bit);
+    }
+    if (lane == 0) out[w] = word;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+sign_int8_kernel(int rows, int cols, int u_bf16, const void* __restrict__ u, int64_t ld_u,
+                 int8_t* __restrict__ out) {
+  const int64_t n = (int64_t)rows * cols;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / cols, c = e - r * cols;
+    out[e] = (load_u(u, r * ld_u + c, u_bf16) < 0.f) ? int8_t(-1) : int8_t(1);
+  }
+}
+
+static int grid_for(int64_t work, int per_block, int cap = 148 * 32) {
+  int64_t g = (work + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return (int)g;
+}
+
+cudaError_t launch_sign_pack(signmuon_shape shape, int u_bf16, const void* u, int64_t ld_u,
+                             int int8_out, void* out, int64_t out_words, cudaStream_t stream) {
+  if (int8_out) {
+    sign_int8_kernel<<<grid_for((int64_t)shape.rows * shape.cols, 256), 256, 0, stream>>>(
+        shape.rows, shape.cols, u_bf16, u, ld_u, static_cast<int8_t*>(out));
+  } else {
+    sign_pack_kernel<<<grid_for(out_words, 8), 256, 0, stream>>>(
+        shape.rows, shape.cols, u_bf16, u, ld_u, static_cast<uint32_t*>(out), out_words);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Majority vote + update
+// ---------------------------------------------------------------------------
+// Bit-sliced vertical counter: bit j of plane p is bit p of the number of
+// workers whose sign at bit position j is +1.  Seven planes count to 127.
+struct BitCount {
+  uint32_t p[7];
+};
+
+__device__ __forceinline__ void csa(uint32_t& carry, uint32_t& sum, uint32_t a, uint32_t b,
+                                    uint32_t c) {
+  const uint32_t u = a ^ b;
+  carry = (a & b) | (u & c);
+  sum = u ^ c;
+}
+
+__device__ __forceinline__ void ripple(BitCount& bc, uint32_t x, int from) {
+#pragma unroll
+  for (int p = 0; p < 7; ++p) {
+    if (p < from) continue;
+    const uint32_t t = bc.p[p] & x;
+    bc.p[p] ^= x;
+    x = t;
+  }
+}
+
+// Vote masks from the counts: gt = (2c > M), tie = (2c == M).
+__device__ __forceinline__ void vote_masks(const BitCount& bc, int m, uint32_t& gt, uint32_t& tie) {
+  const int t = m >> 1;
+  uint32_t g = 0, eq = 0xffffffffu;
+#pragma unroll
+  for (int p = 6; p >= 0; --p) {
+    const uint32_t tb = ((t >> p) & 1) ? 0xffffffffu : 0u;
+    g |= eq & bc.p[p] & ~tb;
+    eq &= ~(bc.p[p] ^ tb);
+  }
+  gt = g;
+  tie = (m & 1) ? 0u : eq;
+}
+
+// W - eta*v for fp32 W: one correctly rounded subtraction (v in {-1,0,1}).
+__device__ __forceinline__ float upd_f32(float w, float eta, int v) {
+  return v == 0 ? w : (v > 0 ? w - eta : w + eta);
+}
+
+// W - eta*v for bf16 W with a single rounding: the difference is exact in
+// fp64; it is rounded to fp32 with round-to-odd (truncate, then force the
+// last bit if anything was dropped) and then to bf16 with round-to-nearest-
+// even.  Round-to-odd at 24 bits followed by rounding to 8 bits equals the
+// direct rounding because 24 >= 8 + 2.
+__device__ __forceinline__ __nv_bfloat16 upd_bf16(__nv_bfloat16 wb, float eta, int v) {
+  if (v == 0) return wb;
+  const double d = (double)__bfloat162float(wb) - (v > 0 ? (double)eta : -(double)eta);
+  float r = __double2float_rz(d);
+  if ((double)r != d) r = __uint_as_float(__float_as_uint(r) | 1u);
+  return __float2bfloat16_rn(r);
+}
+
+__device__ __forceinline__ int vote_of(uint32_t gt, uint32_t tie, int j) {
+  return ((gt >> j) & 1) ? 1 : (((tie >> j) & 1) ? 0 : -1);
+}
+
+__device__ __forceinline__ int find_vote_mat(const VoteMat* mats, int n, int b) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (mats[mid].block_begin <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Packed fast path (cols % 32 == 0): packed word w covers W[32w, 32w+32).
+// Each thread counts 4 consecutive words (one 16-byte load per worker); a
+// warp covers 128 words = 4096 weights, which it then updates with
+// coalesced vector accesses, fetching the masks by shuffle.
+constexpr int kVoteWordsPerThread = 4;
+constexpr int kVoteWordsPerBlock = kVoteThreads * kVoteWordsPerThread;  // 1024
+constexpr int kVoteInt8PerThread = 16;
+constexpr int kVoteInt8PerBlock = kVoteThreads * kVoteInt8PerThread;   // 4096
+constexpr int kVoteGeneralWordsPerBlock = kVoteThreads;
+
+template <typename Count>
+__device__ __forceinline__ void count_words(const void* const* __restrict__ tab, int m_workers,
+                                            int64_t q, BitCount (&bc)[4], Count) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int p = 0; p < 7; ++p) bc[k].p[p] = 0;
+  int m = 0;
+  for (; m + 8 <= m_workers; m += 8) {
+    uint4 x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = __ldg(static_cast<const uint4*>(tab[m + j]) + q);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      auto comp = [&](int j) -> uint32_t {
+        return k == 0 ? x[j].x : (k == 1 ? x[j].y : (k == 2 ? x[j].z : x[j].w));
+      };
+      uint32_t t2a, t2b, t4a, t4b, t8;
+      csa(t2a, bc[k].p[0], bc[k].p[0], comp(0), comp(1));
+      csa(t2b, bc[k].p[0], bc[k].p[0], comp(2), comp(3));
+      csa(t4a, bc[k].p[1], bc[k].p[1], t2a, t2b);
+      csa(t2a, bc[k].p[0], bc[k].p[0], comp(4), comp(5));
+      csa(t2b, bc[k].p[0], bc[k].p[0], comp(6), comp(7));
+      csa(t4b, bc[k].p[1], bc[k].p[1], t2a, t2b);
+      csa(t8, bc[k].p[2], bc[k].p[2], t4a, t4b);
+      ripple(bc[k], t8, 3);
+    }
+  }
+  for (; m < m_workers; ++m) {
+    const uint4 x = __ldg(static_cast<const uint4*>(tab[m]) + q);
+    ripple(bc[0], x.x, 0);
+    ripple(bc[1], x.y, 0);
+    ripple(bc[2], x.z, 0);
+    ripple(bc[3], x.w, 0);
+  }
+}
+
+struct Dummy {};
+
+__device__ void vote_packed_fast(const VoteMat& mt, const void* const* __restrict__ tab, int m_workers,
+                                 int lb, int w_bf16, float eta, int vote_out,
+                                 unsigned long long* nnz_out) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  // Quad index (16-byte word group) handled by this thread.
+  const int64_t q = ((int64_t)lb * kVoteThreads + threadIdx.x);
+  const int64_t n_quads = (mt.n_words + 3) >> 2;
+  BitCount bc[4];
+  uint32_t gt[4] = {0, 0, 0, 0}, tie[4] = {0, 0, 0, 0};
+  if (q < n_quads) {
+    count_words(tab, m_workers, q, bc, Dummy{});
+#pragma unroll
+    for (int k = 0; k < 4; ++k) vote_masks(bc[k], m_workers, gt[k], tie[k]);
+  }
+  // The warp's 128 words cover weights [p0, p0 + 4096).
+  const int64_t warp_q0 = (int64_t)lb * kVoteThreads + warp * 32;
+  const int64_t p0 = warp_q0 * 128;
+  unsigned long long nz = 0;
+  // 4096 weights = 1024 groups of 4; 32 iterations of 32 lanes.
+#pragma unroll 4
+  for (int it = 0; it < 32; ++it) {
+    const int g4 = it * 32 + lane;          // group of 4 weights within the warp chunk
+    const int word = g4 >> 3;                // 0..127 within the warp chunk
+    const int src_lane = word >> 2;
+    const int comp = word & 3;
+    const uint32_t g0 = __shfl_sync(0xffffffffu, gt[0], src_lane);
+    const uint32_t g1 = __shfl_sync(0xffffffffu, gt[1], src_lane);
+    const uint32_t g2 = __shfl_sync(0xffffffffu, gt[2], src_lane);
+    const uint32_t g3 = __shfl_sync(0xffffffffu, gt[3], src_lane);
+    const uint32_t t0 = __shfl_sync(0xffffffffu, tie[0], src_lane);
+    const uint32_t t1 = __shfl_sync(0xffffffffu, tie[1], src_lane);
+    const uint32_t t2 = __shfl_sync(0xffffffffu, tie[2], src_lane);
+    const uint32_t t3 = __shfl_sync(0xffffffffu, tie[3], src_lane);
+    const uint32_t gw = comp == 0 ? g0 : (comp == 1 ? g1 : (comp == 2 ? g2 : g3));
+    const uint32_t tw = comp == 0 ? t0 : (comp == 1 ? t1 : (comp == 2 ? t2 : t3));
+    const int sh = (g4 & 7) * 4;
+    const int64_t p = p0 + (int64_t)g4 * 4;
+    if (p >= mt.n) continue;  // n is a multiple of 32, so a group is all-in or all-out
+    int v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = vote_of(gw, tw, sh + j);
+    if (vote_out) {
+      __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(mt.vote);
+      __nv_bfloat162 h[2];
+      h[0] = __floats2bfloat162_rn((float)v[0], (float)v[1]);
+      h[1] = __floats2bfloat162_rn((float)v[2], (float)v[3]);
+      *reinterpret_cast<uint2*>(vo + p) = *reinterpret_cast<const uint2*>(h);
+      nz += (v[0] != 0) + (v[1] != 0) + (v[2] != 0) + (v[3] != 0);
+    } else if (w_bf16) {
+      __nv_bfloat16* w = static_cast<__nv_bfloat16*>(mt.w);
+      uint2 raw = *reinterpret_cast<const uint2*>(w + p);
+      __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) e[j] = upd_bf16(e[j], eta, v[j]);
+      *reinterpret_cast<uint2*>(w + p) = raw;
+    } else {
+      float* w = static_cast<float*>(mt.w);
+      float4 x = *reinterpret_cast<const float4*>(w + p);
+      x.x = upd_f32(x.x, eta, v[0]);
+      x.y = upd_f32(x.y, eta, v[1]);
+      x.z = upd_f32(x.z, eta, v[2]);
+      x.w = upd_f32(x.w, eta, v[3]);
+      *reinterpret_cast<float4*>(w + p) = x;
+    }
+  }
+  if (vote_out) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xffffffffu, nz, o);
+    if (lane == 0 && nz) atomicAdd(nnz_out, nz);
+  }
+}
+
+// Packed general path (cols % 32 != 0): one thread per word, scalar W.
+__device__ void vote_packed_general(const VoteMat& mt, const void* const* __restrict__ tab,
+                                    int m_workers, int lb, int w_bf16, float eta, int vote_out,
+                                    unsigned long long* nnz_out) {
+  const int64_t w = (int64_t)lb * kVoteThreads + threadIdx.x;
+  unsigned long long nz = 0;
+  if (w < mt.n_words) {
+    BitCount bc;
+#pragma unroll
+    for (int p = 0; p < 7; ++p) bc.p[p] = 0;
+    for (int m = 0; m < m_workers; ++m) ripple(bc, __ldg(static_cast<const uint32_t*>(tab[m]) + w), 0);
+    uint32_t gt, tie;
+    vote_masks(bc, m_workers, gt, tie);
+    const int64_t r = w / mt.wpr;
+    const int c0 = (int)(w - r * mt.wpr) * 32;
+    const int nc = min(32, mt.cols - c0);
+    for (int j = 0; j < nc; ++j) {
+      const int v = vote_of(gt, tie, j);
+      const int64_t e = r * mt.cols + c0 + j;
+      if (vote_out) {
+        static_cast<__nv_bfloat16*>(mt.vote)[r * mt.ld_x + c0 + j] = __float2bfloat16_rn((float)v);
+        nz += (v != 0);
+      } else if (w_bf16) {
+        __nv_bfloat16* wp = static_cast<__nv_bfloat16*>(mt.w);
+        wp[e] = upd_bf16(wp[e], eta, v);
+      } else {
+        float* wp = static_cast<float*>(mt.w);
+        wp[e] = upd_f32(wp[e], eta, v);
+      }
+    }
+  }
+  if (vote_out) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xffffffffu, nz, o);
+    if ((threadIdx.x & 31) == 0 && nz) atomicAdd(nnz_out, nz);
+  }
+}
+
+// int8 path: 16 weights per thread; per-byte sums with SIMD byte adds
+// (|sum| <= M <= 127 fits a signed byte), vote = sign(sum).
+__device__ void vote_int8(const VoteMat& mt, const void* const* __restrict__ tab, int m_workers,
+                          int lb, int w_bf16, float eta, int vote_out,
+                          unsigned long long* nnz_out) {
+  const int64_t e0 = ((int64_t)lb * kVoteThreads + threadIdx.x) * kVoteInt8PerThread;
+  unsigned long long nz = 0;
+  if (e0 < mt.n) {
+    int v[16];
+    if (e0 + 16 <= mt.n) {
+      uint32_t acc[4] = {0, 0, 0, 0};
+      for (int m = 0; m < m_workers; ++m) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(tab[m]) + e0));
+        acc[0] = __vadd4(acc[0], x.x);
+        acc[1] = __vadd4(acc[1], x.y);
+        acc[2] = __vadd4(acc[2], x.z);
+        acc[3] = __vadd4(acc[3], x.w);
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int s = (int)(int8_t)((acc[j >> 2] >> ((j & 3) * 8)) & 0xff);
+        v[j] = (s > 0) - (s < 0);
+      }
+    } else {
+      for (int j = 0; j < 16; ++j) {
+        int s = 0;
+        if (e0 + j < mt.n)
+          for (int m = 0; m < m_workers; ++m) s += static_cast<const int8_t*>(tab[m])[e0 + j];
+        v[j] = (s > 0) - (s < 0);
+      }
+    }
+    const bool full = (e0 + 16 <= mt.n);
+    for (int j = 0; j < 16; ++j) {
+      const int64_t e = e0 + j;
+      if (!full && e >= mt.n) break;
+      if (vote_out) {
+        const int64_t r = e / mt.cols, c = e - r * mt.cols;
+        static_cast<__nv_bfloat16*>(mt.vote)[r * mt.ld_x + c] = __float2bfloat16_rn((float)v[j]);
+        nz += (v[j] != 0);
+      } else if (w_bf16) {
+        __nv_bfloat16* wp = static_cast<__nv_bfloat16*>(mt.w);
+        wp[e] = upd_bf16(wp[e], eta, v[j]);
+      } else {
+        float* wp = static_cast<float*>(mt.w);
+        wp[e] = upd_f32(wp[e], eta, v[j]);
+      }
+    }
+  }
+  if (vote_out) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xffffffffu, nz, o);
+    if ((threadIdx.x & 31) == 0 && nz) atomicAdd(nnz_out, nz);
+  }
+}
+
+__global__ void __launch_bounds__(kVoteThreads)
+vote_kernel(const VoteMat* __restrict__ mats, int n_mats, const void* const* __restrict__ table,
+            int n_workers, int int8_in, int w_bf16, float eta, int vote_out,
+            unsigned long long* __restrict__ nnz) {
+  const int b = blockIdx.x;
+  const int i = find_vote_mat(mats, n_mats, b);
+  const VoteMat mt = mats[i];
+  const int lb = b - mt.block_begin;
+  const void* const* tab = table + mt.sign_ptr_offset;
+  if (int8_in) {
+    vote_int8(mt, tab, n_workers, lb, w_bf16, eta, vote_out, nnz + i);
+  } else if ((mt.cols & 31) == 0) {
+    vote_packed_fast(mt, tab, n_workers, lb, w_bf16, eta, vote_out, nnz + i);
+  } else {
+    vote_packed_general(mt, tab, n_workers, lb, w_bf16, eta, vote_out, nnz + i);
+  }
+}
+
+__global__ void vote_inv_kernel(const int64_t* __restrict__ nnz, float* __restrict__ inv, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) inv[i] = nnz[i] > 0 ? (float)(1.0 / sqrt((double)nnz[i])) : 0.f;
+}
+
+cudaError_t launch_vote(const VoteMat* mats, int n_mats, int total_blocks, const void* const* sign_table,
+                        int n_workers, int int8_in, int w_bf16, float eta, int vote_out,
+                        unsigned long long* nnz, cudaStream_t stream) {
+  if (total_blocks <= 0) return cudaSuccess;
+  vote_kernel<<<total_blocks, kVoteThreads, 0, stream>>>(mats, n_mats, sign_table, n_workers, int8_in,
+                                                        w_bf16, eta, vote_out, nnz);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vote_inv(const int64_t* nnz, float* inv, int n_mats, cudaStream_t stream) {
+  vote_inv_kernel<<<(n_mats + 127) / 128, 128, 0, stream>>>(nnz, inv, n_mats);
+  return cudaGetLastError();
+}
+
+int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words) {
+  if (int8_in) return (int)((n + kVoteInt8PerBlock - 1) / kVoteInt8PerBlock);
+  if ((cols & 31) == 0) return (int)((((n_words + 3) >> 2) + kVoteThreads - 1) / kVoteThreads);
+  return (int)((n_words + kVoteGeneralWordsPerBlock - 1) / kVoteGeneralWordsPerBlock);
+}
+
+// ---------------------------------------------------------------------------
+// k = 0: the Newton-Schulz output is X0 itself.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+ns_identity_kernel(const NsUnit* __restrict__ units, int out_kind, int w_bf16, float eta) {
+  const NsUnit u = units[blockIdx.y];
+  const float s = *u.scale;
+  const int lane = threadIdx.x & 31;
+  if (out_kind == kOutPack1) {
+    const int wpr = (u.cols + 31) >> 5;
+    const int64_t n_words = (int64_t)u.rows * wpr;
+    const int64_t n_out = ((n_words + 3) / 4) * 4;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t w = warp; w < n_out; w += n_warps) {
+      uint32_t word = 0;
+      if (w < n_words) {
+        const int64_t r = w / wpr;
+        const int c = (int)(w - r * wpr) * 32 + lane;
+        bool bit = false;
+        if (c < u.cols) bit = !(s * __bfloat162float(u.x[r * u.ld_x + c]) < 0.f);
+        word = __ballot_sync(0xffffffffu, bit);
+      }
+      if (lane == 0) static_cast<uint32_t*>(u.out)[w] = word;
+    }
+    return;
+  }
+  const int64_t n = (int64_t)u.rows * u.cols;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / u.cols, c = e - r * u.cols;
+    const float v = s * __bfloat162float(u.x[r * u.ld_x + c]);
+    if (out_kind == kOutInt8) {
+      static_cast<int8_t*>(u.out)[e] = v < 0.f ? int8_t(-1) : int8_t(1);
+    } else if (out_kind == kOutUF32) {
+      static_cast<float*>(u.out)[e] = v;
+    } else {  // kOutUpdateW
+      if (w_bf16) {
+        __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u.out);
+        w[e] = __float2bfloat16_rn(__bfloat162float(w[e]) - eta * v);
+      } else {
+        float* w = static_cast<float*>(u.out);
+        w[e] = w[e] - eta * v;
+      }
+    }
+  }
+}
+
+cudaError_t launch_ns_identity(const NsUnit* units, int n_units, int64_t max_elems, int out_kind,
+                               int w_dtype, float eta, cudaStream_t stream) {
+  dim3 grid((unsigned)grid_for(max_elems, 256, 1024), (unsigned)n_units);
+  ns_identity_kernel<<<grid, 256, 0, stream>>>(units, out_kind, w_dtype == SIGNMUON_BF16, eta);
+  return cudaGetLastError();
+}
+
+}  // namespace signmuon

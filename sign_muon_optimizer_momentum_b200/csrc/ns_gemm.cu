@@ -1,0 +1,559 @@
+// Newton-Schulz GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One persistent, warp-specialised kernel runs one of the three products of
+// a Newton-Schulz iteration (SignMuon summary, section 2 "Core mechanism"
+// item 1: the momentum is orthogonalised toward its polar factor) over every
+// (matrix, worker) unit of a launch:
+//   stage Gram:   A = X X^T            (X^T X for tall X), symmetric output
+//   stage Square: B = b A + c A A      (A symmetric, so A A = A A^T)
+//   stage Apply:  X' = a X + B X       (X B for tall X)
+// with, in the last iteration, the entrywise sign fused into the epilogue and
+// written as packed bits or int8 (steps 2-3 of the summary's flow), or the
+// update W <- W - eta U (the optional local polar step, step 5).
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0     TMA producer: 64x64 bf16 boxes, 128-byte swizzle, 4 stages
+//   warp 1     MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128 N=256
+//              K=16, fp32 accumulators in TMEM, double-buffered (2 x 256 cols)
+//   warps 2-5  epilogue: tcgen05.ld 32x32b, fp32 math, stores
+// Every mbarrier wait is bounded; on timeout the kernel records an error
+// code, lets the other roles drain, waits (bounded) for its own copies and
+// MMAs, frees TMEM and returns.
+#include "common.cuh"
+
+namespace signmuon {
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase of `bar` with the given parity to complete.  Returns
+// false if it did not within kWaitTimeoutNs, or if another role has already
+// given up (abort flag set).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_test(bar, parity)) return true;
+    if ((++n & 63) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tensormap_acquire(const CUtensorMap* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(
+                   reinterpret_cast<uint64_t>(map))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a 128-byte-swizzled bf16 operand.
+//   K-major:  rows of 64 K-elements (128 B), 8-row atoms of 1 KB stacked
+//             along M/N (stride-byte-offset 1 KB); the leading offset is
+//             unused for swizzled K-major layouts.
+//   MN-major: rows of 64 M/N-elements (128 B) along K, 8-row atoms of 1 KB
+//             stacked along K (stride-byte-offset 1 KB), 64-element M/N
+//             blocks 8 KB apart (leading-byte-offset 8 KB, one TMA box).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, int mn_major) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(mn_major ? (kBoxBytes >> 4) : 1) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;  // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: D fp32, A and B bf16, M = 128, N = 256.
+__device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Tile decoding (identical in all roles)
+// ---------------------------------------------------------------------------
+struct Tile {
+  const NsUnit* u;
+  int M, N, K;
+  int m0, n0;
+  int a_mn, b_mn, sym;
+  const CUtensorMap* ma;
+  const CUtensorMap* mb;
+};
+
+__device__ __forceinline__ Tile decode_tile(const NsLaunch& L, int t) {
+  int lo = 0, hi = L.n_units - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (L.units[mid].tile_begin[L.stage] <= t) lo = mid; else hi = mid - 1;
+  }
+  const NsUnit* u = &L.units[lo];
+  int li = t - u->tile_begin[L.stage];
+  const int rows = u->rows, cols = u->cols;
+  const bool tall = rows > cols;
+  const int s = tall ? cols : rows, l = tall ? rows : cols;
+  const CUtensorMap* xin = L.parity ? &u->map_xalt : &u->map_x;
+  Tile T;
+  T.u = u;
+  if (L.stage == kStageGram) {
+    T.M = s; T.N = s; T.K = l; T.sym = 1;
+    T.ma = xin; T.mb = xin; T.a_mn = tall; T.b_mn = tall;
+  } else if (L.stage == kStageSquare) {
+    T.M = s; T.N = s; T.K = s; T.sym = 1;
+    T.ma = &u->map_a; T.mb = &u->map_a; T.a_mn = 0; T.b_mn = 0;
+  } else if (!tall) {  // X' = a X + B X: A-op = B (K-major), B-op = X (MN-major)
+    T.M = rows; T.N = cols; T.K = s; T.sym = 0;
+    T.ma = &u->map_b; T.a_mn = 0; T.mb = xin; T.b_mn = 1;
+  } else {             // X' = a X + X B: A-op = X (K-major), B-op = B (symmetric)
+    T.M = rows; T.N = cols; T.K = s; T.sym = 0;
+    T.ma = xin; T.a_mn = 0; T.mb = &u->map_b; T.b_mn = 0;
+  }
+  const int tiles_n = (T.N + kBN - 1) / kBN;
+  int tm = 0, tn = 0;
+  if (T.sym) {
+    // Tiles entirely below the diagonal are skipped: row tile tm starts at
+    // column tile tm/2.
+    while (true) {
+      const int cnt = tiles_n - (tm >> 1);
+      if (li < cnt) { tn = (tm >> 1) + li; break; }
+      li -= cnt;
+      ++tm;
+    }
+  } else {
+    tm = li / tiles_n;
+    tn = li - tm * tiles_n;
+  }
+  T.m0 = tm * kBM;
+  T.n0 = tn * kBN;
+  return T;
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, bool vec, int nvalid, float (&v)[32]) {
+  if (vec) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(p + q * 8);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h[j]);
+        v[q * 8 + 2 * j] = f.x;
+        v[q * 8 + 2 * j + 1] = f.y;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = j < nvalid ? __bfloat162float(p[j]) : 0.f;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, bool vec, int nvalid, const float (&v)[32]) {
+  if (vec) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 h[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) h[j] = __floats2bfloat162_rn(v[q * 8 + 2 * j], v[q * 8 + 2 * j + 1]);
+      *reinterpret_cast<uint4*>(p + q * 8) = *reinterpret_cast<const uint4*>(h);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) p[j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ NsLaunch L) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Stage buffers must be 1 KB aligned for the 128-byte swizzle atoms.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* full_bar = bars;                   // [kStages]
+  uint64_t* empty_bar = bars + kStages;        // [kStages]
+  uint64_t* tfull_bar = bars + 2 * kStages;    // [2]
+  uint64_t* tempty_bar = bars + 2 * kStages + 2;  // [2]
+  uint64_t* drain_bar = bars + 2 * kStages + 4;   // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_addr(&full_bar[s]), 1);
+      mbar_init(smem_addr(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_addr(&tfull_bar[a]), 1);
+      mbar_init(smem_addr(&tempty_bar[a]), 128);
+    }
+    mbar_init(smem_addr(drain_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  uint32_t issued_kb = 0;  // producer: k-blocks issued (for the exit drain)
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const NsUnit* last_unit = nullptr;
+      bool ok = true;
+      for (int t = blockIdx.x; t < L.total_tiles && ok; t += gridDim.x) {
+        const Tile T = decode_tile(L, t);
+        if (T.u != last_unit) {
+          tensormap_acquire(T.ma);
+          tensormap_acquire(T.mb);
+          last_unit = T.u;
+        }
+        const int nkb = (T.K + kBK - 1) / kBK;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(smem_addr(&empty_bar[stage]), phase ^ 1, abort_flag)) {
+            atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutProducer);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_addr(&full_bar[stage]);
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          const uint32_t sa = smem_addr(smem + stage * kStageBytes);
+          const uint32_t sb = sa + kAStageBytes;
+          const int k0 = kb * kBK;
+#pragma unroll
+          for (int j = 0; j < kBM / kBoxRows; ++j) {
+            const int mn = T.m0 + j * kBoxRows;
+            tma_load_2d(sa + j * kBoxBytes, T.ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
+          }
+#pragma unroll
+          for (int j = 0; j < kBN / kBoxRows; ++j) {
+            const int mn = T.n0 + j * kBoxRows;
+            tma_load_2d(sb + j * kBoxBytes, T.mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
+          }
+          ++issued_kb;
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < L.total_tiles && ok; t += gridDim.x) {
+        const Tile T = decode_tile(L, t);
+        const uint32_t idesc = instr_desc(T.a_mn, T.b_mn);
+        const int nkb = (T.K + kBK - 1) / kBK;
+        if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag)) {
+          atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tmem_d = tmem_base + (uint32_t)(acc * kAccCols);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(smem_addr(&full_bar[stage]), phase, abort_flag)) {
+            atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(smem + stage * kStageBytes);
+          const uint32_t sb = sa + kAStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+            const uint32_t aoff = T.a_mn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
+            const uint32_t boff = T.b_mn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
+            tc_mma(tmem_d, smem_desc(sa + aoff, T.a_mn), smem_desc(sb + boff, T.b_mn), idesc,
+                   (kb | kk) != 0);
+          }
+          tc_commit(smem_addr(&empty_bar[stage]));  // stage free once these MMAs finish
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(smem_addr(&tfull_bar[acc]));  // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // Drain: wait until every MMA this thread issued has completed.
+      tc_commit(smem_addr(drain_bar));
+      if (!mbar_wait(smem_addr(drain_bar), 0, abort_flag)) {
+        // Ignore the abort flag for the drain itself: wait out the full limit.
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_test(smem_addr(drain_bar), 0)) {
+          if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+            atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutDrain);
+            break;
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < L.total_tiles; t += gridDim.x) {
+      const Tile T = decode_tile(L, t);
+      const NsUnit* u = T.u;
+      if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag)) {
+        atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutEpilogue);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int grow = T.m0 + row_in_tile;
+      const bool row_ok = grow < T.M;
+      const float s = L.first ? *u->scale : 1.f;
+      for (int ch = 0; ch < kBN / 32; ++ch) {
+        const int gc0 = T.n0 + ch * 32;
+        if (gc0 >= T.N) break;  // warp-uniform
+        uint32_t raw[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols + ch * 32), raw);
+        if (!row_ok) continue;
+        const int nvalid = min(32, T.N - gc0);
+        float v[32];
+        if (L.stage == kStageGram) {
+          const float s2 = s * s;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) * s2;
+        } else if (L.stage == kStageSquare) {
+          float av[32];
+          load_bf16x32(u->a + (int64_t)grow * u->ld_s + gc0, nvalid == 32, nvalid, av);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = fmaf(L.b, av[j], L.c * __uint_as_float(raw[j]));
+        } else {
+          const __nv_bfloat16* xin = L.parity ? u->xalt : u->x;
+          float xv[32];
+          load_bf16x32(xin + (int64_t)grow * u->ld_x + gc0, nvalid == 32, nvalid, xv);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = s * fmaf(L.a, xv[j], __uint_as_float(raw[j]));
+        }
+        if (T.sym) {
+          // Store the upper triangle (col >= row) and mirror it (col > row).
+          __nv_bfloat16* out = (L.stage == kStageGram) ? u->a : u->b;
+          const int ld = u->ld_s;
+          if (gc0 >= grow) {
+            store_bf16x32(out + (int64_t)grow * ld + gc0, nvalid == 32, nvalid, v);
+          } else if (gc0 + 31 >= grow) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid && gc0 + j >= grow) out[(int64_t)grow * ld + gc0 + j] = __float2bfloat16_rn(v[j]);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nvalid && gc0 + j > grow) out[(int64_t)(gc0 + j) * ld + grow] = __float2bfloat16_rn(v[j]);
+        } else if (L.out_kind == kOutIterate) {
+          __nv_bfloat16* xout = L.parity ? u->x : u->xalt;
+          store_bf16x32(xout + (int64_t)grow * u->ld_x + gc0, nvalid == 32, nvalid, v);
+        } else if (L.out_kind == kOutPack1) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) word |= (j < nvalid && !(v[j] < 0.f)) ? (1u << j) : 0u;
+          const int wpr = (u->cols + 31) >> 5;
+          static_cast<uint32_t*>(u->out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
+        } else if (L.out_kind == kOutInt8) {
+          int8_t* o = static_cast<int8_t*>(u->out) + (int64_t)grow * u->cols + gc0;
+          if (nvalid == 32 && (u->cols & 15) == 0) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+              uint32_t x = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) x |= (uint32_t)((v[4 * w + j] < 0.f) ? 0xFFu : 0x01u) << (8 * j);
+              pk[w] = x;
+            }
+            reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) o[j] = v[j] < 0.f ? int8_t(-1) : int8_t(1);
+          }
+        } else if (L.out_kind == kOutUF32) {
+          float* o = static_cast<float*>(u->out) + (int64_t)grow * u->cols + gc0;
+          if (nvalid == 32 && (u->cols & 3) == 0) {
+#pragma unroll
+            for (int w = 0; w < 8; ++w)
+              reinterpret_cast<float4*>(o)[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) o[j] = v[j];
+          }
+        } else {  // kOutUpdateW: W <- W - eta * U
+          const int64_t off = (int64_t)grow * u->cols + gc0;
+          if (L.w_dtype == SIGNMUON_BF16) {
+            __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u->out) + off;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) w[j] = __float2bfloat16_rn(fmaf(-L.eta, v[j], __bfloat162float(w[j])));
+          } else {
+            float* w = static_cast<float*>(u->out) + off;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_addr(&tempty_bar[acc]));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  // ------------------------------------------------------------------ exit
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0 && lane == 0) {
+    // Wait (bounded) for every TMA copy this CTA issued: the last phase armed
+    // on each stage's full barrier must have completed.
+    for (int s = 0; s < kStages; ++s) {
+      if (issued_kb <= (uint32_t)s) continue;
+      const uint32_t last_round = (issued_kb - 1 - s) / kStages;
+      const uint32_t bar = smem_addr(&full_bar[s]);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_test(bar, last_round & 1)) {
+        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+          atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutDrain);
+          break;
+        }
+      }
+    }
+  }
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+static int g_num_sms[64] = {0};
+
+cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
+  if (p.total_tiles <= 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+    if (e != cudaSuccess) return e;
+    g_num_sms[dev] = n;
+  }
+  const int grid = p.total_tiles < g_num_sms[dev] ? p.total_tiles : g_num_sms[dev];
+  ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace signmuon

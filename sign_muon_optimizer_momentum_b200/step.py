@@ -1,0 +1,203 @@
+"""SignMuonStep: one Sign-Muon optimizer step over M simulated workers.
+
+The step follows the SignMuon summary's "Algorithmic flow (distributed)"
+(section 2), with the M workers held as M gradient and momentum buffers on
+one GPU, so that the exchange of step 3 becomes the local M-way reduction of
+the vote kernel:
+
+  1. signmuon_momentum_norm          momentum, bf16 copy, Frobenius norm
+  2. signmuon_newton_schulz_batched  k iterations, sign fused into the last
+  3-4. signmuon_vote_update          majority vote + W <- W - eta * vote
+  5. (polar) vote matrix -> one Newton-Schulz iteration -> W update
+
+PyTorch is used only to allocate device buffers and to pick the stream; all
+arithmetic runs in libsignmuon.so.
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib as L
+
+NS_QUINTIC = (3.4445, -4.7750, 2.0315)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return L.SIGNMUON_F32
+    if dt == torch.bfloat16:
+        return L.SIGNMUON_BF16
+    raise TypeError(f"unsupported dtype {dt} (fp32 or bf16)")
+
+
+def _check_buf(t: torch.Tensor, shape, dtype, what: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{what}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{what}: expected a contiguous tensor of shape {tuple(shape)}")
+    p = t.data_ptr()
+    if p % 16:
+        raise ValueError(f"{what}: data pointer must be 16-byte aligned")
+    return p
+
+
+class SignMuonStep:
+    """Holds the optimizer state (one fp32 momentum buffer per worker and
+    matrix) and the scratch buffers of the step.
+
+    shapes:    list of (rows, cols) weight matrices
+    n_workers: M, the number of simulated data-parallel workers
+    k:         Newton-Schulz iterations
+    variant:   "pack1" (1-bit packed signs) or "int8" (integer-sum vote)
+    polar:     run the optional local polar step on the voted matrix
+    """
+
+    def __init__(self, shapes: Sequence[Tuple[int, int]], n_workers: int, k: int, variant: str,
+                 beta: float, eta: float, w_dtype: torch.dtype, polar: bool = False,
+                 coeffs=NS_QUINTIC, device: Optional[torch.device] = None,
+                 ns_workspace_cap: int = 16 << 30):
+        if variant not in ("pack1", "int8"):
+            raise ValueError("variant must be 'pack1' or 'int8'")
+        L.load()
+        self.shapes = [(int(r), int(c)) for r, c in shapes]
+        self.n_workers = int(n_workers)
+        self.k = int(k)
+        self.variant = variant
+        self.beta = float(beta)
+        self.eta = float(eta)
+        self.w_dtype = w_dtype
+        self.polar = bool(polar)
+        self.coeffs = tuple(float(x) for x in coeffs)
+        self.device = torch.device(device or "cuda")
+        dev = self.device
+        M = self.n_workers
+        self.units = len(self.shapes) * M
+        self.mom: List[torch.Tensor] = []
+        self.x: List[torch.Tensor] = []
+        self.signs: List[torch.Tensor] = []
+        for (r, c) in self.shapes:
+            for _ in range(M):
+                self.mom.append(torch.zeros((r, c), dtype=torch.float32, device=dev))
+                self.x.append(torch.empty((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device=dev))
+                if variant == "pack1":
+                    self.signs.append(torch.empty(L.signmuon_packed_words((r, c)), dtype=torch.int32,
+                                                  device=dev))
+                else:
+                    self.signs.append(torch.empty((r, c), dtype=torch.int8, device=dev))
+        self.inv_norm = torch.empty(self.units, dtype=torch.float32, device=dev)
+        self.ws_mom = torch.empty(L.signmuon_momentum_workspace_bytes(self.shapes, M), dtype=torch.uint8,
+                                  device=dev)
+        full = L.signmuon_newton_schulz_workspace_bytes(self.shapes, M)
+        minimal = L.signmuon_newton_schulz_workspace_bytes(self.shapes, M, minimal=True)
+        self.ws_ns = torch.empty(max(minimal, min(full, ns_workspace_cap)), dtype=torch.uint8, device=dev)
+        self.ws_vote = torch.empty(L.signmuon_vote_workspace_bytes(self.shapes, M), dtype=torch.uint8,
+                                   device=dev)
+        if self.polar:
+            self.vote = [torch.empty((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device=dev)
+                         for (r, c) in self.shapes]
+            n = len(self.shapes)
+            self.nnz = torch.zeros(max(n, 2), dtype=torch.int64, device=dev)
+            self.vote_inv = torch.zeros(max(n, 4), dtype=torch.float32, device=dev)
+            full1 = L.signmuon_newton_schulz_workspace_bytes(self.shapes, 1)
+            min1 = L.signmuon_newton_schulz_workspace_bytes(self.shapes, 1, minimal=True)
+            self.ws_polar = torch.empty(max(min1, min(full1, ns_workspace_cap)), dtype=torch.uint8,
+                                        device=dev)
+
+    # ------------------------------------------------------------------
+    def state_dict(self):
+        return {"mom": [m.clone() for m in self.mom]}
+
+    def load_state_dict(self, sd):
+        for dst, src in zip(self.mom, sd["mom"]):
+            dst.copy_(src)
+
+    # ------------------------------------------------------------------
+    def momentum_norm(self, grads: Sequence[torch.Tensor], stream: int) -> None:
+        gdt = self.w_dtype
+        gptr = []
+        for u, g in enumerate(grads):
+            r, c = self.shapes[u // self.n_workers]
+            gptr.append(_check_buf(g, (r, c), gdt, f"grad[{u}]"))
+        L.signmuon_momentum_norm(self.shapes, self.n_workers, _dtype_code(gdt), gptr,
+                                 [m.data_ptr() for m in self.mom], self.beta,
+                                 [x.data_ptr() for x in self.x], self.inv_norm.data_ptr(),
+                                 self.ws_mom.data_ptr(), self.ws_mom.numel(), stream)
+
+    def newton_schulz(self, stream: int, out_mode: Optional[int] = None, outs=None) -> None:
+        if out_mode is None:
+            out_mode = L.SIGNMUON_OUT_PACK1 if self.variant == "pack1" else L.SIGNMUON_OUT_INT8
+        outs = self.signs if outs is None else outs
+        a, b, c = self.coeffs
+        L.signmuon_newton_schulz_batched(self.shapes, self.n_workers, [x.data_ptr() for x in self.x],
+                                         self.inv_norm.data_ptr(), self.k, a, b, c, out_mode,
+                                         [o.data_ptr() for o in outs], L.SIGNMUON_F32, None, 0.0,
+                                         self.ws_ns.data_ptr(), self.ws_ns.numel(), stream)
+
+    def vote_update(self, weights: Sequence[torch.Tensor], stream: int) -> None:
+        wptr = [_check_buf(w, s, self.w_dtype, f"weight[{i}]")
+                for i, (w, s) in enumerate(zip(weights, self.shapes))]
+        sptr = [s.data_ptr() for s in self.signs]
+        int8_in = self.variant == "int8"
+        if not self.polar:
+            L.signmuon_vote_update(self.shapes, self.n_workers, int8_in, sptr, _dtype_code(self.w_dtype),
+                                   wptr, self.eta, None, 0, 0, self.ws_vote.data_ptr(),
+                                   self.ws_vote.numel(), stream)
+            return
+        L.signmuon_vote_update(self.shapes, self.n_workers, int8_in, sptr, _dtype_code(self.w_dtype),
+                               None, self.eta, [v.data_ptr() for v in self.vote], self.nnz.data_ptr(),
+                               self.vote_inv.data_ptr(), self.ws_vote.data_ptr(), self.ws_vote.numel(),
+                               stream)
+        a, b, c = self.coeffs
+        L.signmuon_newton_schulz_batched(self.shapes, 1, [v.data_ptr() for v in self.vote],
+                                         self.vote_inv.data_ptr(), 1, a, b, c, L.SIGNMUON_OUT_UPDATE_W,
+                                         None, _dtype_code(self.w_dtype), wptr, self.eta,
+                                         self.ws_polar.data_ptr(), self.ws_polar.numel(), stream)
+
+    def step(self, weights: Sequence[torch.Tensor], grads: Sequence[torch.Tensor]) -> None:
+        """One optimizer step: updates `weights` (one tensor per matrix) in place
+        from `grads` (n_mats * n_workers tensors, index i * n_workers + m)."""
+        if len(weights) != len(self.shapes) or len(grads) != self.units:
+            raise ValueError("expected one weight per matrix and one gradient per (matrix, worker)")
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        self.momentum_norm(grads, stream)
+        self.newton_schulz(stream)
+        self.vote_update(weights, stream)
+
+    def kernel_launches_per_step(self) -> int:
+        """Number of libsignmuon kernels one step enqueues (descriptor uploads included)."""
+        def uploads(nbytes):
+            return max(1, -(-nbytes // (32768 - 512)))
+        M = self.n_workers
+        n_mats = len(self.shapes)
+        mom = uploads(self.units * 56) + 2
+        unit_bytes = 640
+        ns_waves = self._waves(self.shapes, M, self.ws_ns.numel())
+        ns = uploads(self.units * unit_bytes) + (3 * self.k if self.k > 0 else 1) * ns_waves
+        vote = uploads(n_mats * 64) + uploads(self.units * 8) + 1
+        total = mom + ns + vote
+        if self.polar:
+            total += 1  # 1/sqrt(nnz) kernel (the nnz clear is a memset, not a kernel)
+            total += uploads(n_mats * unit_bytes) + 3 * self._waves(self.shapes, 1, self.ws_polar.numel())
+        return total
+
+    @staticmethod
+    def _waves(shapes, M, ws_bytes) -> int:
+        def al(x, a):
+            return (x + a - 1) // a * a
+        units = len(shapes) * M
+        arena = ws_bytes - 256 - al(units * 640, 1024)
+        waves, used = 0, arena
+        for (r, c) in shapes:
+            s = min(r, c)
+            lds = al(s, 8)
+            b = 2 * al(s * lds * 2, 1024) + al(r * al(c, 8) * 2, 1024)
+            for _ in range(M):
+                if used + b > arena:
+                    waves += 1
+                    used = 0
+                used += b
+        return waves

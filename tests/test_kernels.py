@@ -1,0 +1,480 @@
+"""GPU parity of the C-ABI kernels against the CPU oracle.
+
+Every case draws seeded synthetic inputs, runs them through libsignmuon.so
+(via the thin binding) and through the fp64 oracle, and compares:
+  * sign/pack, vote and update: bit-exact;
+  * momentum: bit-exact fp32 state, bf16 copy exact, norm to 1e-5 relative;
+  * Newton-Schulz: relative Frobenius error <= 2e-2 against the fp64 oracle
+    and sign agreement >= 99.5 % on entries with |U| > 1e-3.
+The oracle never consumes a GPU output: both sides start from the same
+seeded inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import signmuon_oracle as O
+from sign_muon_optimizer_momentum_b200 import _lib as L
+from sign_muon_optimizer_momentum_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+NS_TOL = 2e-2          # relative Frobenius error of U (bf16 operands, fp32 accumulation)
+SIGN_AGREE = 0.995     # on |U_oracle| > 1e-3
+A, B, C = O.NS_QUINTIC
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_lib):
+    return cuda_lib
+
+
+def stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def ws(nbytes):
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device="cuda")
+
+
+def assert_no_device_error(w):
+    assert L.signmuon_device_error(w.data_ptr(), stream()) == 0
+
+
+# ---------------------------------------------------------------------------
+# helpers running the GPU path
+# ---------------------------------------------------------------------------
+def gpu_momentum(shapes, M, grads, moms, beta, grad_dtype):
+    xs = [torch.empty((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device="cuda")
+          for (r, c) in shapes for _ in range(M)]
+    inv = torch.empty(len(shapes) * M, dtype=torch.float32, device="cuda")
+    w = ws(L.signmuon_momentum_workspace_bytes(shapes, M))
+    code = L.SIGNMUON_BF16 if grad_dtype == torch.bfloat16 else L.SIGNMUON_F32
+    L.signmuon_momentum_norm(shapes, M, code, [g.data_ptr() for g in grads], [m.data_ptr() for m in moms],
+                             beta, [x.data_ptr() for x in xs], inv.data_ptr(), w.data_ptr(), w.numel(),
+                             stream())
+    torch.cuda.synchronize()
+    assert_no_device_error(w)
+    return xs, inv
+
+
+def gpu_ns(shapes, M, xs, inv, k, out_mode, outs=None, w_dtype=L.SIGNMUON_F32, weights=None, eta=0.0,
+           minimal_ws=False):
+    nbytes = L.signmuon_newton_schulz_workspace_bytes(shapes, M, minimal=minimal_ws)
+    w = ws(nbytes)
+    L.signmuon_newton_schulz_batched(shapes, M, [x.data_ptr() for x in xs], inv.data_ptr(), k, A, B, C,
+                                     out_mode, None if outs is None else [o.data_ptr() for o in outs],
+                                     w_dtype, None if weights is None else [x.data_ptr() for x in weights],
+                                     eta, w.data_ptr(), w.numel(), stream())
+    torch.cuda.synchronize()
+    assert_no_device_error(w)
+
+
+def seeded_state(shapes, M, seed, grad_dtype=torch.float32, mom_std=1.0, g_std=2.0):
+    grads, moms = [], []
+    for i, s in enumerate(shapes):
+        for m in range(M):
+            grads.append(syn.gaussian(s, g_std, "cpu", "tg", seed, i, m, dtype=grad_dtype))
+            moms.append(syn.gaussian(s, mom_std, "cpu", "tm", seed, i, m))
+    return grads, moms
+
+
+def oracle_u(mom0, grad, beta, k):
+    m = O.momentum_update(f64(mom0), f64(grad), float(np.float32(beta)))
+    return m, O.newton_schulz(O.frobenius_normalize(m), k)
+
+
+def unpack_words(words, rows, cols):
+    """Decodes a packed sign buffer (bit j of word w in row r = entry (r, 32w+j))."""
+    wpr = (cols + 31) // 32
+    w = np.ascontiguousarray(words[: rows * wpr].reshape(rows, wpr).astype("<u4"))
+    bits = np.unpackbits(w.view(np.uint8), axis=1, bitorder="little")[:, :cols]
+    return np.where(bits == 1, 1, -1).astype(np.int8)
+
+
+def rel_fro(x, ref):
+    return np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-30)
+
+
+# ---------------------------------------------------------------------------
+# sign + pack
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(1, 1), (3, 31), (31, 33), (64, 147), (5, 96), (300, 1000), (129, 4096)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_sign_pack_bit_exact(shape, dtype):
+    u = syn.gaussian(shape, 1.0, "cpu", "u", *shape, dtype=dtype)
+    flat = u.view(-1)
+    flat[::7] = 0.0
+    flat[1::11] = -0.0
+    if dtype == torch.float32:
+        flat[2::13] = float("nan")
+    ud = u.cuda()
+    nwords = L.signmuon_packed_words(shape)
+    out = torch.full((nwords,), -1, dtype=torch.int32, device="cuda")
+    code = L.SIGNMUON_BF16 if dtype == torch.bfloat16 else L.SIGNMUON_F32
+    L.signmuon_sign_pack(shape, code, ud.data_ptr(), shape[1], 0, out.data_ptr(), stream())
+    o8 = torch.zeros(shape, dtype=torch.int8, device="cuda")
+    L.signmuon_sign_pack(shape, code, ud.data_ptr(), shape[1], 1, o8.data_ptr(), stream())
+    torch.cuda.synchronize()
+    s = O.sign_entries(f64(u))
+    ref = O.pack_signs(s).reshape(-1)
+    got = out.cpu().numpy().view(np.uint32)
+    assert np.array_equal(got[: ref.size], ref)
+    assert np.all(got[ref.size:] == 0)          # trailing pad words are zero
+    assert np.array_equal(o8.cpu().numpy(), s)
+
+
+def test_sign_pack_strided_input():
+    shape, ld = (17, 40), 56
+    u = syn.gaussian((shape[0], ld), 1.0, "cpu", "us")
+    out = torch.zeros(L.signmuon_packed_words(shape), dtype=torch.int32, device="cuda")
+    L.signmuon_sign_pack(shape, L.SIGNMUON_F32, u.cuda().data_ptr(), ld, 0, out.data_ptr(), stream())
+    torch.cuda.synchronize()
+    ref = O.pack_signs(O.sign_entries(f64(u)[:, :shape[1]])).reshape(-1)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32)[: ref.size], ref)
+
+
+# ---------------------------------------------------------------------------
+# vote + update
+# ---------------------------------------------------------------------------
+def _signs(shape, M, seed):
+    n = shape[0] * shape[1]
+    return [s.view(shape) for _, s in syn.vote_sweep_signs(n, M, seed=seed)]
+
+
+def _packed_device(s_list, shape):
+    outs = []
+    for s in s_list:
+        words = np.zeros(L.signmuon_packed_words(shape), dtype=np.uint32)
+        p = O.pack_signs(s.numpy())
+        words[: p.size] = p.reshape(-1)
+        outs.append(torch.from_numpy(words.view(np.int32)).cuda())
+    return outs
+
+
+VOTE_CASES = [((4, 32), 1), ((64, 64), 2), ((37, 96), 3), ((256, 256), 8), ((100, 1024), 16),
+              ((64, 4096), 64), ((33, 147), 5), ((31, 33), 4), ((2, 1000), 7), ((512, 1024), 64)]
+
+
+@pytest.mark.parametrize("shape,M", VOTE_CASES)
+@pytest.mark.parametrize("int8_in", [False, True])
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
+def test_vote_update_bit_exact(shape, M, int8_in, w_dtype):
+    s_list = _signs(shape, M, seed=M * 1000 + shape[0])
+    w0 = syn.gaussian(shape, 0.02, "cpu", "w", *shape, dtype=w_dtype)
+    eta = 0.01
+    if int8_in:
+        dev_signs = [s.cuda() for s in s_list]
+    else:
+        dev_signs = _packed_device(s_list, shape)
+    w = w0.cuda()
+    wk = ws(L.signmuon_vote_workspace_bytes([shape], M))
+    code = L.SIGNMUON_BF16 if w_dtype == torch.bfloat16 else L.SIGNMUON_F32
+    L.signmuon_vote_update([shape], M, int8_in, [s.data_ptr() for s in dev_signs], code, [w.data_ptr()], eta,
+                           None, 0, 0, wk.data_ptr(), wk.numel(), stream())
+    torch.cuda.synchronize()
+    v = O.majority_vote([s.numpy() for s in s_list])
+    ref = O.apply_update(f64(w0), eta, v, "bf16" if w_dtype == torch.bfloat16 else "f32")
+    assert np.array_equal(f64(w), ref)
+
+
+def test_vote_update_multi_matrix_and_vote_out():
+    shapes = [(64, 147), (128, 256), (33, 64), (7, 5)]
+    M = 6
+    all_signs = [_signs(s, M, seed=10 + i) for i, s in enumerate(shapes)]
+    for int8_in in (False, True):
+        flat = []
+        for s_list, shp in zip(all_signs, shapes):
+            flat += [x.cuda() for x in s_list] if int8_in else _packed_device(s_list, shp)
+        votes = [torch.full((r, L.signmuon_x_ld(c)), 7.0, dtype=torch.bfloat16, device="cuda") for r, c in shapes]
+        nnz = torch.full((4,), -5, dtype=torch.int64, device="cuda")
+        inv = torch.zeros(4, dtype=torch.float32, device="cuda")
+        wk = ws(L.signmuon_vote_workspace_bytes(shapes, M))
+        L.signmuon_vote_update(shapes, M, int8_in, [x.data_ptr() for x in flat], L.SIGNMUON_F32, None, 0.01,
+                               [v.data_ptr() for v in votes], nnz.data_ptr(), inv.data_ptr(), wk.data_ptr(),
+                               wk.numel(), stream())
+        torch.cuda.synchronize()
+        for i, (shp, s_list) in enumerate(zip(shapes, all_signs)):
+            ref = O.majority_vote([s.numpy() for s in s_list])
+            got = f64(votes[i])[:, : shp[1]]
+            assert np.array_equal(got, ref)
+            assert nnz[i].item() == np.count_nonzero(ref)
+            assert math.isclose(inv[i].item(), 1 / math.sqrt(np.count_nonzero(ref)), rel_tol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# momentum
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shapes,M", [([(256, 256)], 4), ([(64, 147), (1, 1), (7, 9)], 3),
+                                      ([(768, 2304), (3072, 768)], 2)])
+@pytest.mark.parametrize("grad_dtype", [torch.float32, torch.bfloat16])
+def test_momentum_norm_exact(shapes, M, grad_dtype):
+    beta = 0.9
+    grads, moms = seeded_state(shapes, M, 3, grad_dtype)
+    g_d = [g.cuda() for g in grads]
+    m_d = [m.cuda() for m in moms]
+    xs, inv = gpu_momentum(shapes, M, g_d, m_d, beta, grad_dtype)
+    for u in range(len(grads)):
+        r, c = shapes[u // M]
+        ref = O.momentum_update(f64(moms[u]), f64(grads[u]), float(np.float32(beta)))
+        got = f64(m_d[u])
+        assert np.array_equal(got, ref), np.max(np.abs(got - ref))
+        assert np.array_equal(f64(xs[u])[:, :c], O.round_to_bf16(ref))
+        ref_inv = 1.0 / (math.sqrt(np.sum(ref * ref)) + O.NORM_EPS)
+        assert math.isclose(inv[u].item(), ref_inv, rel_tol=1e-5)
+
+
+def test_momentum_zero_gradient_gives_zero_x():
+    shapes, M = [(32, 64)], 2
+    g = [torch.zeros(32, 64, device="cuda") for _ in range(M)]
+    m = [torch.zeros(32, 64, device="cuda") for _ in range(M)]
+    xs, inv = gpu_momentum(shapes, M, g, m, 0.9, torch.float32)
+    assert all(torch.all(x[:, :64] == 0) for x in xs)
+    assert torch.allclose(inv, torch.full_like(inv, 1e7))
+
+
+# ---------------------------------------------------------------------------
+# Newton-Schulz
+# ---------------------------------------------------------------------------
+NS_CASES = [([(256, 256)], 4, 1), ([(128, 384), (384, 128)], 2, 2), ([(100, 300), (300, 100)], 2, 5),
+            ([(64, 147), (147, 64)], 3, 1), ([(768, 2304)], 1, 5), ([(3072, 768)], 1, 5),
+            ([(1, 1), (1, 40), (40, 1)], 2, 3), ([(513, 513)], 1, 2), ([(2048, 1000)], 1, 1)]
+
+
+@pytest.mark.parametrize("shapes,M,k", NS_CASES)
+def test_newton_schulz_matches_oracle(shapes, M, k):
+    beta = 0.9
+    grads, moms = seeded_state(shapes, M, 5)
+    g_d = [g.cuda() for g in grads]
+    m_d = [m.cuda() for m in moms]
+    xs, inv = gpu_momentum(shapes, M, g_d, m_d, beta, torch.float32)
+    us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, us)
+    for u in range(len(xs)):
+        _, ref = oracle_u(moms[u], grads[u], beta, k)
+        got = f64(us[u])
+        err = rel_fro(got, ref)
+        assert err <= NS_TOL, (shapes[u // M], k, err)
+        big = np.abs(ref) > 1e-3
+        if big.sum() > 0:
+            agree = np.mean(np.sign(got[big]) == np.sign(ref[big]))
+            assert agree >= SIGN_AGREE, (shapes[u // M], agree)
+
+
+def test_newton_schulz_fused_outputs_are_signs_of_u():
+    """The packed and int8 epilogues write exactly the signs of the fp32 U the
+    same launch configuration produces (sign(0) = +1)."""
+    shapes, M, k = [(96, 300), (300, 96), (64, 147)], 2, 2
+    grads, moms = seeded_state(shapes, M, 7)
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9,
+                           torch.float32)
+    saved = [x.clone() for x in xs]
+    us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, us)
+    for x, s in zip(xs, saved):
+        x.copy_(s)
+    packed = [torch.zeros(L.signmuon_packed_words(shapes[u // M]), dtype=torch.int32, device="cuda")
+              for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_PACK1, packed)
+    for x, s in zip(xs, saved):
+        x.copy_(s)
+    i8 = [torch.zeros(shapes[u // M], dtype=torch.int8, device="cuda") for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_INT8, i8)
+    for u in range(len(xs)):
+        r, c = shapes[u // M]
+        uu = us[u].cpu().numpy()
+        plus = ~(uu < 0)
+        assert np.array_equal(i8[u].cpu().numpy(), np.where(plus, 1, -1))
+        words = packed[u].cpu().numpy().view(np.uint32)
+        wpr = (c + 31) // 32
+        for j in range(c):
+            bit = (words[: r * wpr].reshape(r, wpr)[:, j // 32] >> np.uint32(j % 32)) & 1
+            assert np.array_equal(bit.astype(bool), plus[:, j])
+
+
+def test_newton_schulz_waves_match_single_wave():
+    shapes, M, k = [(128, 256), (256, 128), (200, 200)], 3, 2
+    grads, moms = seeded_state(shapes, M, 9)
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9,
+                           torch.float32)
+    saved = [x.clone() for x in xs]
+    u1 = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, u1)
+    for x, s in zip(xs, saved):
+        x.copy_(s)
+    u2 = [torch.empty_like(t) for t in u1]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, u2, minimal_ws=True)
+    for a, b in zip(u1, u2):
+        assert torch.equal(a, b)
+
+
+def test_newton_schulz_k0_and_zero_input():
+    shapes, M = [(40, 72), (72, 40)], 2
+    grads, moms = seeded_state(shapes, M, 11)
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9,
+                           torch.float32)
+    us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, 0, L.SIGNMUON_OUT_U_F32, us)
+    for u in range(len(xs)):
+        m, ref = oracle_u(moms[u], grads[u], 0.9, 0)
+        assert rel_fro(f64(us[u]), ref) < 4e-3     # bf16 rounding of X0 only
+    # Zero momentum: U = 0 and every sign is +1.
+    z = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
+    xs, inv = gpu_momentum(shapes, M, z, [torch.zeros_like(t) for t in z], 0.9, torch.float32)
+    packed = [torch.zeros(L.signmuon_packed_words(shapes[u // M]), dtype=torch.int32, device="cuda")
+              for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, 3, L.SIGNMUON_OUT_PACK1, packed)
+    for u in range(len(xs)):
+        r, c = shapes[u // M]
+        ref = O.pack_signs(np.ones((r, c), dtype=np.int8)).reshape(-1)
+        assert np.array_equal(packed[u].cpu().numpy().view(np.uint32)[: ref.size], ref)
+
+
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
+def test_polar_step_update(w_dtype):
+    """Vote-out, then one Newton-Schulz iteration on the voted matrix fused with
+    W <- W - eta * U_V (the optional local polar step)."""
+    shapes, M, eta = [(256, 256), (128, 384)], 4, 0.02
+    all_signs = [_signs(s, M, seed=20 + i) for i, s in enumerate(shapes)]
+    flat = []
+    for s_list, shp in zip(all_signs, shapes):
+        flat += _packed_device(s_list, shp)
+    votes = [torch.zeros((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device="cuda") for r, c in shapes]
+    nnz = torch.zeros(2, dtype=torch.int64, device="cuda")
+    inv = torch.zeros(4, dtype=torch.float32, device="cuda")
+    wk = ws(L.signmuon_vote_workspace_bytes(shapes, M))
+    L.signmuon_vote_update(shapes, M, False, [x.data_ptr() for x in flat], L.SIGNMUON_F32, None, eta,
+                           [v.data_ptr() for v in votes], nnz.data_ptr(), inv.data_ptr(), wk.data_ptr(),
+                           wk.numel(), stream())
+    w0 = [syn.gaussian(s, 0.02, "cpu", "pw", i, dtype=w_dtype) for i, s in enumerate(shapes)]
+    w = [t.cuda() for t in w0]
+    code = L.SIGNMUON_BF16 if w_dtype == torch.bfloat16 else L.SIGNMUON_F32
+    gpu_ns(shapes, 1, votes, inv, 1, L.SIGNMUON_OUT_UPDATE_W, None, code, w, eta)
+    for i, s_list in enumerate(all_signs):
+        vote = O.majority_vote([s.numpy() for s in s_list])
+        d = O.polar_direction(vote, 1)
+        if w_dtype == torch.float32:
+            delta = (f64(w[i]) - f64(w0[i])) / -eta
+            assert rel_fro(delta, d) <= NS_TOL
+        else:
+            ref = O.apply_update(f64(w0[i]), eta, d, "bf16")
+            diff = np.abs(f64(w[i]) - ref)
+            ulp = np.abs(ref) * 2.0 ** -7 + 1e-30
+            # bf16 rounding decides a few ties differently; everything else is exact or 1 ulp.
+            assert np.mean(diff <= ulp) > 0.99
+
+
+# ---------------------------------------------------------------------------
+# whole step
+# ---------------------------------------------------------------------------
+def _run_steps(wl, steps, seed=0, restore_after=None):
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    dt = syn.torch_dtype(wl.w_dtype)
+    opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
+                       polar=wl.polar)
+    weights = [w.cuda() for w in syn.initial_weights(wl, seed)]
+    signal = syn.gradient_signal(wl, seed)       # drawn on the CPU, like the oracle's inputs
+    grads = [torch.empty(s, dtype=dt, device="cuda") for s in wl.shapes for _ in range(wl.n_workers)]
+    for t in range(steps):
+        for i in range(len(wl.shapes)):
+            for m in range(wl.n_workers):
+                grads[i * wl.n_workers + m].copy_(syn.worker_gradient(wl, signal[i], i, m, t, seed))
+        opt.step(weights, grads)
+        if restore_after is not None and t == restore_after:
+            sd = opt.state_dict()
+            wsave = [w.clone() for w in weights]
+            opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
+                               polar=wl.polar)
+            opt.load_state_dict(sd)
+            for w, s in zip(weights, wsave):
+                w.copy_(s)
+    torch.cuda.synchronize()
+    return opt, weights
+
+
+def test_full_step_single256_against_oracle():
+    wl = syn.WORKLOADS["single256"]
+    opt, weights = _run_steps(wl, 1)
+    w0 = syn.initial_weights(wl, 0)[0]
+    signal = syn.gradient_signal(wl, 0)[0]
+    grads = [syn.worker_gradient(wl, signal, 0, m, 0, 0) for m in range(wl.n_workers)]
+    moms = [np.zeros(wl.shapes[0]) for _ in range(wl.n_workers)]
+    ref = O.signmuon_step(f64(w0), [f64(g) for g in grads], moms, beta=float(np.float32(wl.beta)),
+                          eta=wl.eta, k=wl.ns_iters, w_dtype=wl.w_dtype, int8_variant=True)
+    for m in range(wl.n_workers):
+        assert np.array_equal(f64(opt.mom[m]), ref["mom"][m])
+        s_gpu = opt.signs[m].cpu().numpy()
+        big = np.abs(ref["u"][m]) > 1e-3
+        assert np.mean(s_gpu[big] == ref["signs"][m][big]) >= SIGN_AGREE
+    got = f64(weights[0])
+    # Where the GPU's vote equals the oracle's the update is bit-exact; the
+    # votes can differ only where some worker's |U| is tiny.
+    same = got == ref["w"]
+    assert same.mean() >= 0.99
+    steps = np.abs(got - ref["w"])[~same] / np.float32(wl.eta)
+    assert np.all((np.abs(steps - 1) < 1e-3) | (np.abs(steps - 2) < 1e-3))
+
+
+def test_step_is_deterministic_and_resumable():
+    wl = syn.Workload("mini", ((96, 160), (160, 96), (64, 147)), 3, 2, "pack1", "bf16", g_noise_std=2.0)
+    _, w_a = _run_steps(wl, 4)
+    _, w_b = _run_steps(wl, 4)
+    _, w_c = _run_steps(wl, 4, restore_after=1)
+    for a, b, c in zip(w_a, w_b, w_c):
+        assert torch.equal(a, b)
+        assert torch.equal(a, c)
+
+
+def test_polar_workload_small_runs():
+    wl = syn.Workload("mini_polar", ((256, 256), (128, 384)), 4, 2, "pack1", "bf16", g_noise_std=4.0,
+                      polar=True)
+    opt, weights = _run_steps(wl, 2)
+    w0 = syn.initial_weights(wl, 0)
+    for w, w_init in zip(weights, w0):
+        assert torch.isfinite(w.float()).all()
+        assert not torch.equal(w.cpu(), w_init)
+
+
+@pytest.mark.slow
+def test_nanogpt_full_size_sampled_parity():
+    """The nanoGPT-small workload at full size (48 matrices, M = 8, k = 5,
+    1-bit vote), one step through the same path bench.py times.  Sampled
+    checks: momentum of every worker of one matrix per shape, sign agreement
+    of the packed output, and the vote + update of the 768x768 matrix."""
+    wl = syn.WORKLOADS["nanogpt_small"]
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    dt = syn.torch_dtype(wl.w_dtype)
+    opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt)
+    weights = [w.cuda() for w in syn.initial_weights(wl, 0)]
+    w0 = [weights[i].clone() for i in range(4)]
+    signal = [g.cuda() for g in syn.gradient_signal(wl, 0)]
+    grads = [syn.worker_gradient(wl, signal[i], i, m, 0, 0).cuda() for i in range(len(wl.shapes))
+             for m in range(wl.n_workers)]
+    opt.step(weights, grads)
+    torch.cuda.synchronize()
+    M = wl.n_workers
+    for i in range(4):  # one matrix of each shape (layer 0)
+        r, c = wl.shapes[i]
+        workers = range(M) if i == 1 else [0]
+        ref_signs = []
+        for m in workers:
+            u = i * M + m
+            mom = O.momentum_update(np.zeros((r, c)), f64(grads[u]), float(np.float32(wl.beta)))
+            assert np.array_equal(f64(opt.mom[u]), mom)
+            U = O.newton_schulz(O.frobenius_normalize(mom), wl.ns_iters)
+            s_ref = O.sign_entries(U)
+            words = opt.signs[u].cpu().numpy().view(np.uint32)
+            s_gpu = unpack_words(words, r, c)
+            big = np.abs(U) > 1e-3
+            assert np.mean(s_gpu[big] == s_ref[big]) >= SIGN_AGREE
+            ref_signs.append(s_ref)
+        if i == 1:
+            ref_w = O.apply_update(f64(w0[i]), wl.eta, O.majority_vote(ref_signs), "bf16")
+            same = f64(weights[i]) == ref_w
+            assert same.mean() >= 0.99
