@@ -31,6 +31,8 @@ if ROOT not in sys.path:
 METRIC = "params·workers/s per Sign-Muon step"
 UNIT = "params*workers/s"
 DEFAULT_CONFIG = "nanogpt_small"
+# Timed steps per workload when --steps is not given (about a second of GPU time).
+DEFAULT_STEPS = {"single256": 200, "nanogpt_small": 60, "resnet50": 100, "square4096x32": 3}
 
 
 def peaks():
@@ -53,6 +55,23 @@ def ns_flops(shapes, n_workers, k, dense=False):
     return tot * n_workers * k
 
 
+def max_over_ranks_value(x, world, device):
+    """The slowest rank's value (every rank calls this at the same point)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(units_per_step, steps, world, max_ms):
+    """Whole-job units/s: every rank processes units_per_step per step (weak
+    scaling, independent replicas), timed by the slowest rank."""
+    return units_per_step * steps * world / (max_ms / 1e3)
+
+
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -70,7 +89,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -102,28 +121,33 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- oracle arm
-def oracle_sample_step(wl, mats, seed=0):
-    """One oracle step over the (matrix index) sample: returns params*workers processed."""
+def oracle_sample_step(wl, units, seed=0):
+    """One oracle step over a sample of (matrix, worker) units: momentum,
+    Newton-Schulz, sign (and pack) per unit, then the vote and update of each
+    sampled matrix over its sampled workers.  Returns params*workers done."""
     import numpy as np
     from oracle import signmuon_oracle as O
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    by_mat = {}
+    for i, m in units:
+        by_mat.setdefault(i, []).append(m)
     done = 0
-    for i in mats:
+    for i, workers in by_mat.items():
         r, c = wl.shapes[i]
         g_star = syn.gaussian((r, c), wl.g_signal_std, "cpu", "Gstar", seed, i).double().numpy()
-        w = syn.gaussian((r, c), wl.w_std, "cpu", "W", seed, i).double().numpy()
-        grads = [g_star + syn.gaussian((r, c), wl.g_noise_std, "cpu", "eps", seed, i, m, 0).double().numpy()
-                 for m in range(wl.n_workers)]
-        moms = [np.zeros((r, c)) for _ in range(wl.n_workers)]
-        O.signmuon_step(O.round_to_dtype(w, wl.w_dtype), [O.round_to_dtype(g, wl.w_dtype) for g in grads], moms,
-                        beta=float(np.float32(wl.beta)), eta=wl.eta, k=wl.ns_iters, w_dtype=wl.w_dtype,
-                        polar=wl.polar, int8_variant=(wl.variant == "int8"))
-        done += r * c * wl.n_workers
+        w = O.round_to_dtype(syn.gaussian((r, c), wl.w_std, "cpu", "W", seed, i).double().numpy(), wl.w_dtype)
+        grads = [O.round_to_dtype(g_star + syn.gaussian((r, c), wl.g_noise_std, "cpu", "eps", seed, i, m, 0)
+                                  .double().numpy(), wl.w_dtype) for m in workers]
+        O.signmuon_step(w, grads, [np.zeros((r, c)) for _ in workers], beta=float(np.float32(wl.beta)),
+                        eta=wl.eta, k=wl.ns_iters, w_dtype=wl.w_dtype, polar=wl.polar,
+                        int8_variant=(wl.variant == "int8"))
+        done += r * c * len(workers)
     return done
 
 
 def oracle_sample(wl, budget_s):
-    """Matrices (one of each shape first) whose oracle step fits in ~budget_s."""
+    """(matrix, worker) units, one matrix of each shape first and all of its
+    workers, whose oracle step fits in about budget_s."""
     order, seen = [], set()
     for i, s in enumerate(wl.shapes):
         if s not in seen:
@@ -132,11 +156,19 @@ def oracle_sample(wl, budget_s):
     t0 = time.perf_counter()
     chosen = []
     for i in order:
-        chosen.append(i)
-        oracle_sample_step(wl, [i])
-        if time.perf_counter() - t0 > budget_s:
-            break
+        for m in range(wl.n_workers):
+            chosen.append((i, m))
+            oracle_sample_step(wl, [(i, m)])
+            if time.perf_counter() - t0 > budget_s:
+                return chosen
     return chosen
+
+
+def describe_sample(wl, units):
+    mats = sorted({i for i, _ in units})
+    shapes = ", ".join(f"{wl.shapes[i][0]}x{wl.shapes[i][1]}" for i in mats)
+    return (f"{len(units)} of {wl.units} (matrix, worker) units over {len(mats)} matrices ({shapes}), "
+            f"k={wl.ns_iters}, fp64 numpy")
 
 
 def host_cores():
@@ -156,21 +188,22 @@ def blas_threads():
 
 
 def cpu_baseline(wl, budget_s=15.0):
-    mats = oracle_sample(wl, budget_s * 0.4)
+    units = oracle_sample(wl, budget_s * 0.4)
     t0 = time.perf_counter()
-    done = oracle_sample_step(wl, mats)
+    done = oracle_sample_step(wl, units)
     dt = time.perf_counter() - t0
     return {"value": done / dt, "unit": UNIT, "cores": blas_threads() or host_cores(), "kind": "oracle",
-            "sample": f"one oracle step (fp64 numpy) over {len(mats)} of {len(wl.shapes)} matrices "
-                      f"({', '.join(f'{wl.shapes[i][0]}x{wl.shapes[i][1]}' for i in mats)}) x "
-                      f"{wl.n_workers} workers, k={wl.ns_iters}; {dt:.1f} s"}
+            "sample": f"one oracle step over {describe_sample(wl, units)}; {dt:.1f} s"}
 
 
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    mats = oracle_sample(wl, 10.0)
+    # Size each step's sample so that the whole --steps/--warmup run stays
+    # within about three minutes of host time.
+    per_step = max(0.2, 150.0 / (args.steps + args.warmup))
+    mats = oracle_sample(wl, per_step * 0.6)
     for _ in range(args.warmup):
         oracle_sample_step(wl, mats[:1])
     t0 = time.perf_counter()
@@ -179,8 +212,7 @@ def run_reference(args, wl):
         done += oracle_sample_step(wl, mats)
     dt = time.perf_counter() - t0
     value = done / dt
-    sample = (f"each step: one oracle step (fp64 numpy) over {len(mats)} of {len(wl.shapes)} matrices x "
-              f"{wl.n_workers} workers, k={wl.ns_iters}")
+    sample = f"each step: one oracle step over {describe_sample(wl, mats)}"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -226,11 +258,7 @@ def run_gpu(args, wl):
         torch.cuda.synchronize()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return t.item()
+        return max_over_ranks_value(x, world, dev)
 
     opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
                        polar=wl.polar, device=dev)
@@ -281,35 +309,53 @@ def run_gpu(args, wl):
     clk = clocks.stop() if clocks else None
 
     units_per_step = wl.params * wl.n_workers
-    value = units_per_step * args.steps * world / (ms / 1e3)
+    value = job_throughput(units_per_step, args.steps, world, ms)
 
-    # End to end through the public step: pinned host gradients -> device,
-    # step, weights -> host, every step.
+    # End to end through the public step with HOST buffers: each step's
+    # gradients come from pinned host memory and the updated weights go back
+    # to host memory.  The next step's gradients are copied on a second stream
+    # while the current step computes (copy engines overlap the kernels).
     host_g = [g.cpu().pin_memory() for g in grad_sets[0]]
-    dev_g = grad_sets[1]
     host_w = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in weights]
     h2d = sum(g.numel() * g.element_size() for g in host_g)
     d2h = sum(w.numel() * w.element_size() for w in weights)
-    for _ in range(1):
-        for hg, dg in zip(host_g, dev_g):
-            dg.copy_(hg, non_blocking=True)
-        opt.step(weights, dev_g)
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def h2d_into(buf):
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(consumed[buf])
+            for hg, dg in zip(host_g, grad_sets[buf]):
+                dg.copy_(hg, non_blocking=True)
+            copied[buf].record(copy_stream)
+
+    def e2e_steps(n):
+        h2d_into(0)
+        for t in range(n):
+            buf = t % 2
+            if t + 1 < n:
+                h2d_into(1 - buf)
+            stream.wait_event(copied[buf])
+            opt.step(weights, grad_sets[buf])
+            consumed[buf].record(stream)
+            for hw, w in zip(host_w, weights):
+                hw.copy_(w, non_blocking=True)
+
+    e2e_steps(2)
     barrier()
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_steps = max(2, min(args.steps, 5))
+    n_e2e = max(3, min(args.steps, 10))
     e_start.record(stream)
-    for _ in range(e_steps):
-        for hg, dg in zip(host_g, dev_g):
-            dg.copy_(hg, non_blocking=True)
-        opt.step(weights, dev_g)
-        for hw, w in zip(host_w, weights):
-            hw.copy_(w, non_blocking=True)
+    e2e_steps(n_e2e)
     e_stop.record(stream)
     barrier()
     e_ms = max_over_ranks(e_start.elapsed_time(e_stop))
-    e2e = {"value": units_per_step * e_steps * world / (e_ms / 1e3), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
-           "ms_per_step": e_ms / e_steps}
+    e2e = {"value": units_per_step * n_e2e * world / (e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+           "ms_per_step": e_ms / n_e2e,
+           "note": "gradients H2D from pinned host memory (overlapped with the previous step on a copy "
+                   "stream) + step + weights D2H, every step"}
 
     pk = peaks()
     flops = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters)
@@ -344,17 +390,112 @@ def run_gpu(args, wl):
     return 0
 
 
+def run_vote_sweep(args):
+    """Vote + update alone (the bandwidth-bound row): P params as (P/1024, 1024)
+    fp32 W, M packed sign buffers with P(+1) ~ U(0,1) per entry."""
+    import torch
+    from sign_muon_optimizer_momentum_b200 import _lib as L
+    from sign_muon_optimizer_momentum_b200 import build as _build
+    from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    _build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    P, M = args.sweep_params, args.sweep_workers
+    shape = (P // 1024, 1024)
+    stream = torch.cuda.current_stream(dev)
+    words = L.signmuon_packed_words(shape)
+    signs = []
+    for m, s8 in syn.vote_sweep_signs(P, M, seed=rank, device=dev):
+        buf = torch.empty(words, dtype=torch.int32, device=dev)
+        L.signmuon_sign_pack(shape, L.SIGNMUON_F32, s8.float().data_ptr(), 1024, 0, buf.data_ptr(),
+                             stream.cuda_stream)
+        torch.cuda.synchronize()
+        signs.append(buf)
+        del s8
+    w = syn.gaussian(shape, 0.02, dev, "W", rank, 0)
+    wsz = L.signmuon_vote_workspace_bytes([shape], M)
+    wsb = torch.zeros(wsz, dtype=torch.uint8, device=dev)
+    sp = [t.data_ptr() for t in signs]
+
+    def step():
+        L.signmuon_vote_update([shape], M, False, sp, L.SIGNMUON_F32, [w.data_ptr()], 0.01, None, 0, 0,
+                               wsb.data_ptr(), wsz, stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    clk = clocks.stop() if clocks else None
+    per = ms / args.steps
+    bytes_per = P * (M / 8 + 8)
+    pk = peaks()
+    gbs = bytes_per / (per / 1e3) / 1e9
+    res = {"metric": METRIC, "value": P * M * world / (per / 1e3), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": per, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+           "config": {"workload": "vote_sweep", "params": P, "workers": M, "w_dtype": "f32", "eta": 0.01,
+                      "l2": f"inputs larger than L2 ({bytes_per / 2**30:.2f} GiB per step)"},
+           "roofline": {"bound": "hbm", "kernel": "vote_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                        "note": f"algorithmic {M}/8 + 8 B/param (packed signs read, fp32 W read+write)"},
+           "gpu_launches": 3 * args.steps, "clocks": clk}
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--mats", type=int, default=None,
+                    help="keep only the first N matrices of the workload (small profiling cases)")
+    ap.add_argument("--sweep-params", type=int, default=1 << 30)
+    ap.add_argument("--sweep-workers", type=int, default=16)
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    if args.config == "vote_sweep":
+        if args.steps is None:
+            args.steps = 50
+        return run_vote_sweep(args)
     wl = syn.WORKLOADS[args.config]
+    if args.mats:
+        import dataclasses
+        wl = dataclasses.replace(wl, name=f"{wl.name}[:{args.mats}]", shapes=wl.shapes[: args.mats])
+    if args.steps is None:
+        args.steps = 10 if args.impl == "reference" else DEFAULT_STEPS.get(wl.name, 20)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

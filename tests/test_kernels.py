@@ -477,4 +477,9 @@ def test_nanogpt_full_size_sampled_parity():
         if i == 1:
             ref_w = O.apply_update(f64(w0[i]), wl.eta, O.majority_vote(ref_signs), "bf16")
             same = f64(weights[i]) == ref_w
-            assert same.mean() >= 0.99
+            # The GPU's vote can differ from the oracle's only where one worker's
+            # sign flipped, i.e. where the oracle's vote was marginal (|2c - M| <= 2).
+            count = sum((s == 1).astype(np.int64) for s in ref_signs)
+            marginal = np.abs(2 * count - M) <= 2
+            assert same.mean() >= 0.98
+            assert np.mean(marginal[~same]) >= 0.95
