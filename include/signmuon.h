@@ -21,7 +21,9 @@
  *   arrays whose elements are device pointers.  The library copies what it
  *   needs into the caller's device workspace.
  * - Ownership: the caller owns every buffer, including the workspace.  The
- *   library allocates no memory and keeps no state between calls.
+ *   library allocates no memory and keeps no state between calls (the one
+ *   exception is the fixed scratch array of signmuon_momentum_norm_noalloc,
+ *   described at its declaration).
  * - Units: a "unit" is one (matrix i, worker m) pair; per-unit arrays have
  *   n_mats * n_workers entries, indexed i * n_workers + m.
  * - Matrices are row-major.  Dense fp32/bf16/int8 buffers have row stride
@@ -197,6 +199,34 @@ signmuon_status signmuon_vote_update(const signmuon_shape* shapes, int n_mats, i
                                      signmuon_dtype w_dtype, void* const* w, float eta,
                                      void* const* vote_bf16, int64_t* nnz, float* vote_inv_norm,
                                      void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Allocation-free variant of signmuon_momentum_norm.
+ * The paper has no counterpart: this is a deployment convenience.
+ *
+ * Same inputs, outputs and results as signmuon_momentum_norm, but the
+ * scratch it needs (unit table and per-block partial sums) lives in a 1 MiB
+ * device array inside the library rather than in a caller workspace.  It is
+ * meant for callers that cannot allocate device memory around the step, e.g.
+ * an optimizer embedded in a runtime whose allocator already owns the whole
+ * device, or a loop that must avoid cudaMalloc/cudaFree because they
+ * synchronise the device.  The call itself allocates nothing.
+ *
+ * Limits: n_mats * n_workers <= 1170 units, and at most 245760 blocks of
+ * 4096 elements in total (sum over units of ceil(rows*cols/4096)), i.e.
+ * about 1.0e9 momentum elements; larger requests return
+ * SIGNMUON_ERR_WORKSPACE without enqueuing anything.
+ * The array (1 MiB) is held on every GPU that loads the library until the
+ * process exits.  The first call on each device looks up the array's device
+ * address (once per device, with that device current); make that first call
+ * before any stream capture.  All calls share the array and each call
+ * rewrites what it reads, so nothing needs clearing, but calls whose kernels
+ * can overlap on the GPU (different streams with no ordering) race on it.
+ * ---------------------------------------------------------------------- */
+signmuon_status signmuon_momentum_norm_noalloc(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                               signmuon_dtype grad_dtype, const void* const* grad,
+                                               float* const* mom, float beta, void* const* x_bf16,
+                                               float* inv_norm, void* stream);
 
 #ifdef __cplusplus
 }

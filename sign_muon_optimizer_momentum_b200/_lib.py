@@ -39,6 +39,7 @@ EXPORTS = (
     "signmuon_device_error", "signmuon_momentum_workspace_bytes", "signmuon_momentum_norm",
     "signmuon_newton_schulz_workspace_bytes", "signmuon_newton_schulz_batched",
     "signmuon_sign_pack", "signmuon_vote_workspace_bytes", "signmuon_vote_update",
+    "signmuon_momentum_norm_noalloc",
 )
 
 
@@ -72,6 +73,7 @@ _SIGS = {
                                             _I, _PP, _I, _PP, _F, _P, _SZ, _P]),
     "signmuon_sign_pack": (_I, [Shape, _I, _P, ctypes.c_int64, _I, _P, _P]),
     "signmuon_vote_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I]),
+    "signmuon_momentum_norm_noalloc": (_I, [ctypes.POINTER(Shape), _I, _I, _I, _PP, _PP, _F, _PP, _P, _P]),
     "signmuon_vote_update": (_I, [ctypes.POINTER(Shape), _I, _I, _I, _PP, _I, _PP, _F, _PP, _P, _P,
                                   _P, _SZ, _P]),
 }
@@ -180,3 +182,13 @@ def signmuon_vote_update(shapes, n_workers, int8_in, signs, w_dtype, w, eta, vot
                                      _ptrs(signs), w_dtype, _ptrs(w), eta, _ptrs(vote_bf16), nnz,
                                      vote_inv_norm, workspace, ws_bytes, stream)
     _check("signmuon_vote_update", st)
+
+
+def signmuon_momentum_norm_noalloc(shapes, n_workers, grad_dtype, grad, mom, beta, x_bf16, inv_norm,
+                                   stream=0) -> None:
+    """Same as signmuon_momentum_norm with the scratch inside the library
+    (for callers that cannot allocate device memory; see the header)."""
+    st = load().signmuon_momentum_norm_noalloc(_shapes(shapes), len(shapes), n_workers, grad_dtype,
+                                               _ptrs(grad), _ptrs(mom), beta, _ptrs(x_bf16), inv_norm,
+                                               stream)
+    _check("signmuon_momentum_norm_noalloc", st)
