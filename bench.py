@@ -44,6 +44,36 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+KERNEL_SOURCES = ("sign_muon_optimizer_momentum_b200/csrc/ns_gemm.cu",
+                  "sign_muon_optimizer_momentum_b200/csrc/elementwise.cu",
+                  "sign_muon_optimizer_momentum_b200/csrc/common.cuh")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the ncu summary in
+    profiles/dram_traffic.json, or None if absent or taken on other sources."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        entries = json.load(open(p))
+    except ValueError:
+        return None
+    src = kernel_source_hash()
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_hash") == src:
+            return e.get("bytes_per_launch")
+    return None
+
+
 def ns_flops(shapes, n_workers, k, dense=False):
     """Algorithmic Newton-Schulz FLOPs per step: per iteration and unit,
     Gram s^2 l (symmetric output), square s^3 (symmetric output) and apply
@@ -366,7 +396,7 @@ def run_gpu(args, wl):
     achieved = flops / (ns_ms / 1e3) / 1e12
     roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved,
                 "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                "traffic": None,
+                "traffic": captured_traffic("ns_gemm_kernel", wl.name),
                 "note": f"{flops_note}: {flops / 1e12:.3f} TFLOP algorithmic (symmetric-aware) per step "
                         f"over {ns_ms:.3f} ms (CUDA events, mean of {args.steps} timed steps); "
                         f"dense-equivalent {ns_flops(wl.shapes, wl.n_workers, wl.ns_iters, True) / (ns_ms / 1e3) / 1e12:.1f} "
@@ -461,7 +491,8 @@ def run_vote_sweep(args):
            "config": {"workload": "vote_sweep", "params": P, "workers": M, "w_dtype": "f32", "eta": 0.01,
                       "l2": f"inputs larger than L2 ({bytes_per / 2**30:.2f} GiB per step)"},
            "roofline": {"bound": "hbm", "kernel": "vote_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
-                        "unit": "GB/s", "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                        "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                        "traffic": captured_traffic("vote_kernel", f"vote_sweep_P{P}_M{M}"),
                         "note": f"algorithmic {M}/8 + 8 B/param (packed signs read, fp32 W read+write)"},
            "gpu_launches": 3 * args.steps, "clocks": clk}
     if world > 1:

@@ -43,8 +43,13 @@ constexpr int kBStageBytes = kBN * kBK * 2;               // 32 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;  // 48 KB
 constexpr int kAccCols = kBN;                             // fp32 columns per accumulator
 constexpr int kTmemCols = 2 * kAccCols;                   // double-buffered: 512
-constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kEpilogueThreads = 256;                     // warps 2-9
+constexpr int kGemmThreads = 64 + kEpilogueThreads;       // warp 0 TMA, warp 1 MMA
+constexpr int kBarrierBytes = 256;
+constexpr int kXposeStride = 40;  // bf16 elements per row of a transpose buffer (80 B)
+constexpr int kXposeBytes = (kEpilogueThreads / 32) * 32 * kXposeStride * 2;  // 20 KB
+constexpr int kGemmSmemBytes = kStages * kStageBytes + kBarrierBytes + kXposeBytes + 1024 /*align*/;
+static_assert(kGemmSmemBytes <= 232448, "shared memory per CTA");
 
 enum NsStage : int { kStageGram = 0, kStageSquare = 1, kStageApply = 2 };
 
@@ -64,7 +69,7 @@ struct alignas(64) NsUnit {
   CUtensorMap map_x;     // caller's bf16 X buffer  [rows, ld_x]
   CUtensorMap map_xalt;  // workspace bf16 X buffer [rows, ld_x]
   CUtensorMap map_a;     // workspace Gram A        [s, ld_s]
-  CUtensorMap map_b;     // workspace polynomial B  [s, ld_s]
+  CUtensorMap map_b;     // workspace B' = aI + bA + cA^2 [s, ld_s]
   __nv_bfloat16* x;
   __nv_bfloat16* xalt;
   __nv_bfloat16* a;

@@ -294,17 +294,27 @@ __device__ __forceinline__ float upd_f32(float w, float eta, int v) {
   return v == 0 ? w : (v > 0 ? w - eta : w + eta);
 }
 
-// W - eta*v for bf16 W with a single rounding: the difference is exact in
-// fp64; it is rounded to fp32 with round-to-odd (truncate, then force the
-// last bit if anything was dropped) and then to bf16 with round-to-nearest-
-// even.  Round-to-odd at 24 bits followed by rounding to 8 bits equals the
-// direct rounding because 24 >= 8 + 2.
+// W - eta*v for bf16 W with a single rounding.  s = w - eta*v in fp32 is the
+// correctly rounded fp32 value, and rounding s to bf16 equals rounding the
+// exact difference unless s lies exactly on a bf16 rounding midpoint (low 16
+// bits 0x8000): the bf16 midpoints are fp32 numbers and rounding is
+// monotonic, so otherwise s and the exact value are on the same side of
+// every midpoint.  On a midpoint the exact fp32 rounding error (Knuth's
+// two-sum) says which way the exact value lies: above -> round away from
+// zero, below -> toward zero, zero -> a true tie, rounded to even.
 __device__ __forceinline__ __nv_bfloat16 upd_bf16(__nv_bfloat16 wb, float eta, int v) {
   if (v == 0) return wb;
-  const double d = (double)__bfloat162float(wb) - (v > 0 ? (double)eta : -(double)eta);
-  float r = __double2float_rz(d);
-  if ((double)r != d) r = __uint_as_float(__float_as_uint(r) | 1u);
-  return __float2bfloat16_rn(r);
+  const float w = __bfloat162float(wb);
+  const float d = v > 0 ? -eta : eta;
+  const float s = __fadd_rn(w, d);
+  const uint32_t bits = __float_as_uint(s);
+  if ((bits & 0xFFFFu) != 0x8000u) return __float2bfloat16_rn(s);
+  const float bb = __fsub_rn(s, w);
+  const float err = __fadd_rn(__fsub_rn(w, __fsub_rn(s, bb)), __fsub_rn(d, bb));
+  if (err == 0.f) return __float2bfloat16_rn(s);
+  const uint32_t hi = bits & 0xFFFF0000u;  // magnitude truncated (sign-magnitude)
+  const bool away = (err > 0.f) == (s > 0.f);
+  return __ushort_as_bfloat16((unsigned short)((away ? hi + 0x10000u : hi) >> 16));
 }
 
 __device__ __forceinline__ int vote_of(uint32_t gt, uint32_t tie, int j) {
@@ -321,93 +331,61 @@ __device__ __forceinline__ int find_vote_mat(const VoteMat* mats, int n, int b) 
 }
 
 // Packed fast path (cols % 32 == 0): packed word w covers W[32w, 32w+32).
-// Each thread counts 4 consecutive words (one 16-byte load per worker); a
-// warp covers 128 words = 4096 weights, which it then updates with
-// coalesced vector accesses, fetching the masks by shuffle.
-constexpr int kVoteWordsPerThread = 4;
-constexpr int kVoteWordsPerBlock = kVoteThreads * kVoteWordsPerThread;  // 1024
+// Each thread counts one word (a 4-byte load per worker, 128 contiguous bytes
+// per warp and worker); a warp covers 32 words = 1024 weights, which it then
+// updates with coalesced vector accesses, fetching each word's vote masks by
+// shuffle.  One word per thread keeps the counter in 7 registers, so many
+// warps (and many loads) are in flight per SM.
+constexpr int kVoteWordsPerBlock = kVoteThreads;  // 256 words = 8192 weights
 constexpr int kVoteInt8PerThread = 16;
 constexpr int kVoteInt8PerBlock = kVoteThreads * kVoteInt8PerThread;   // 4096
 constexpr int kVoteGeneralWordsPerBlock = kVoteThreads;
 
-template <typename Count>
-__device__ __forceinline__ void count_words(const void* const* __restrict__ tab, int m_workers,
-                                            int64_t q, BitCount (&bc)[4], Count) {
+__device__ __forceinline__ void count_word(const void* const* __restrict__ tab, int m_workers, int64_t w,
+                                           BitCount& bc) {
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-#pragma unroll
-    for (int p = 0; p < 7; ++p) bc[k].p[p] = 0;
+  for (int p = 0; p < 7; ++p) bc.p[p] = 0;
   int m = 0;
   for (; m + 8 <= m_workers; m += 8) {
-    uint4 x[8];
+    uint32_t x[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = __ldg(static_cast<const uint4*>(tab[m + j]) + q);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      auto comp = [&](int j) -> uint32_t {
-        return k == 0 ? x[j].x : (k == 1 ? x[j].y : (k == 2 ? x[j].z : x[j].w));
-      };
-      uint32_t t2a, t2b, t4a, t4b, t8;
-      csa(t2a, bc[k].p[0], bc[k].p[0], comp(0), comp(1));
-      csa(t2b, bc[k].p[0], bc[k].p[0], comp(2), comp(3));
-      csa(t4a, bc[k].p[1], bc[k].p[1], t2a, t2b);
-      csa(t2a, bc[k].p[0], bc[k].p[0], comp(4), comp(5));
-      csa(t2b, bc[k].p[0], bc[k].p[0], comp(6), comp(7));
-      csa(t4b, bc[k].p[1], bc[k].p[1], t2a, t2b);
-      csa(t8, bc[k].p[2], bc[k].p[2], t4a, t4b);
-      ripple(bc[k], t8, 3);
-    }
+    for (int j = 0; j < 8; ++j) x[j] = __ldg(static_cast<const uint32_t*>(tab[m + j]) + w);
+    uint32_t t2a, t2b, t4a, t4b, t8;
+    csa(t2a, bc.p[0], bc.p[0], x[0], x[1]);
+    csa(t2b, bc.p[0], bc.p[0], x[2], x[3]);
+    csa(t4a, bc.p[1], bc.p[1], t2a, t2b);
+    csa(t2a, bc.p[0], bc.p[0], x[4], x[5]);
+    csa(t2b, bc.p[0], bc.p[0], x[6], x[7]);
+    csa(t4b, bc.p[1], bc.p[1], t2a, t2b);
+    csa(t8, bc.p[2], bc.p[2], t4a, t4b);
+    ripple(bc, t8, 3);
   }
-  for (; m < m_workers; ++m) {
-    const uint4 x = __ldg(static_cast<const uint4*>(tab[m]) + q);
-    ripple(bc[0], x.x, 0);
-    ripple(bc[1], x.y, 0);
-    ripple(bc[2], x.z, 0);
-    ripple(bc[3], x.w, 0);
-  }
+  for (; m < m_workers; ++m) ripple(bc, __ldg(static_cast<const uint32_t*>(tab[m]) + w), 0);
 }
-
-struct Dummy {};
 
 __device__ void vote_packed_fast(const VoteMat& mt, const void* const* __restrict__ tab, int m_workers,
                                  int lb, int w_bf16, float eta, int vote_out,
                                  unsigned long long* nnz_out) {
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  // Quad index (16-byte word group) handled by this thread.
-  const int64_t q = ((int64_t)lb * kVoteThreads + threadIdx.x);
-  const int64_t n_quads = (mt.n_words + 3) >> 2;
-  BitCount bc[4];
-  uint32_t gt[4] = {0, 0, 0, 0}, tie[4] = {0, 0, 0, 0};
-  if (q < n_quads) {
-    count_words(tab, m_workers, q, bc, Dummy{});
-#pragma unroll
-    for (int k = 0; k < 4; ++k) vote_masks(bc[k], m_workers, gt[k], tie[k]);
+  const int64_t w = (int64_t)lb * kVoteThreads + threadIdx.x;  // word of this thread
+  uint32_t gt = 0, tie = 0;
+  if (w < mt.n_words) {
+    BitCount bc;
+    count_word(tab, m_workers, w, bc);
+    vote_masks(bc, m_workers, gt, tie);
   }
-  // The warp's 128 words cover weights [p0, p0 + 4096).
-  const int64_t warp_q0 = (int64_t)lb * kVoteThreads + warp * 32;
-  const int64_t p0 = warp_q0 * 128;
+  // The warp's 32 words cover weights [p0, p0 + 1024): 256 groups of 4.
+  const int64_t p0 = (w - lane) * 32;
   unsigned long long nz = 0;
-  // 4096 weights = 1024 groups of 4; 32 iterations of 32 lanes.
-#pragma unroll 4
-  for (int it = 0; it < 32; ++it) {
-    const int g4 = it * 32 + lane;          // group of 4 weights within the warp chunk
-    const int word = g4 >> 3;                // 0..127 within the warp chunk
-    const int src_lane = word >> 2;
-    const int comp = word & 3;
-    const uint32_t g0 = __shfl_sync(0xffffffffu, gt[0], src_lane);
-    const uint32_t g1 = __shfl_sync(0xffffffffu, gt[1], src_lane);
-    const uint32_t g2 = __shfl_sync(0xffffffffu, gt[2], src_lane);
-    const uint32_t g3 = __shfl_sync(0xffffffffu, gt[3], src_lane);
-    const uint32_t t0 = __shfl_sync(0xffffffffu, tie[0], src_lane);
-    const uint32_t t1 = __shfl_sync(0xffffffffu, tie[1], src_lane);
-    const uint32_t t2 = __shfl_sync(0xffffffffu, tie[2], src_lane);
-    const uint32_t t3 = __shfl_sync(0xffffffffu, tie[3], src_lane);
-    const uint32_t gw = comp == 0 ? g0 : (comp == 1 ? g1 : (comp == 2 ? g2 : g3));
-    const uint32_t tw = comp == 0 ? t0 : (comp == 1 ? t1 : (comp == 2 ? t2 : t3));
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int g4 = it * 32 + lane;    // group of 4 weights within the warp chunk
+    const int src = g4 >> 3;          // lane holding the word of this group
+    const uint32_t gw = __shfl_sync(0xffffffffu, gt, src);
+    const uint32_t tw = __shfl_sync(0xffffffffu, tie, src);
     const int sh = (g4 & 7) * 4;
     const int64_t p = p0 + (int64_t)g4 * 4;
-    if (p >= mt.n) continue;  // n is a multiple of 32, so a group is all-in or all-out
+    if (p >= mt.n) continue;  // n is a multiple of 32: a group is all-in or all-out
     int v[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) v[j] = vote_of(gw, tw, sh + j);
@@ -419,20 +397,20 @@ __device__ void vote_packed_fast(const VoteMat& mt, const void* const* __restric
       *reinterpret_cast<uint2*>(vo + p) = *reinterpret_cast<const uint2*>(h);
       nz += (v[0] != 0) + (v[1] != 0) + (v[2] != 0) + (v[3] != 0);
     } else if (w_bf16) {
-      __nv_bfloat16* w = static_cast<__nv_bfloat16*>(mt.w);
-      uint2 raw = *reinterpret_cast<const uint2*>(w + p);
+      __nv_bfloat16* wp = static_cast<__nv_bfloat16*>(mt.w);
+      uint2 raw = *reinterpret_cast<const uint2*>(wp + p);
       __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&raw);
 #pragma unroll
       for (int j = 0; j < 4; ++j) e[j] = upd_bf16(e[j], eta, v[j]);
-      *reinterpret_cast<uint2*>(w + p) = raw;
+      *reinterpret_cast<uint2*>(wp + p) = raw;
     } else {
-      float* w = static_cast<float*>(mt.w);
-      float4 x = *reinterpret_cast<const float4*>(w + p);
+      float* wp = static_cast<float*>(mt.w);
+      float4 x = *reinterpret_cast<const float4*>(wp + p);
       x.x = upd_f32(x.x, eta, v[0]);
       x.y = upd_f32(x.y, eta, v[1]);
       x.z = upd_f32(x.z, eta, v[2]);
       x.w = upd_f32(x.w, eta, v[3]);
-      *reinterpret_cast<float4*>(w + p) = x;
+      *reinterpret_cast<float4*>(wp + p) = x;
     }
   }
   if (vote_out) {
@@ -574,7 +552,7 @@ cudaError_t launch_vote_inv(const int64_t* nnz, float* inv, int n_mats, cudaStre
 
 int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words) {
   if (int8_in) return (int)((n + kVoteInt8PerBlock - 1) / kVoteInt8PerBlock);
-  if ((cols & 31) == 0) return (int)((((n_words + 3) >> 2) + kVoteThreads - 1) / kVoteThreads);
+  if ((cols & 31) == 0) return (int)((n_words + kVoteWordsPerBlock - 1) / kVoteWordsPerBlock);
   return (int)((n_words + kVoteGeneralWordsPerBlock - 1) / kVoteGeneralWordsPerBlock);
 }
 

@@ -5,17 +5,18 @@
 // item 1: the momentum is orthogonalised toward its polar factor) over every
 // (matrix, worker) unit of a launch:
 //   stage Gram:   A = X X^T            (X^T X for tall X), symmetric output
-//   stage Square: B = b A + c A A      (A symmetric, so A A = A A^T)
-//   stage Apply:  X' = a X + B X       (X B for tall X)
+//   stage Square: B' = a I + b A + c A A   (A symmetric, so A A = A A^T)
+//   stage Apply:  X' = B' X            (X B' for tall X), i.e. a X + (b A + c A^2) X
 // with, in the last iteration, the entrywise sign fused into the epilogue and
 // written as packed bits or int8 (steps 2-3 of the summary's flow), or the
 // update W <- W - eta U (the optional local polar step, step 5).
 //
-// Roles (192 threads, one CTA per SM):
+// Roles (320 threads, one CTA per SM):
 //   warp 0     TMA producer: 64x64 bf16 boxes, 128-byte swizzle, 4 stages
 //   warp 1     MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128 N=256
 //              K=16, fp32 accumulators in TMEM, double-buffered (2 x 256 cols)
-//   warps 2-5  epilogue: tcgen05.ld 32x32b, fp32 math, stores
+//   warps 2-9  epilogue: tcgen05.ld 32x32b, fp32 math, stores (two warps per
+//              TMEM lane quadrant, one per half of the accumulator columns)
 // Every mbarrier wait is bounded; on timeout the kernel records an error
 // code, lets the other roles drain, waits (bounded) for its own copies and
 // MMAs, frees TMEM and returns.
@@ -114,7 +115,9 @@ __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// Issues a 32-lane x 32-column fp32 TMEM load; the registers are valid only
+// after tmem_wait_ld on the same array.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -125,7 +128,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
         "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Waits for this thread's outstanding TMEM loads.  The registers are tied to
+// the wait so the compiler cannot read them before it.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                 "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                 "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled bf16 operand.
@@ -152,43 +167,61 @@ __device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn) {
 }
 
 // ---------------------------------------------------------------------------
-// Tile decoding (identical in all roles)
+// Tile scheduling.  Tiles of a launch are numbered unit by unit (each unit's
+// tiles are consecutive, prefix in NsUnit::tile_begin); CTA b takes tiles
+// b, b + grid, b + 2 grid, ...  Every role walks the same sequence with its
+// own cursor, so a unit's record is read once per unit, not once per tile.
 // ---------------------------------------------------------------------------
+struct UnitCursor {
+  int idx = -1;    // current unit
+  int begin = 0;   // its first tile
+  int end = 0;     // one past its last tile
+  int rows = 0, cols = 0;
+};
+
+// Moves the cursor to the unit holding tile t (t never decreases).  Returns
+// true when the unit changed.
+__device__ __forceinline__ bool cursor_seek(const NsLaunch& L, UnitCursor& c, int t) {
+  if (c.idx >= 0 && t < c.end) return false;
+  int lo = c.idx < 0 ? 0 : c.idx + 1;
+  if (c.idx >= 0 && lo < L.n_units && t < L.units[lo].tile_begin[L.stage] + L.units[lo].tile_count[L.stage]) {
+    // common case: the next unit
+  } else {
+    int hi = L.n_units - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (L.units[mid].tile_begin[L.stage] <= t) lo = mid; else hi = mid - 1;
+    }
+  }
+  const NsUnit& u = L.units[lo];
+  c.idx = lo;
+  c.begin = u.tile_begin[L.stage];
+  c.end = c.begin + u.tile_count[L.stage];
+  c.rows = u.rows;
+  c.cols = u.cols;
+  return true;
+}
+
 struct Tile {
-  const NsUnit* u;
   int M, N, K;
   int m0, n0;
   int a_mn, b_mn, sym;
-  const CUtensorMap* ma;
-  const CUtensorMap* mb;
 };
 
-__device__ __forceinline__ Tile decode_tile(const NsLaunch& L, int t) {
-  int lo = 0, hi = L.n_units - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (L.units[mid].tile_begin[L.stage] <= t) lo = mid; else hi = mid - 1;
-  }
-  const NsUnit* u = &L.units[lo];
-  int li = t - u->tile_begin[L.stage];
-  const int rows = u->rows, cols = u->cols;
+// Problem dimensions, operand majors and tile origin of local tile li of a
+// unit with the given shape.
+__device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li) {
   const bool tall = rows > cols;
   const int s = tall ? cols : rows, l = tall ? rows : cols;
-  const CUtensorMap* xin = L.parity ? &u->map_xalt : &u->map_x;
   Tile T;
-  T.u = u;
-  if (L.stage == kStageGram) {
-    T.M = s; T.N = s; T.K = l; T.sym = 1;
-    T.ma = xin; T.mb = xin; T.a_mn = tall; T.b_mn = tall;
-  } else if (L.stage == kStageSquare) {
-    T.M = s; T.N = s; T.K = s; T.sym = 1;
-    T.ma = &u->map_a; T.mb = &u->map_a; T.a_mn = 0; T.b_mn = 0;
-  } else if (!tall) {  // X' = a X + B X: A-op = B (K-major), B-op = X (MN-major)
-    T.M = rows; T.N = cols; T.K = s; T.sym = 0;
-    T.ma = &u->map_b; T.a_mn = 0; T.mb = xin; T.b_mn = 1;
-  } else {             // X' = a X + X B: A-op = X (K-major), B-op = B (symmetric)
-    T.M = rows; T.N = cols; T.K = s; T.sym = 0;
-    T.ma = xin; T.a_mn = 0; T.mb = &u->map_b; T.b_mn = 0;
+  if (stage == kStageGram) {
+    T.M = s; T.N = s; T.K = l; T.sym = 1; T.a_mn = tall; T.b_mn = tall;
+  } else if (stage == kStageSquare) {
+    T.M = s; T.N = s; T.K = s; T.sym = 1; T.a_mn = 0; T.b_mn = 0;
+  } else if (!tall) {  // X' = B' X: A-op = B' (K-major), B-op = X (MN-major)
+    T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 1;
+  } else {             // X' = X B': A-op = X (K-major), B-op = B' (symmetric, K-major)
+    T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 0;
   }
   const int tiles_n = (T.N + kBN - 1) / kBN;
   int tm = 0, tn = 0;
@@ -210,25 +243,31 @@ __device__ __forceinline__ Tile decode_tile(const NsLaunch& L, int t) {
   return T;
 }
 
+// Tensor maps of the two operands of a unit's tile.
+__device__ __forceinline__ void operand_maps(const NsLaunch& L, const NsUnit* u, bool tall, const CUtensorMap*& ma,
+                                             const CUtensorMap*& mb) {
+  const CUtensorMap* xin = L.parity ? &u->map_xalt : &u->map_x;
+  if (L.stage == kStageGram) {
+    ma = xin; mb = xin;
+  } else if (L.stage == kStageSquare) {
+    ma = &u->map_a; mb = &u->map_a;
+  } else if (!tall) {
+    ma = &u->map_b; mb = xin;
+  } else {
+    ma = xin; mb = &u->map_b;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Epilogue helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, bool vec, int nvalid, float (&v)[32]) {
-  if (vec) {
+__device__ __forceinline__ void unpack_bf16x8(const uint4& raw, float* v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(p + q * 8);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(h[j]);
-        v[q * 8 + 2 * j] = f.x;
-        v[q * 8 + 2 * j + 1] = f.y;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = j < nvalid ? __bfloat162float(p[j]) : 0.f;
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(h[j]);
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
   }
 }
 
@@ -263,6 +302,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   uint64_t* drain_bar = bars + 2 * kStages + 4;   // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // Per-epilogue-warp 32x32 transpose buffers (row stride 80 B: the 16-byte
+  // row reads of 8 consecutive lanes hit 8 distinct bank groups).
+  __nv_bfloat16* xpose = reinterpret_cast<__nv_bfloat16*>(smem + kStages * kStageBytes + kBarrierBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -274,7 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_addr(&tfull_bar[a]), 1);
-      mbar_init(smem_addr(&tempty_bar[a]), 128);
+      mbar_init(smem_addr(&tempty_bar[a]), kEpilogueThreads);
     }
     mbar_init(smem_addr(drain_bar), 1);
     *abort_flag = 0;
@@ -299,15 +341,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const NsUnit* last_unit = nullptr;
       bool ok = true;
+      UnitCursor cur;
+      const CUtensorMap* ma = nullptr;
+      const CUtensorMap* mb = nullptr;
       for (int t = blockIdx.x; t < L.total_tiles && ok; t += gridDim.x) {
-        const Tile T = decode_tile(L, t);
-        if (T.u != last_unit) {
-          tensormap_acquire(T.ma);
-          tensormap_acquire(T.mb);
-          last_unit = T.u;
+        if (cursor_seek(L, cur, t)) {
+          operand_maps(L, &L.units[cur.idx], cur.rows > cur.cols, ma, mb);
+          tensormap_acquire(ma);
+          tensormap_acquire(mb);
         }
+        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin);
         const int nkb = (T.K + kBK - 1) / kBK;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(smem_addr(&empty_bar[stage]), phase ^ 1, abort_flag)) {
@@ -324,12 +368,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < kBM / kBoxRows; ++j) {
             const int mn = T.m0 + j * kBoxRows;
-            tma_load_2d(sa + j * kBoxBytes, T.ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
+            tma_load_2d(sa + j * kBoxBytes, ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
           }
 #pragma unroll
           for (int j = 0; j < kBN / kBoxRows; ++j) {
             const int mn = T.n0 + j * kBoxRows;
-            tma_load_2d(sb + j * kBoxBytes, T.mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
+            tma_load_2d(sb + j * kBoxBytes, mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
           }
           ++issued_kb;
           if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -344,8 +388,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      UnitCursor cur;
       for (int t = blockIdx.x; t < L.total_tiles && ok; t += gridDim.x) {
-        const Tile T = decode_tile(L, t);
+        cursor_seek(L, cur, t);
+        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin);
         const uint32_t idesc = instr_desc(T.a_mn, T.b_mn);
         const int nkb = (T.K + kBK - 1) / kBK;
         if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag)) {
@@ -394,13 +440,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // Two warps per TMEM lane quadrant: warp w reads lanes 32*(w%4).. and the
+    // column half (w-2)/4 of the accumulator.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row_in_tile = q * 32 + lane;
+    constexpr int kChunks = kBN / 32 / 2;  // 32-column chunks per warp
     int acc = 0;
     uint32_t acc_phase = 0;
+    UnitCursor cur;
+    // The unit's fields are copied to registers once per unit: read through
+    // a global pointer they would be reloaded after every store (aliasing).
+    struct {
+      __nv_bfloat16* a;
+      __nv_bfloat16* b;
+      __nv_bfloat16* xout;
+      void* out;
+      int ld_x, ld_s, cols;
+    } uf = {nullptr, nullptr, nullptr, nullptr, 0, 0, 0};
+    float s = 1.f;
     for (int t = blockIdx.x; t < L.total_tiles; t += gridDim.x) {
-      const Tile T = decode_tile(L, t);
-      const NsUnit* u = T.u;
+      if (cursor_seek(L, cur, t)) {
+        const NsUnit* un = &L.units[cur.idx];
+        uf.a = un->a;
+        uf.b = un->b;
+        uf.xout = L.parity ? un->x : un->xalt;
+        uf.out = un->out;
+        uf.ld_x = un->ld_x;
+        uf.ld_s = un->ld_s;
+        uf.cols = un->cols;
+        s = L.first ? *un->scale : 1.f;
+      }
+      const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin);
       if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag)) {
         atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutEpilogue);
         *abort_flag = 1;
@@ -409,12 +480,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       tc_fence_after();
       const int grow = T.m0 + row_in_tile;
       const bool row_ok = grow < T.M;
-      const float s = L.first ? *u->scale : 1.f;
-      for (int ch = 0; ch < kBN / 32; ++ch) {
+      // Square stage: prefetch the A tile values of the first chunk.
+      uint4 aux[4];
+      const bool want_aux = (L.stage == kStageSquare) && row_ok;
+      auto aux_ptr = [&](int ch) { return uf.a + (int64_t)grow * uf.ld_s + T.n0 + ch * 32; };
+      auto aux_vec = [&](int ch) { return T.n0 + ch * 32 + 32 <= T.N; };
+      if (want_aux && aux_vec(half * kChunks)) {
+        const uint4* p = reinterpret_cast<const uint4*>(aux_ptr(half * kChunks));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) aux[k] = p[k];
+      }
+      // Chunks of this warp's column half that hold valid columns (warp-uniform).
+      const int n_ch = max(0, min(kChunks, (T.N - T.n0 - half * kChunks * 32 + 31) / 32));
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
+      uint32_t nxt[32];
+      if (n_ch > 0) tmem_ld32_async(tbase + (uint32_t)(half * kChunks * 32), nxt);
+#pragma unroll 1
+      for (int cc = 0; cc < n_ch; ++cc) {
+        const int ch = half * kChunks + cc;
         const int gc0 = T.n0 + ch * 32;
-        if (gc0 >= T.N) break;  // warp-uniform
+        tmem_wait_ld(nxt);
         uint32_t raw[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols + ch * 32), raw);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) raw[j] = nxt[j];
+        // The next chunk's TMEM load overlaps this chunk's math and stores.
+        if (cc + 1 < n_ch) tmem_ld32_async(tbase + (uint32_t)((ch + 1) * 32), nxt);
         if (!row_ok) continue;
         const int nvalid = min(32, T.N - gc0);
         float v[32];
@@ -423,21 +513,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) * s2;
         } else if (L.stage == kStageSquare) {
-          float av[32];
-          load_bf16x32(u->a + (int64_t)grow * u->ld_s + gc0, nvalid == 32, nvalid, av);
+          // B' = a I + b A + c A^2: folding a*I here lets the apply product
+          // X' = B' X run without reading X a second time.
+          if (nvalid == 32) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = fmaf(L.b, av[j], L.c * __uint_as_float(raw[j]));
+            for (int k = 0; k < 4; ++k) {
+              float av[8];
+              unpack_bf16x8(aux[k], av);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) v[8 * k + j] = fmaf(L.b, av[j], L.c * __uint_as_float(raw[8 * k + j]));
+            }
+            if (cc + 1 < kChunks && aux_vec(ch + 1)) {
+              const uint4* p = reinterpret_cast<const uint4*>(aux_ptr(ch + 1));
+#pragma unroll
+              for (int k = 0; k < 4; ++k) aux[k] = p[k];
+            }
+          } else {
+            const __nv_bfloat16* p = aux_ptr(ch);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              v[j] = fmaf(L.b, j < nvalid ? __bfloat162float(p[j]) : 0.f, L.c * __uint_as_float(raw[j]));
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] += (gc0 + j == grow) ? L.a : 0.f;  // diagonal of B'
         } else {
-          const __nv_bfloat16* xin = L.parity ? u->xalt : u->x;
-          float xv[32];
-          load_bf16x32(xin + (int64_t)grow * u->ld_x + gc0, nvalid == 32, nvalid, xv);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = s * fmaf(L.a, xv[j], __uint_as_float(raw[j]));
+          for (int j = 0; j < 32; ++j) v[j] = s * __uint_as_float(raw[j]);
         }
         if (T.sym) {
           // Store the upper triangle (col >= row) and mirror it (col > row).
-          __nv_bfloat16* out = (L.stage == kStageGram) ? u->a : u->b;
-          const int ld = u->ld_s;
+          __nv_bfloat16* out = (L.stage == kStageGram) ? uf.a : uf.b;
+          const int ld = uf.ld_s;
+          const int grow0 = T.m0 + q * 32;  // first row of this warp's 32x32 block
           if (gc0 >= grow) {
             store_bf16x32(out + (int64_t)grow * ld + gc0, nvalid == 32, nvalid, v);
           } else if (gc0 + 31 >= grow) {
@@ -445,21 +552,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             for (int j = 0; j < 32; ++j)
               if (j < nvalid && gc0 + j >= grow) out[(int64_t)grow * ld + gc0 + j] = __float2bfloat16_rn(v[j]);
           }
+          if (gc0 >= grow0 + 32 && nvalid == 32 && grow0 + 32 <= T.M) {
+            // Whole block strictly above the diagonal (warp-uniform): stage it
+            // transposed in shared memory, then lane j writes row gc0 + j of
+            // the mirror with 16-byte stores.
+            __nv_bfloat16* tb = xpose + (warp - 2) * (32 * kXposeStride);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < nvalid && gc0 + j > grow) out[(int64_t)(gc0 + j) * ld + grow] = __float2bfloat16_rn(v[j]);
+            for (int j = 0; j < 32; ++j) tb[j * kXposeStride + lane] = __float2bfloat16_rn(v[j]);
+            __syncwarp();
+            const uint4* src = reinterpret_cast<const uint4*>(tb + lane * kXposeStride);
+            uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(gc0 + lane) * ld + grow0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = src[k];
+            __syncwarp();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid && gc0 + j > grow) out[(int64_t)(gc0 + j) * ld + grow] = __float2bfloat16_rn(v[j]);
+          }
         } else if (L.out_kind == kOutIterate) {
-          __nv_bfloat16* xout = L.parity ? u->x : u->xalt;
-          store_bf16x32(xout + (int64_t)grow * u->ld_x + gc0, nvalid == 32, nvalid, v);
+          store_bf16x32(uf.xout + (int64_t)grow * uf.ld_x + gc0, nvalid == 32, nvalid, v);
         } else if (L.out_kind == kOutPack1) {
           uint32_t word = 0;
 #pragma unroll
           for (int j = 0; j < 32; ++j) word |= (j < nvalid && !(v[j] < 0.f)) ? (1u << j) : 0u;
-          const int wpr = (u->cols + 31) >> 5;
-          static_cast<uint32_t*>(u->out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
+          const int wpr = (uf.cols + 31) >> 5;
+          static_cast<uint32_t*>(uf.out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
         } else if (L.out_kind == kOutInt8) {
-          int8_t* o = static_cast<int8_t*>(u->out) + (int64_t)grow * u->cols + gc0;
-          if (nvalid == 32 && (u->cols & 15) == 0) {
+          int8_t* o = static_cast<int8_t*>(uf.out) + (int64_t)grow * uf.cols + gc0;
+          if (nvalid == 32 && (uf.cols & 15) == 0) {
             uint32_t pk[8];
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
@@ -476,8 +597,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
               if (j < nvalid) o[j] = v[j] < 0.f ? int8_t(-1) : int8_t(1);
           }
         } else if (L.out_kind == kOutUF32) {
-          float* o = static_cast<float*>(u->out) + (int64_t)grow * u->cols + gc0;
-          if (nvalid == 32 && (u->cols & 3) == 0) {
+          float* o = static_cast<float*>(uf.out) + (int64_t)grow * uf.cols + gc0;
+          if (nvalid == 32 && (uf.cols & 3) == 0) {
 #pragma unroll
             for (int w = 0; w < 8; ++w)
               reinterpret_cast<float4*>(o)[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
@@ -487,14 +608,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
               if (j < nvalid) o[j] = v[j];
           }
         } else {  // kOutUpdateW: W <- W - eta * U
-          const int64_t off = (int64_t)grow * u->cols + gc0;
+          const int64_t off = (int64_t)grow * uf.cols + gc0;
           if (L.w_dtype == SIGNMUON_BF16) {
-            __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u->out) + off;
+            __nv_bfloat16* w = static_cast<__nv_bfloat16*>(uf.out) + off;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (j < nvalid) w[j] = __float2bfloat16_rn(fmaf(-L.eta, v[j], __bfloat162float(w[j])));
           } else {
-            float* w = static_cast<float*>(u->out) + off;
+            float* w = static_cast<float*>(uf.out) + off;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);

@@ -483,3 +483,28 @@ def test_nanogpt_full_size_sampled_parity():
             marginal = np.abs(2 * count - M) <= 2
             assert same.mean() >= 0.98
             assert np.mean(marginal[~same]) >= 0.95
+
+
+@pytest.mark.parametrize("int8_in", [False, True])
+def test_vote_update_bf16_single_rounding_on_midpoint(int8_in):
+    """eta = 2^-9 + 2^-30 puts the fp32 difference 1 - eta exactly on the bf16
+    midpoint 1 - 2^-9 although the exact difference lies below it: a
+    double-rounded update would give 1.0, the single rounding 0.99609375."""
+    shape, M = (4, 64), 1
+    eta = float(np.float32(2.0 ** -9 + 2.0 ** -30))
+    assert eta == 2.0 ** -9 + 2.0 ** -30
+    w0 = torch.ones(shape, dtype=torch.bfloat16)
+    w0[1] = -1.0
+    w0[2] = 2.0
+    w0[3] = syn.gaussian((64,), 1.0, "cpu", "mid", dtype=torch.bfloat16)
+    signs = torch.ones(shape, dtype=torch.int8)
+    signs[1] = -1
+    dev = [signs.cuda()] if int8_in else _packed_device([signs], shape)
+    w = w0.cuda()
+    wk = ws(L.signmuon_vote_workspace_bytes([shape], M))
+    L.signmuon_vote_update([shape], M, int8_in, [d.data_ptr() for d in dev], L.SIGNMUON_BF16, [w.data_ptr()], eta,
+                           None, 0, 0, wk.data_ptr(), wk.numel(), stream())
+    torch.cuda.synchronize()
+    ref = O.apply_update(f64(w0), eta, signs.numpy(), "bf16")
+    assert ref[0, 0] == 0.99609375
+    assert np.array_equal(f64(w), ref)
