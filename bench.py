@@ -32,7 +32,8 @@ METRIC = "params·workers/s per Sign-Muon step"
 UNIT = "params*workers/s"
 DEFAULT_CONFIG = "nanogpt_small"
 # Timed steps per workload when --steps is not given (about a second of GPU time).
-DEFAULT_STEPS = {"single256": 200, "nanogpt_small": 60, "resnet50": 100, "square4096x32": 3}
+DEFAULT_STEPS = {"single256": 200, "nanogpt_small": 60, "resnet50": 100, "square4096x32": 3,
+                 "signum_nanogpt_small": 100}
 
 
 def peaks():
@@ -309,13 +310,17 @@ def run_gpu(args, wl):
 
     def one_step(t, ev=None):
         gs = grad_sets[t % n_sets]
-        opt.momentum_norm(gs, s_ptr)
         if ev is not None:
             ev[0].record(stream)
-        opt.newton_schulz(s_ptr)
+        opt.momentum_norm(gs, s_ptr)
         if ev is not None:
             ev[1].record(stream)
+        opt.newton_schulz(s_ptr)
+        if ev is not None:
+            ev[2].record(stream)
         opt.vote_update(weights, s_ptr)
+        if ev is not None:
+            ev[3].record(stream)
 
     for t in range(args.warmup):
         one_step(t)
@@ -325,8 +330,7 @@ def run_gpu(args, wl):
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    ns_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
+    ns_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     start.record(stream)
@@ -335,7 +339,9 @@ def run_gpu(args, wl):
     stop.record(stream)
     barrier()
     ms = max_over_ranks(start.elapsed_time(stop))
-    ns_ms = sum(a.elapsed_time(b) for a, b in ns_ev) / args.steps
+    mom_ms = sum(e[0].elapsed_time(e[1]) for e in ns_ev) / args.steps
+    ns_ms = sum(e[1].elapsed_time(e[2]) for e in ns_ev) / args.steps
+    vote_ms = sum(e[2].elapsed_time(e[3]) for e in ns_ev) / args.steps
     clk = clocks.stop() if clocks else None
 
     units_per_step = wl.params * wl.n_workers
@@ -388,26 +394,37 @@ def run_gpu(args, wl):
                    "stream) + step + weights D2H, every step"}
 
     pk = peaks()
-    flops = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters)
-    if wl.polar:
-        flops_note = "Newton-Schulz call of the step (the local polar step is timed with the vote)"
+    if wl.ns_iters > 0:
+        flops = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters)
+        if wl.polar:
+            flops_note = "Newton-Schulz call of the step (the local polar step is timed with the vote)"
+        else:
+            flops_note = "Newton-Schulz call of the step"
+        achieved = flops / (ns_ms / 1e3) / 1e12
+        dense = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters, True) / (ns_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved,
+                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                    "traffic": captured_traffic("ns_gemm_kernel", wl.name),
+                    "note": f"{flops_note}: {flops / 1e12:.3f} TFLOP algorithmic (symmetric-aware: 3s^2l + s^3 "
+                            f"per iteration and unit) per step over {ns_ms:.3f} ms (CUDA events, mean of "
+                            f"{args.steps} timed steps); dense-equivalent {dense:.1f} TFLOP/s; peak = "
+                            f"{pk['source']} burst bf16 cuBLAS (sustained {pk['bf16_tflops_sustained']})"}
     else:
-        flops_note = "Newton-Schulz call of the step"
-    achieved = flops / (ns_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                "traffic": captured_traffic("ns_gemm_kernel", wl.name),
-                "note": f"{flops_note}: {flops / 1e12:.3f} TFLOP algorithmic (symmetric-aware) per step "
-                        f"over {ns_ms:.3f} ms (CUDA events, mean of {args.steps} timed steps); "
-                        f"dense-equivalent {ns_flops(wl.shapes, wl.n_workers, wl.ns_iters, True) / (ns_ms / 1e3) / 1e12:.1f} "
-                        f"TFLOP/s; peak = {pk['source']} burst bf16 cuBLAS "
-                        f"(sustained {pk['bf16_tflops_sustained']})"}
+        # k = 0 (majority-vote Signum): the momentum pass dominates.
+        gbytes = wl.params * wl.n_workers * ((2 if wl.w_dtype == "bf16" else 4) + 8 + 2)
+        achieved = gbytes / (mom_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "momentum_kernel", "achieved": achieved, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                    "traffic": captured_traffic("momentum_kernel", wl.name),
+                    "note": f"momentum call: {gbytes / 1e9:.3f} GB algorithmic (gradient read, fp32 momentum "
+                            f"read+write, bf16 copy write) per step over {mom_ms:.3f} ms"}
     result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
               "config": dict(workload_config(wl), parallelism=f"replicas{world}",
                              l2=f"inputs larger than L2 ({resident / 2**30:.1f} GiB gradients+momentum resident)"),
               "roofline": roofline, "e2e": e2e,
+              "phases_ms": {"momentum": mom_ms, "newton_schulz": ns_ms, "vote_update": vote_ms},
               "gpu_launches": opt.kernel_launches_per_step() * args.steps,
               "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

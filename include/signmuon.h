@@ -88,6 +88,10 @@ const char* signmuon_status_string(int status);
 /* Library ABI version (incremented on any signature change). */
 int signmuon_abi_version(void);
 
+/* Text of the CUDA error behind the most recent SIGNMUON_ERR_CUDA returned to
+ * the calling thread ("no error" if none); static storage. */
+const char* signmuon_last_error_string(void);
+
 /* Row stride, in elements, of a bf16 Newton-Schulz buffer with `cols` columns:
  * cols rounded up to a multiple of 8 (16 bytes, the TMA stride granule). */
 int32_t signmuon_x_ld(int32_t cols);
@@ -139,7 +143,9 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
  *   rows <= cols:  A = X X^T,  B = b A + c A^2,  X <- a X + B X
  *   rows >  cols:  A = X^T X,  B = b A + c A^2,  X <- a X + X B
  * on the tensor cores (bf16 operands, fp32 accumulation, bf16 between
- * iterations).  The last iteration's epilogue writes, per out_mode:
+ * iterations).  The kernels form B' = a I + b A + c A^2 (bf16) and compute
+ * X <- B' X (X B'), the same map with the a X term folded into the product.
+ * The last iteration's epilogue writes, per out_mode:
  *   PACK1:    out[u] = packed sign(U)   (uint32, signmuon_packed_words words)
  *   INT8:     out[u] = int8 sign(U)     ([rows, cols])
  *   U_F32:    out[u] = U                (fp32 [rows, cols])

@@ -39,14 +39,15 @@ EXPORTS = (
     "signmuon_device_error", "signmuon_momentum_workspace_bytes", "signmuon_momentum_norm",
     "signmuon_newton_schulz_workspace_bytes", "signmuon_newton_schulz_batched",
     "signmuon_sign_pack", "signmuon_vote_workspace_bytes", "signmuon_vote_update",
-    "signmuon_momentum_norm_noalloc",
+    "signmuon_momentum_norm_noalloc", "signmuon_last_error_string",
 )
 
 
 class SignMuonError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        detail = f": {signmuon_last_error_string()}" if status == SIGNMUON_ERR_CUDA else ""
+        super().__init__(f"{fn} failed: {status_string(status)} ({status}){detail}")
 
 
 class Shape(ctypes.Structure):
@@ -62,6 +63,7 @@ _F = ctypes.c_float
 _SIGS = {
     "signmuon_status_string": (ctypes.c_char_p, [_I]),
     "signmuon_abi_version": (_I, []),
+    "signmuon_last_error_string": (ctypes.c_char_p, []),
     "signmuon_x_ld": (ctypes.c_int32, [ctypes.c_int32]),
     "signmuon_packed_words": (ctypes.c_int64, [Shape]),
     "signmuon_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -121,6 +123,10 @@ def _ptrs(ptrs):
     for i, p in enumerate(ptrs):
         arr[i] = int(p) if p else None
     return arr
+
+
+def signmuon_last_error_string() -> str:
+    return load().signmuon_last_error_string().decode()
 
 
 def signmuon_abi_version() -> int:

@@ -2,6 +2,7 @@
 // planning (tensor maps, unit tables) and kernel launches.  The declarations
 // and their contracts are in include/signmuon.h.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -47,7 +48,13 @@ signmuon_status check_workspace(void* ws, size_t have, size_t need) {
   return SIGNMUON_OK;
 }
 
-inline signmuon_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SIGNMUON_OK : SIGNMUON_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+inline signmuon_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SIGNMUON_OK;
+  g_last_cuda_error = e;
+  return SIGNMUON_ERR_CUDA;
+}
 
 // ----------------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -68,18 +75,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] with row stride ld elements; 64x64 boxes,
-// 128-byte swizzle, zero fill outside the tensor.
-bool encode_bf16_2d(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld) {
+// 2-D bf16 tensor [outer, inner] with row stride ld elements.  Operand maps:
+// 64x64 boxes, 128-byte swizzle, zero fill outside the tensor.  Store maps:
+// 32x32 boxes, 64-byte swizzle (writes outside the tensor are dropped).
+bool encode_bf16_2d(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                    bool store_box = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {store_box ? 32u : 64u, store_box ? 32u : 64u};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, store_box ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ----------------------------------------------------------------- NS planning
@@ -98,15 +107,19 @@ UnitBytes ns_unit_bytes(signmuon_shape sh) {
   return u;
 }
 
-int ns_tiles(int rows, int cols, int stage) {
+// Tiles of one unit in one stage; pair = 1 for 256x256 CTA-pair tiles.
+int ns_tiles(int rows, int cols, int stage, int pair) {
   const bool tall = rows > cols;
   const int s = tall ? cols : rows;
+  const int bm = ns_tile_m(pair);
   if (stage == kStageApply) {
-    return ((rows + kBM - 1) / kBM) * ((cols + kBN - 1) / kBN);
+    return ((rows + bm - 1) / bm) * ((cols + kBN - 1) / kBN);
   }
-  const int tm = (s + kBM - 1) / kBM, tn = (s + kBN - 1) / kBN;
+  // Symmetric outputs: row tile tm starts at column tile tm * bm / 256.
+  const int tm = (s + bm - 1) / bm, tn = (s + kBN - 1) / kBN;
+  const int sh = pair ? 0 : 1;
   int n = 0;
-  for (int i = 0; i < tm; ++i) n += tn - (i >> 1);
+  for (int i = 0; i < tm; ++i) n += tn - (i >> sh);
   return n;
 }
 
@@ -130,6 +143,10 @@ const char* signmuon_status_string(int status) {
 
 int signmuon_abi_version(void) { return kAbiVersion; }
 
+const char* signmuon_last_error_string(void) {
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
+
 int32_t signmuon_x_ld(int32_t cols) { return cols <= 0 ? -1 : x_ld_of(cols); }
 
 int64_t signmuon_packed_words(signmuon_shape shape) {
@@ -141,10 +158,11 @@ signmuon_status signmuon_device_error(void* workspace, uint32_t* code, void* str
   if (!workspace || !code) return SIGNMUON_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t v = 0;
-  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SIGNMUON_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SIGNMUON_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_status(e);
   *code = v;
-  if (v != 0 && cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return SIGNMUON_ERR_CUDA;
+  if (v != 0 && (e = cudaMemsetAsync(workspace, 0, 4, st)) != cudaSuccess) return cuda_status(e);
   return SIGNMUON_OK;
 }
 
@@ -285,30 +303,53 @@ signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int
       if (!encode_bf16_2d(&u.map_x, u.x, cols, rows, u.ld_x) ||
           !encode_bf16_2d(&u.map_xalt, u.xalt, cols, rows, u.ld_x) ||
           !encode_bf16_2d(&u.map_a, u.a, sdim, sdim, u.ld_s) ||
-          !encode_bf16_2d(&u.map_b, u.b, sdim, sdim, u.ld_s))
+          !encode_bf16_2d(&u.map_b, u.b, sdim, sdim, u.ld_s) ||
+          !encode_bf16_2d(&u.st_x, u.x, cols, rows, u.ld_x, true) ||
+          !encode_bf16_2d(&u.st_xalt, u.xalt, cols, rows, u.ld_x, true) ||
+          !encode_bf16_2d(&u.st_a, u.a, sdim, sdim, u.ld_s, true) ||
+          !encode_bf16_2d(&u.st_b, u.b, sdim, sdim, u.ld_s, true))
         return SIGNMUON_ERR_UNSUPPORTED;
     }
   }
   wave_begin.push_back(units);
-  // Tile prefixes restart at each wave (a launch covers one wave).
+  // Per wave and stage, pick the tile mode with the least padded work (the
+  // CTA-pair mode is preferred unless it pads more than 15 % extra), then
+  // number the tiles; prefixes restart at each wave (a launch covers one
+  // wave).
+  std::vector<int> wave_pair((wave_begin.size() - 1) * 3, 0);
+  // SIGNMUON_NS_TILE_MODE=single|pair forces one tile mode (used by the tests
+  // to compare the two modes on the same inputs); unset = automatic.
+  int forced_mode = -1;
+  if (const char* m = getenv("SIGNMUON_NS_TILE_MODE")) {
+    if (!strcmp(m, "single")) forced_mode = 0;
+    else if (!strcmp(m, "pair")) forced_mode = 1;
+  }
   for (size_t wv = 0; wv + 1 < wave_begin.size(); ++wv) {
-    int pre[3] = {0, 0, 0};
-    for (int ui = wave_begin[wv]; ui < wave_begin[wv + 1]; ++ui) {
-      for (int stg = 0; stg < 3; ++stg) {
-        hu[ui].tile_begin[stg] = pre[stg];
-        hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg);
-        pre[stg] += hu[ui].tile_count[stg];
+    for (int stg = 0; stg < 3; ++stg) {
+      double single_area = 0, pair_area = 0;
+      for (int ui = wave_begin[wv]; ui < wave_begin[wv + 1]; ++ui) {
+        single_area += (double)ns_tiles(hu[ui].rows, hu[ui].cols, stg, 0) * 128.0 * kBN;
+        pair_area += (double)ns_tiles(hu[ui].rows, hu[ui].cols, stg, 1) * 256.0 * kBN;
+      }
+      int pair = pair_area <= 1.15 * single_area ? 1 : 0;
+      if (forced_mode >= 0) pair = forced_mode;
+      wave_pair[wv * 3 + stg] = pair;
+      int pre = 0;
+      for (int ui = wave_begin[wv]; ui < wave_begin[wv + 1]; ++ui) {
+        hu[ui].tile_begin[stg] = pre;
+        hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg, pair);
+        pre += hu[ui].tile_count[stg];
       }
     }
   }
   cudaError_t e = upload_bytes(d_units, hu.data(), hu.size() * sizeof(NsUnit), s);
-  if (e != cudaSuccess) return SIGNMUON_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
 
   for (size_t wv = 0; wv + 1 < wave_begin.size(); ++wv) {
     const int u0 = wave_begin[wv], nu = wave_begin[wv + 1] - u0;
     if (k == 0) {
       e = launch_ns_identity(d_units + u0, nu, max_elems, (int)out_mode, (int)w_dtype, eta, s);
-      if (e != cudaSuccess) return SIGNMUON_ERR_CUDA;
+      if (e != cudaSuccess) return cuda_status(e);
       continue;
     }
     int total[3] = {0, 0, 0};
@@ -332,9 +373,10 @@ signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int
       for (int stg = 0; stg < 3; ++stg) {
         L.stage = stg;
         L.total_tiles = total[stg];
+        L.pair = wave_pair[wv * 3 + stg];
         L.out_kind = (stg == kStageApply && it == k - 1) ? (int)out_mode : (int)kOutIterate;
         e = launch_ns_gemm(L, s);
-        if (e != cudaSuccess) return SIGNMUON_ERR_CUDA;
+        if (e != cudaSuccess) return cuda_status(e);
       }
     }
   }

@@ -31,25 +31,23 @@ constexpr uint64_t kWaitTimeoutNs = 2000ull * 1000ull * 1000ull;  // 2 s
 // ---------------------------------------------------------------------------
 // Newton-Schulz GEMM tiling (tcgen05, one CTA per tile, cta_group::1).
 // ---------------------------------------------------------------------------
-constexpr int kBM = 128;          // MMA M (TMEM lanes)
 constexpr int kBN = 256;          // MMA N (TMEM fp32 columns per accumulator)
 constexpr int kBK = 64;           // K per stage: 64 bf16 = 128 B = one swizzle row
 constexpr int kUmmaK = 16;        // K per tcgen05.mma for kind::f16
-constexpr int kStages = 4;
 constexpr int kBoxRows = 64;      // every TMA box is 64 x 64 bf16 (8 KB)
 constexpr int kBoxBytes = 64 * 64 * 2;
-constexpr int kAStageBytes = kBM * kBK * 2;               // 16 KB
-constexpr int kBStageBytes = kBN * kBK * 2;               // 32 KB
-constexpr int kStageBytes = kAStageBytes + kBStageBytes;  // 48 KB
 constexpr int kAccCols = kBN;                             // fp32 columns per accumulator
 constexpr int kTmemCols = 2 * kAccCols;                   // double-buffered: 512
 constexpr int kEpilogueThreads = 256;                     // warps 2-9
 constexpr int kGemmThreads = 64 + kEpilogueThreads;       // warp 0 TMA, warp 1 MMA
 constexpr int kBarrierBytes = 256;
-constexpr int kXposeStride = 40;  // bf16 elements per row of a transpose buffer (80 B)
-constexpr int kXposeBytes = (kEpilogueThreads / 32) * 32 * kXposeStride * 2;  // 20 KB
-constexpr int kGemmSmemBytes = kStages * kStageBytes + kBarrierBytes + kXposeBytes + 1024 /*align*/;
-static_assert(kGemmSmemBytes <= 232448, "shared memory per CTA");
+// Epilogue output staging: two 32x32 bf16 blocks (2 KB each, 64-byte swizzle)
+// per epilogue warp, written to global memory by TMA stores.
+constexpr int kStageBlockBytes = 32 * 32 * 2;
+constexpr int kStagingBytes = (kEpilogueThreads / 32) * 2 * kStageBlockBytes;  // 32 KB
+
+// Output rows per tile: 128 for one CTA, 256 for a CTA pair.
+inline int ns_tile_m(int pair) { return pair ? 256 : 128; }
 
 enum NsStage : int { kStageGram = 0, kStageSquare = 1, kStageApply = 2 };
 
@@ -66,10 +64,16 @@ enum NsOut : int {
 // they stay 64-byte aligned (the struct is 64-byte aligned and a multiple
 // of 64 bytes long).
 struct alignas(64) NsUnit {
+  // Load maps: 64x64 boxes, 128-byte swizzle (GEMM operands).
   CUtensorMap map_x;     // caller's bf16 X buffer  [rows, ld_x]
   CUtensorMap map_xalt;  // workspace bf16 X buffer [rows, ld_x]
   CUtensorMap map_a;     // workspace Gram A        [s, ld_s]
   CUtensorMap map_b;     // workspace B' = aI + bA + cA^2 [s, ld_s]
+  // Store maps: 32x32 boxes, 64-byte swizzle (epilogue output blocks).
+  CUtensorMap st_x;
+  CUtensorMap st_xalt;
+  CUtensorMap st_a;
+  CUtensorMap st_b;
   __nv_bfloat16* x;
   __nv_bfloat16* xalt;
   __nv_bfloat16* a;
@@ -92,6 +96,7 @@ struct NsLaunch {
   int out_kind;     // NsOut: kOutIterate for non-final APPLY
   int w_dtype;      // for kOutUpdateW
   int total_tiles;
+  int pair;         // 1: CTA-pair (cta_group::2) 256x256 tiles; 0: one CTA, 128x256
   float a, b, c, eta;
   uint32_t* err;
 };
@@ -120,7 +125,7 @@ struct VoteMat {
   int32_t pad_;
 };
 
-static_assert(sizeof(NsUnit) == 640, "descriptor size is part of the launch-count bookkeeping");
+static_assert(sizeof(NsUnit) == 1152, "descriptor size is part of the launch-count bookkeeping");
 static_assert(sizeof(MomUnit) == 56, "descriptor size is part of the launch-count bookkeeping");
 static_assert(sizeof(VoteMat) == 64, "descriptor size is part of the launch-count bookkeeping");
 

@@ -11,10 +11,21 @@
 // written as packed bits or int8 (steps 2-3 of the summary's flow), or the
 // update W <- W - eta U (the optional local polar step, step 5).
 //
-// Roles (320 threads, one CTA per SM):
-//   warp 0     TMA producer: 64x64 bf16 boxes, 128-byte swizzle, 4 stages
-//   warp 1     MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128 N=256
-//              K=16, fp32 accumulators in TMEM, double-buffered (2 x 256 cols)
+// Two tile modes (chosen per launch by the host from the padding cost):
+//   single: one CTA per SM computes a 128x256 tile with
+//           tcgen05.mma.cta_group::1 (A 128 rows + B 256 rows per k-block,
+//           48 KB stages, 4 stages);
+//   pair:   a cluster of two CTAs on two SMs computes a 256x256 tile with
+//           tcgen05.mma.cta_group::2 issued by the even CTA; each CTA holds
+//           128 rows of A and 128 rows of B (32 KB stages, 6 stages), so each
+//           SM streams a third less operand data per FLOP and keeps more
+//           k-blocks in flight.  Each CTA loads its own halves (no TMA
+//           multicast); the odd CTA's copies complete on the even CTA's
+//           barrier.
+// Roles (320 threads per CTA):
+//   warp 0     TMA producer: 64x64 bf16 boxes, 128-byte swizzle
+//   warp 1     MMA issuer (even CTA of a pair): kind::f16, N=256, K=16,
+//              fp32 accumulators in TMEM, double-buffered (2 x 256 cols)
 //   warps 2-9  epilogue: tcgen05.ld 32x32b, fp32 math, stores (two warps per
 //              TMEM lane quadrant, one per half of the accumulator columns)
 // Every mbarrier wait is bounded; on timeout the kernel records an error
@@ -87,6 +98,65 @@ __device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const CUtensorMap
       : "memory");
 }
 
+// Pair mode: the copy completes on the barrier at `bar`, which may be the
+// even CTA's (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t smem_dst, const CUtensorMap* map, uint32_t bar,
+                                                 int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Bulk tensor store of a 32x32 block from shared memory (async proxy).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until this thread's bulk stores have read their shared-memory sources.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until this thread's bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Make this thread's shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_smem_to_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Byte offset of element (r, c) in a 32x32 bf16 staging block laid out as the
+// 64-byte TMA swizzle expects: 64-byte rows, 16-byte chunk index XOR-ed with
+// bits 1-2 of the row (the block base is 1 KB aligned).
+__device__ __forceinline__ uint32_t stage_off(int r, int c) {
+  return (uint32_t)(r * 64 + ((((c >> 3) ^ (r >> 1)) & 3) << 4) + (c & 7) * 2);
+}
+
 __device__ __forceinline__ void tensormap_acquire(const CUtensorMap* map) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(
                    reinterpret_cast<uint64_t>(map))
@@ -100,19 +170,56 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+template <bool kPair>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+  if constexpr (kPair)
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
 }
 
+template <bool kPair>
 __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if constexpr (kPair)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+template <bool kPair>
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_addr) {
+  if constexpr (kPair) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_addr),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_addr),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+}
+
+template <bool kPair>
+__device__ __forceinline__ void tmem_dealloc(uint32_t base) {
+  if constexpr (kPair)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(kTmemCols) : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(kTmemCols) : "memory");
 }
 
 // Issues a 32-lane x 32-column fp32 TMEM load; the registers are valid only
@@ -160,11 +267,27 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, int mn_major) {
   return d;
 }
 
-// Instruction descriptor: D fp32, A and B bf16, M = 128, N = 256.
-__device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn) {
+// Instruction descriptor: D fp32, A and B bf16, M = tile_m (128, or 256 for a
+// CTA pair), N = 256.
+__device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn, int tile_m) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+         ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(tile_m >> 4) << 24);
 }
+
+// Per-mode tile and pipeline shape.
+template <bool kPair>
+struct GemmCfg {
+  static constexpr int kTileM = kPair ? 256 : 128;  // output rows per tile
+  static constexpr int kRowsA = 128;                // A-operand rows held by one CTA
+  static constexpr int kRowsB = kPair ? 128 : 256;  // B-operand rows held by one CTA
+  static constexpr int kStageA = kRowsA * kBK * 2;
+  static constexpr int kStageB = kRowsB * kBK * 2;
+  static constexpr int kStageBytes = kStageA + kStageB;  // 32 KB or 48 KB
+  static constexpr int kStages = kPair ? 6 : 4;
+  static constexpr int kSmem = kStages * kStageBytes + kStagingBytes + kBarrierBytes + 1024 /*align*/;
+  static_assert(kSmem <= 232448, "shared memory per CTA");
+  static_assert((2 * kStages + 5) * 8 + 8 <= kBarrierBytes, "barrier area");
+};
 
 // ---------------------------------------------------------------------------
 // Tile scheduling.  Tiles of a launch are numbered unit by unit (each unit's
@@ -210,7 +333,7 @@ struct Tile {
 
 // Problem dimensions, operand majors and tile origin of local tile li of a
 // unit with the given shape.
-__device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li) {
+__device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, int tile_m) {
   const bool tall = rows > cols;
   const int s = tall ? cols : rows, l = tall ? rows : cols;
   Tile T;
@@ -227,10 +350,11 @@ __device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li) {
   int tm = 0, tn = 0;
   if (T.sym) {
     // Tiles entirely below the diagonal are skipped: row tile tm starts at
-    // column tile tm/2.
+    // column tile tm * tile_m / 256.
+    const int sh = tile_m == 256 ? 0 : 1;
     while (true) {
-      const int cnt = tiles_n - (tm >> 1);
-      if (li < cnt) { tn = (tm >> 1) + li; break; }
+      const int cnt = tiles_n - (tm >> sh);
+      if (li < cnt) { tn = (tm >> sh) + li; break; }
       li -= cnt;
       ++tm;
     }
@@ -238,7 +362,7 @@ __device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li) {
     tm = li / tiles_n;
     tn = li - tm * tiles_n;
   }
-  T.m0 = tm * kBM;
+  T.m0 = tm * tile_m;
   T.n0 = tn * kBN;
   return T;
 }
@@ -290,47 +414,47 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, bool vec, int nv
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
+template <bool kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ NsLaunch L) {
+  using C = GemmCfg<kPair>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Stage buffers must be 1 KB aligned for the 128-byte swizzle atoms.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* full_bar = bars;                   // [kStages]
-  uint64_t* empty_bar = bars + kStages;        // [kStages]
-  uint64_t* tfull_bar = bars + 2 * kStages;    // [2]
-  uint64_t* tempty_bar = bars + 2 * kStages + 2;  // [2]
-  uint64_t* drain_bar = bars + 2 * kStages + 4;   // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  // Layout: stage ring | epilogue staging (1 KB aligned) | barriers.
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + kStagingBytes);
+  uint64_t* full_bar = bars;                          // [kStages]
+  uint64_t* empty_bar = bars + C::kStages;            // [kStages]
+  uint64_t* tfull_bar = bars + 2 * C::kStages;        // [2]
+  uint64_t* tempty_bar = bars + 2 * C::kStages + 2;   // [2]
+  uint64_t* drain_bar = bars + 2 * C::kStages + 4;    // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // Per-epilogue-warp 32x32 transpose buffers (row stride 80 B: the 16-byte
-  // row reads of 8 consecutive lanes hit 8 distinct bank groups).
-  __nv_bfloat16* xpose = reinterpret_cast<__nv_bfloat16*>(smem + kStages * kStageBytes + kBarrierBytes);
+  // Per-epilogue-warp output staging: two 2 KB blocks (1 KB aligned).
+  uint8_t* staging = smem + C::kStages * C::kStageBytes;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Pair mode: rank 0 (even CTA) issues the MMAs; both CTAs load and drain.
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const int first_tile = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tile_stride = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(smem_addr(&full_bar[s]), 1);
       mbar_init(smem_addr(&empty_bar[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_addr(&tfull_bar[a]), 1);
-      mbar_init(smem_addr(&tempty_bar[a]), kEpilogueThreads);
+      mbar_init(smem_addr(&tempty_bar[a]), (kPair ? 2 : 1) * kEpilogueThreads);
     }
     mbar_init(smem_addr(drain_bar), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_addr(tmem_slot)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 1) tmem_alloc<kPair>(smem_addr(tmem_slot));
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -345,14 +469,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       UnitCursor cur;
       const CUtensorMap* ma = nullptr;
       const CUtensorMap* mb = nullptr;
-      for (int t = blockIdx.x; t < L.total_tiles && ok; t += gridDim.x) {
+      for (int t = first_tile; t < L.total_tiles && ok; t += tile_stride) {
         if (cursor_seek(L, cur, t)) {
           operand_maps(L, &L.units[cur.idx], cur.rows > cur.cols, ma, mb);
           tensormap_acquire(ma);
           tensormap_acquire(mb);
         }
-        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin);
+        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
         const int nkb = (T.K + kBK - 1) / kBK;
+        const int a_row0 = T.m0 + (int)rank * C::kRowsA;
+        const int b_row0 = T.n0 + (int)rank * C::kRowsB;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(smem_addr(&empty_bar[stage]), phase ^ 1, abort_flag)) {
             atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutProducer);
@@ -360,39 +486,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             ok = false;
             break;
           }
-          const uint32_t fb = smem_addr(&full_bar[stage]);
-          mbar_arrive_expect_tx(fb, kStageBytes);
-          const uint32_t sa = smem_addr(smem + stage * kStageBytes);
-          const uint32_t sb = sa + kAStageBytes;
+          const uint32_t own_full = smem_addr(&full_bar[stage]);
+          // Pair mode: both CTAs' copies complete on the even CTA's barrier,
+          // which the even CTA arms for both.
+          if (rank == 0) mbar_arrive_expect_tx(own_full, (kPair ? 2 : 1) * C::kStageBytes);
+          const uint32_t fb = kPair ? map_to_rank(own_full, 0) : own_full;
+          const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kStageA;
           const int k0 = kb * kBK;
 #pragma unroll
-          for (int j = 0; j < kBM / kBoxRows; ++j) {
-            const int mn = T.m0 + j * kBoxRows;
-            tma_load_2d(sa + j * kBoxBytes, ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
+          for (int j = 0; j < C::kRowsA / kBoxRows; ++j) {
+            const int mn = a_row0 + j * kBoxRows;
+            if constexpr (kPair)
+              tma_load_2d_pair(sa + j * kBoxBytes, ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
+            else
+              tma_load_2d(sa + j * kBoxBytes, ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
           }
 #pragma unroll
-          for (int j = 0; j < kBN / kBoxRows; ++j) {
-            const int mn = T.n0 + j * kBoxRows;
-            tma_load_2d(sb + j * kBoxBytes, mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
+          for (int j = 0; j < C::kRowsB / kBoxRows; ++j) {
+            const int mn = b_row0 + j * kBoxRows;
+            if constexpr (kPair)
+              tma_load_2d_pair(sb + j * kBoxBytes, mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
+            else
+              tma_load_2d(sb + j * kBoxBytes, mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
           }
           ++issued_kb;
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       UnitCursor cur;
-      for (int t = blockIdx.x; t < L.total_tiles && ok; t += gridDim.x) {
+      for (int t = first_tile; t < L.total_tiles && ok; t += tile_stride) {
         cursor_seek(L, cur, t);
-        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin);
-        const uint32_t idesc = instr_desc(T.a_mn, T.b_mn);
+        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
+        const uint32_t idesc = instr_desc(T.a_mn, T.b_mn, C::kTileM);
         const int nkb = (T.K + kBK - 1) / kBK;
         if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag)) {
           atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
@@ -409,24 +544,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_addr(smem + stage * kStageBytes);
-          const uint32_t sb = sa + kAStageBytes;
+          const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kStageA;
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
             const uint32_t aoff = T.a_mn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
             const uint32_t boff = T.b_mn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
-            tc_mma(tmem_d, smem_desc(sa + aoff, T.a_mn), smem_desc(sb + boff, T.b_mn), idesc,
-                   (kb | kk) != 0);
+            tc_mma<kPair>(tmem_d, smem_desc(sa + aoff, T.a_mn), smem_desc(sb + boff, T.b_mn), idesc,
+                          (kb | kk) != 0);
           }
-          tc_commit(smem_addr(&empty_bar[stage]));  // stage free once these MMAs finish
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          // The stage is free (in both CTAs of a pair) once these MMAs finish.
+          tc_commit<kPair>(smem_addr(&empty_bar[stage]));
+          if constexpr (kPair) tc_commit<kPair>(map_to_rank(smem_addr(&empty_bar[stage]), 1));
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(smem_addr(&tfull_bar[acc]));  // accumulator ready for the epilogue
+        // Accumulator ready for the epilogue (of both CTAs of a pair).
+        tc_commit<kPair>(smem_addr(&tfull_bar[acc]));
+        if constexpr (kPair) tc_commit<kPair>(map_to_rank(smem_addr(&tfull_bar[acc]), 1));
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
       // Drain: wait until every MMA this thread issued has completed.
-      tc_commit(smem_addr(drain_bar));
+      tc_commit<kPair>(smem_addr(drain_bar));
       if (!mbar_wait(smem_addr(drain_bar), 0, abort_flag)) {
         // Ignore the abort flag for the drain itself: wait out the full limit.
         const uint64_t t0 = global_timer_ns();
@@ -441,45 +580,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   } else {
     // ------------------------------------------------------------ epilogue
     // Two warps per TMEM lane quadrant: warp w reads lanes 32*(w%4).. and the
-    // column half (w-2)/4 of the accumulator.
+    // column half (w-2)/4 of the accumulator.  bf16 outputs (A, B', the next
+    // X) are staged per 32x32 block in shared memory and written by TMA
+    // stores (whole lines; rows/columns outside the matrix are dropped by the
+    // TMA); the other outputs are stored directly.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int row_in_tile = q * 32 + lane;
     constexpr int kChunks = kBN / 32 / 2;  // 32-column chunks per warp
+    uint8_t* stg0 = staging + (warp - 2) * 2 * kStageBlockBytes;
+    uint8_t* stg1 = stg0 + kStageBlockBytes;
+    const uint32_t stg0_s = smem_addr(stg0), stg1_s = smem_addr(stg1);
+    bool stores_pending = false;  // lane 0 of this warp has bulk stores in flight
     int acc = 0;
     uint32_t acc_phase = 0;
     UnitCursor cur;
     // The unit's fields are copied to registers once per unit: read through
     // a global pointer they would be reloaded after every store (aliasing).
     struct {
-      __nv_bfloat16* a;
-      __nv_bfloat16* b;
-      __nv_bfloat16* xout;
+      const __nv_bfloat16* a;
+      const CUtensorMap* st_out;  // store map of this stage's bf16 output
       void* out;
-      int ld_x, ld_s, cols;
-    } uf = {nullptr, nullptr, nullptr, nullptr, 0, 0, 0};
+      int ld_s, cols;
+    } uf = {nullptr, nullptr, nullptr, 0, 0};
     float s = 1.f;
-    for (int t = blockIdx.x; t < L.total_tiles; t += gridDim.x) {
+    for (int t = first_tile; t < L.total_tiles; t += tile_stride) {
       if (cursor_seek(L, cur, t)) {
         const NsUnit* un = &L.units[cur.idx];
         uf.a = un->a;
-        uf.b = un->b;
-        uf.xout = L.parity ? un->x : un->xalt;
+        uf.st_out = L.stage == kStageGram ? &un->st_a
+                  : L.stage == kStageSquare ? &un->st_b
+                  : (L.parity ? &un->st_x : &un->st_xalt);
         uf.out = un->out;
-        uf.ld_x = un->ld_x;
         uf.ld_s = un->ld_s;
         uf.cols = un->cols;
         s = L.first ? *un->scale : 1.f;
       }
-      const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin);
+      const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
       if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag)) {
         atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutEpilogue);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int grow = T.m0 + row_in_tile;
+      const int grow0 = T.m0 + (int)rank * 128 + q * 32;  // first row of this warp's 32-row block
+      const int grow = grow0 + lane;
       const bool row_ok = grow < T.M;
+      const bool bf16_out = T.sym || L.out_kind == kOutIterate;
       // Square stage: prefetch the A tile values of the first chunk.
       uint4 aux[4];
       const bool want_aux = (L.stage == kStageSquare) && row_ok;
@@ -505,7 +651,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         for (int j = 0; j < 32; ++j) raw[j] = nxt[j];
         // The next chunk's TMEM load overlaps this chunk's math and stores.
         if (cc + 1 < n_ch) tmem_ld32_async(tbase + (uint32_t)((ch + 1) * 32), nxt);
-        if (!row_ok) continue;
         const int nvalid = min(32, T.N - gc0);
         float v[32];
         if (L.stage == kStageGram) {
@@ -515,7 +660,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         } else if (L.stage == kStageSquare) {
           // B' = a I + b A + c A^2: folding a*I here lets the apply product
           // X' = B' X run without reading X a second time.
-          if (nvalid == 32) {
+          if (!row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          } else if (nvalid == 32) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               float av[8];
@@ -540,106 +688,127 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = s * __uint_as_float(raw[j]);
         }
-        if (T.sym) {
-          // Store the upper triangle (col >= row) and mirror it (col > row).
-          __nv_bfloat16* out = (L.stage == kStageGram) ? uf.a : uf.b;
-          const int ld = uf.ld_s;
-          const int grow0 = T.m0 + q * 32;  // first row of this warp's 32x32 block
-          if (gc0 >= grow) {
-            store_bf16x32(out + (int64_t)grow * ld + gc0, nvalid == 32, nvalid, v);
-          } else if (gc0 + 31 >= grow) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid && gc0 + j >= grow) out[(int64_t)grow * ld + gc0 + j] = __float2bfloat16_rn(v[j]);
-          }
-          if (gc0 >= grow0 + 32 && nvalid == 32 && grow0 + 32 <= T.M) {
-            // Whole block strictly above the diagonal (warp-uniform): stage it
-            // transposed in shared memory, then lane j writes row gc0 + j of
-            // the mirror with 16-byte stores.
-            __nv_bfloat16* tb = xpose + (warp - 2) * (32 * kXposeStride);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) tb[j * kXposeStride + lane] = __float2bfloat16_rn(v[j]);
-            __syncwarp();
-            const uint4* src = reinterpret_cast<const uint4*>(tb + lane * kXposeStride);
-            uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(gc0 + lane) * ld + grow0);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) dst[k] = src[k];
-            __syncwarp();
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid && gc0 + j > grow) out[(int64_t)(gc0 + j) * ld + grow] = __float2bfloat16_rn(v[j]);
-          }
-        } else if (L.out_kind == kOutIterate) {
-          store_bf16x32(uf.xout + (int64_t)grow * uf.ld_x + gc0, nvalid == 32, nvalid, v);
-        } else if (L.out_kind == kOutPack1) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) word |= (j < nvalid && !(v[j] < 0.f)) ? (1u << j) : 0u;
-          const int wpr = (uf.cols + 31) >> 5;
-          static_cast<uint32_t*>(uf.out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
-        } else if (L.out_kind == kOutInt8) {
-          int8_t* o = static_cast<int8_t*>(uf.out) + (int64_t)grow * uf.cols + gc0;
-          if (nvalid == 32 && (uf.cols & 15) == 0) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-              uint32_t x = 0;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) x |= (uint32_t)((v[4 * w + j] < 0.f) ? 0xFFu : 0x01u) << (8 * j);
-              pk[w] = x;
+        if (bf16_out) {
+          // Blocks to write (warp-uniform): a symmetric output stores the
+          // blocks above the diagonal together with their transposes, and
+          // each diagonal block once (made symmetric); the iterate stores
+          // every block.
+          const bool diag = T.sym && gc0 == grow0;
+          const bool mirror = T.sym && gc0 > grow0;
+          if (!T.sym || diag || mirror) {
+            if (stores_pending) {
+              if (lane == 0) bulk_wait_read_all();  // staging free again
+              __syncwarp();
             }
-            reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          } else {
+            if (!diag) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) o[j] = v[j] < 0.f ? int8_t(-1) : int8_t(1);
+              for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 h[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) h[j] = __floats2bfloat162_rn(v[8 * k + 2 * j], v[8 * k + 2 * j + 1]);
+                *reinterpret_cast<uint4*>(stg0 + stage_off(lane, 8 * k)) = *reinterpret_cast<const uint4*>(h);
+              }
+              if (mirror) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  *reinterpret_cast<__nv_bfloat16*>(stg1 + stage_off(j, lane)) = __float2bfloat16_rn(v[j]);
+              }
+            } else {
+              // Diagonal block: row `lane` supplies (lane, j >= lane) and, by
+              // symmetry, (j > lane, lane); together the whole block.
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+                if (j >= lane) *reinterpret_cast<__nv_bfloat16*>(stg0 + stage_off(lane, j)) = h;
+                if (j > lane) *reinterpret_cast<__nv_bfloat16*>(stg0 + stage_off(j, lane)) = h;
+              }
+            }
+            fence_smem_to_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(uf.st_out, stg0_s, gc0, grow0);
+              if (mirror) tma_store_2d(uf.st_out, stg1_s, grow0, gc0);
+              bulk_commit();
+            }
+            stores_pending = true;
           }
-        } else if (L.out_kind == kOutUF32) {
-          float* o = static_cast<float*>(uf.out) + (int64_t)grow * uf.cols + gc0;
-          if (nvalid == 32 && (uf.cols & 3) == 0) {
+        } else if (row_ok) {
+          if (L.out_kind == kOutPack1) {
+            uint32_t word = 0;
 #pragma unroll
-            for (int w = 0; w < 8; ++w)
-              reinterpret_cast<float4*>(o)[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
-          } else {
+            for (int j = 0; j < 32; ++j) word |= (j < nvalid && !(v[j] < 0.f)) ? (1u << j) : 0u;
+            const int wpr = (uf.cols + 31) >> 5;
+            static_cast<uint32_t*>(uf.out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
+          } else if (L.out_kind == kOutInt8) {
+            int8_t* o = static_cast<int8_t*>(uf.out) + (int64_t)grow * uf.cols + gc0;
+            if (nvalid == 32 && (uf.cols & 15) == 0) {
+              uint32_t pk[8];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) o[j] = v[j];
-          }
-        } else {  // kOutUpdateW: W <- W - eta * U
-          const int64_t off = (int64_t)grow * uf.cols + gc0;
-          if (L.w_dtype == SIGNMUON_BF16) {
-            __nv_bfloat16* w = static_cast<__nv_bfloat16*>(uf.out) + off;
+              for (int w = 0; w < 8; ++w) {
+                uint32_t x = 0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) w[j] = __float2bfloat16_rn(fmaf(-L.eta, v[j], __bfloat162float(w[j])));
-          } else {
-            float* w = static_cast<float*>(uf.out) + off;
+                for (int j = 0; j < 4; ++j) x |= (uint32_t)((v[4 * w + j] < 0.f) ? 0xFFu : 0x01u) << (8 * j);
+                pk[w] = x;
+              }
+              reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) o[j] = v[j] < 0.f ? int8_t(-1) : int8_t(1);
+            }
+          } else if (L.out_kind == kOutUF32) {
+            float* o = static_cast<float*>(uf.out) + (int64_t)grow * uf.cols + gc0;
+            if (nvalid == 32 && (uf.cols & 3) == 0) {
+#pragma unroll
+              for (int w = 0; w < 8; ++w)
+                reinterpret_cast<float4*>(o)[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) o[j] = v[j];
+            }
+          } else {  // kOutUpdateW: W <- W - eta * U
+            const int64_t off = (int64_t)grow * uf.cols + gc0;
+            if (L.w_dtype == SIGNMUON_BF16) {
+              __nv_bfloat16* w = static_cast<__nv_bfloat16*>(uf.out) + off;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) w[j] = __float2bfloat16_rn(fmaf(-L.eta, v[j], __bfloat162float(w[j])));
+            } else {
+              float* w = static_cast<float*>(uf.out) + off;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);
+            }
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_addr(&tempty_bar[acc]));
+      if constexpr (kPair)
+        mbar_arrive_cluster(map_to_rank(smem_addr(&tempty_bar[acc]), 0));  // the even CTA's barrier
+      else
+        mbar_arrive(smem_addr(&tempty_bar[acc]));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    // All of this warp's bulk stores must complete before the CTA exits.
+    if (lane == 0 && stores_pending) bulk_wait_all();
+    __syncwarp();
   }
 
   // ------------------------------------------------------------------ exit
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  if (warp == 0 && lane == 0) {
-    // Wait (bounded) for every TMA copy this CTA issued: the last phase armed
-    // on each stage's full barrier must have completed.
-    for (int s = 0; s < kStages; ++s) {
+  if (warp == 0 && lane == 0 && issued_kb > 0) {
+    // Wait (bounded) for every TMA copy this CTA issued.  The even CTA checks
+    // that the last phase armed on each stage's full barrier completed; the
+    // odd CTA (whose copies complete on the even CTA's barriers) waits until
+    // its last load of each stage has been consumed.
+    for (int s = 0; s < C::kStages; ++s) {
       if (issued_kb <= (uint32_t)s) continue;
-      const uint32_t last_round = (issued_kb - 1 - s) / kStages;
-      const uint32_t bar = smem_addr(&full_bar[s]);
+      const uint32_t last_round = (issued_kb - 1 - s) / C::kStages;
+      const uint32_t bar = rank == 0 ? smem_addr(&full_bar[s]) : smem_addr(&empty_bar[s]);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_test(bar, last_round & 1)) {
         if (global_timer_ns() - t0 > kWaitTimeoutNs) {
@@ -649,10 +818,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       }
     }
   }
+  tc_fence_before();
+  if constexpr (kPair) cluster_sync_all(); else __syncthreads();
+  tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
-                 : "memory");
+    tmem_dealloc<kPair>(tmem_base);
   }
 }
 
@@ -668,13 +839,35 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
     int n = 0;
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+    e = cudaFuncSetAttribute(ns_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<false>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(ns_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<true>::kSmem);
     if (e != cudaSuccess) return e;
     g_num_sms[dev] = n;
   }
-  const int grid = p.total_tiles < g_num_sms[dev] ? p.total_tiles : g_num_sms[dev];
-  ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  const int sms = g_num_sms[dev];
+  if (!p.pair) {
+    const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+    ns_gemm_kernel<false><<<grid, kGemmThreads, GemmCfg<false>::kSmem, stream>>>(p);
+    return cudaGetLastError();
+  }
+  // One cluster of two CTAs per pair tile worker.
+  const int pairs = p.total_tiles < sms / 2 ? p.total_tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = GemmCfg<true>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true>, p);
 }
 
 }  // namespace signmuon

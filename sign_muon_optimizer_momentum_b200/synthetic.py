@@ -80,6 +80,10 @@ WORKLOADS = {
     # ResNet-50 conv/FC matrices, fp32, M=4, k=1, int8 vote, noise ratio 1:2.
     "resnet50": Workload("resnet50", tuple(resnet50_shapes()), 4, 1, "int8", "f32",
                          g_noise_std=2.0, steps=10),
+    # Majority-vote Signum baseline (k = 0: the sign of the momentum itself) on
+    # the nanoGPT-small matrices, the comparison the SignMuon summary reports.
+    "signum_nanogpt_small": Workload("signum_nanogpt_small", tuple(nanogpt_small_shapes()), 8, 0,
+                                     "pack1", "bf16", g_noise_std=3.0, steps=10),
     # 32 square 4096^2 bf16 matrices, M=16, k=5, 1-bit vote, local polar step.
     "square4096x32": Workload("square4096x32", tuple([(4096, 4096)] * 32), 16, 5,
                               "pack1", "bf16", g_noise_std=4.0, steps=3, polar=True),

@@ -508,3 +508,51 @@ def test_vote_update_bf16_single_rounding_on_midpoint(int8_in):
     ref = O.apply_update(f64(w0), eta, signs.numpy(), "bf16")
     assert ref[0, 0] == 0.99609375
     assert np.array_equal(f64(w), ref)
+
+
+@pytest.mark.parametrize("shapes,M,k", [([(256, 256), (300, 700)], 2, 2), ([(768, 2304), (3072, 768)], 1, 3),
+                                        ([(64, 147), (513, 513)], 2, 1)])
+def test_single_and_pair_tile_modes_agree(shapes, M, k, monkeypatch):
+    """The one-CTA (128x256) and CTA-pair (256x256, cta_group::2) tile modes
+    compute the same products; both stay within the oracle tolerance."""
+    grads, moms = seeded_state(shapes, M, 13)
+    outs = {}
+    for mode in ("single", "pair"):
+        monkeypatch.setenv("SIGNMUON_NS_TILE_MODE", mode)
+        xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], 0.9,
+                               torch.float32)
+        us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+        gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, us)
+        outs[mode] = us
+    for u in range(len(grads)):
+        _, ref = oracle_u(moms[u], grads[u], 0.9, k)
+        for mode in ("single", "pair"):
+            assert rel_fro(f64(outs[mode][u]), ref) <= NS_TOL, (mode, shapes[u // M])
+        assert rel_fro(f64(outs["single"][u]), f64(outs["pair"][u])) <= 1e-2
+
+
+@pytest.mark.parametrize("variant,w_dtype,M", [("pack1", "bf16", 5), ("pack1", "f32", 4), ("int8", "f32", 3),
+                                               ("int8", "bf16", 8)])
+def test_signum_majority_vote_step_bit_exact(variant, w_dtype, M):
+    """k = 0: the Newton-Schulz output is X0 = M/||M||_F, whose sign is the
+    momentum's sign, so the step is the majority-vote Signum baseline the
+    SignMuon summary compares against (beta = 0 gives majority-vote SignSGD).
+    Momentum, vote and update are all exact, so the whole step is bit-exact."""
+    wl = syn.Workload("signum_small", ((64, 96), (96, 64), (33, 147), (128, 256)), M, 0, variant, w_dtype,
+                      g_noise_std=2.0)
+    for beta in (0.9, 0.0):
+        wl_b = syn.Workload(wl.name, wl.shapes, M, 0, variant, w_dtype, beta=beta, g_noise_std=2.0)
+        opt, weights = _run_steps(wl_b, 2)
+        w = [f64(x) for x in syn.initial_weights(wl_b, 0)]
+        moms = [[np.zeros(s) for _ in range(M)] for s in wl_b.shapes]
+        signal = syn.gradient_signal(wl_b, 0)
+        for t in range(2):
+            for i, shape in enumerate(wl_b.shapes):
+                grads = [f64(syn.worker_gradient(wl_b, signal[i], i, m, t, 0)) for m in range(M)]
+                ref = O.signmuon_step(w[i], grads, moms[i], beta=float(np.float32(beta)), eta=wl_b.eta, k=0,
+                                      w_dtype=w_dtype, int8_variant=(variant == "int8"))
+                moms[i], w[i] = ref["mom"], ref["w"]
+        for i in range(len(wl_b.shapes)):
+            assert np.array_equal(f64(weights[i]), w[i]), (beta, wl_b.shapes[i])
+            for m in range(M):
+                assert np.array_equal(f64(opt.mom[i * M + m]), moms[i][m])
