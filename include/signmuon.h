@@ -143,8 +143,9 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
  *   rows <= cols:  A = X X^T,  B = b A + c A^2,  X <- a X + B X
  *   rows >  cols:  A = X^T X,  B = b A + c A^2,  X <- a X + X B
  * on the tensor cores (bf16 operands, fp32 accumulation, bf16 between
- * iterations).  The kernels form B' = a I + b A + c A^2 (bf16) and compute
- * X <- B' X (X B'), the same map with the a X term folded into the product.
+ * iterations).  The kernels store A and P = b I + c A in fp16, form
+ * B' = a I + A P (= a I + b A + c A^2, bf16) and compute X <- B' X (X B'):
+ * the same map with the a X term folded into the product.
  * The last iteration's epilogue writes, per out_mode:
  *   PACK1:    out[u] = packed sign(U)   (uint32, signmuon_packed_words words)
  *   INT8:     out[u] = int8 sign(U)     ([rows, cols])

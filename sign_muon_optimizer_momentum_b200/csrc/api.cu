@@ -75,25 +75,29 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] with row stride ld elements.  Operand maps:
+// 2-D 16-bit tensor [outer, inner] (bf16, or fp16 for A and P) with row
+// stride ld elements.  Operand maps:
 // 64x64 boxes, 128-byte swizzle, zero fill outside the tensor.  Store maps:
 // 32x32 boxes, 64-byte swizzle (writes outside the tensor are dropped).
 bool encode_bf16_2d(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
-                    bool store_box = false) {
+                    bool store_box = false, bool fp16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
   cuuint32_t box[2] = {store_box ? 32u : 64u, store_box ? 32u : 64u};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, store_box ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ----------------------------------------------------------------- NS planning
+// Per-unit workspace: Gram A and P = bI + cA (s x s fp16), B' = aI + A P
+// (s x s bf16) and the second X iterate (bf16).
 struct UnitBytes {
-  size_t a, b, xalt, total;
+  size_t a, xalt, total;
 };
 
 UnitBytes ns_unit_bytes(signmuon_shape sh) {
@@ -101,9 +105,8 @@ UnitBytes ns_unit_bytes(signmuon_shape sh) {
   const int64_t ld_s = x_ld_of((int32_t)s);
   UnitBytes u;
   u.a = align_up((size_t)(s * ld_s * 2), 1024);
-  u.b = u.a;
   u.xalt = align_up((size_t)sh.rows * x_ld_of(sh.cols) * 2, 1024);
-  u.total = u.a + u.b + u.xalt;
+  u.total = 3 * u.a + u.xalt;
   return u;
 }
 
@@ -294,19 +297,22 @@ signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int
       u.ld_x = x_ld_of(cols);
       u.ld_s = x_ld_of(sdim);
       u.x = static_cast<__nv_bfloat16*>(x_bf16[ui]);
-      u.a = reinterpret_cast<__nv_bfloat16*>(arena + used);
+      u.a = arena + used;
       u.b = reinterpret_cast<__nv_bfloat16*>(arena + used + ub.a);
-      u.xalt = reinterpret_cast<__nv_bfloat16*>(arena + used + ub.a + ub.b);
+      u.p = arena + used + 2 * ub.a;
+      u.xalt = reinterpret_cast<__nv_bfloat16*>(arena + used + 3 * ub.a);
       used += ub.total;
       u.out = out_mode == SIGNMUON_OUT_UPDATE_W ? w[i] : out[ui];
       u.scale = inv_norm + ui;
       if (!encode_bf16_2d(&u.map_x, u.x, cols, rows, u.ld_x) ||
           !encode_bf16_2d(&u.map_xalt, u.xalt, cols, rows, u.ld_x) ||
-          !encode_bf16_2d(&u.map_a, u.a, sdim, sdim, u.ld_s) ||
+          !encode_bf16_2d(&u.map_a, u.a, sdim, sdim, u.ld_s, false, true) ||
           !encode_bf16_2d(&u.map_b, u.b, sdim, sdim, u.ld_s) ||
+          !encode_bf16_2d(&u.map_p, u.p, sdim, sdim, u.ld_s, false, true) ||
+          !encode_bf16_2d(&u.st_p, u.p, sdim, sdim, u.ld_s, true, true) ||
           !encode_bf16_2d(&u.st_x, u.x, cols, rows, u.ld_x, true) ||
           !encode_bf16_2d(&u.st_xalt, u.xalt, cols, rows, u.ld_x, true) ||
-          !encode_bf16_2d(&u.st_a, u.a, sdim, sdim, u.ld_s, true) ||
+          !encode_bf16_2d(&u.st_a, u.a, sdim, sdim, u.ld_s, true, true) ||
           !encode_bf16_2d(&u.st_b, u.b, sdim, sdim, u.ld_s, true))
         return SIGNMUON_ERR_UNSUPPORTED;
     }

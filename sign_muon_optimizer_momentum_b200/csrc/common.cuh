@@ -67,23 +67,26 @@ struct alignas(64) NsUnit {
   // Load maps: 64x64 boxes, 128-byte swizzle (GEMM operands).
   CUtensorMap map_x;     // caller's bf16 X buffer  [rows, ld_x]
   CUtensorMap map_xalt;  // workspace bf16 X buffer [rows, ld_x]
-  CUtensorMap map_a;     // workspace Gram A        [s, ld_s]
-  CUtensorMap map_b;     // workspace B' = aI + bA + cA^2 [s, ld_s]
+  CUtensorMap map_a;     // workspace Gram A (fp16)  [s, ld_s]
+  CUtensorMap map_b;     // workspace B' = aI + bA + cA^2 (bf16) [s, ld_s]
+  CUtensorMap map_p;     // workspace P = bI + cA (fp16) [s, ld_s]
   // Store maps: 32x32 boxes, 64-byte swizzle (epilogue output blocks).
   CUtensorMap st_x;
   CUtensorMap st_xalt;
   CUtensorMap st_a;
   CUtensorMap st_b;
+  CUtensorMap st_p;
   __nv_bfloat16* x;
   __nv_bfloat16* xalt;
-  __nv_bfloat16* a;
+  void* a;               // fp16
   __nv_bfloat16* b;
+  void* p;               // fp16
   void* out;             // final output (packed / int8 / fp32 U / W)
   const float* scale;    // &inv_norm[u]
   int32_t rows, cols, ld_x, ld_s;
   int32_t tile_begin[3];  // prefix of tiles over the launch's units, per stage
   int32_t tile_count[3];
-  int32_t pad_[4];
+  int32_t pad_[2];
 };
 static_assert(sizeof(NsUnit) % 64 == 0, "NsUnit must keep 64-byte alignment");
 
@@ -125,7 +128,7 @@ struct VoteMat {
   int32_t pad_;
 };
 
-static_assert(sizeof(NsUnit) == 1152, "descriptor size is part of the launch-count bookkeeping");
+static_assert(sizeof(NsUnit) == 1408, "descriptor size is part of the launch-count bookkeeping");
 static_assert(sizeof(MomUnit) == 56, "descriptor size is part of the launch-count bookkeeping");
 static_assert(sizeof(VoteMat) == 64, "descriptor size is part of the launch-count bookkeeping");
 

@@ -557,48 +557,76 @@ int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words) {
 }
 
 // ---------------------------------------------------------------------------
-// k = 0: the Newton-Schulz output is X0 itself.
+// k = 0: the Newton-Schulz output is X0 = s * X itself (s = inv_norm >= 0), so
+// its sign is the momentum's: the majority-vote Signum baseline.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void load_x32(const __nv_bfloat16* p, float s, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(p + 8 * q);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      v[8 * q + 2 * j] = s * f.x;
+      v[8 * q + 2 * j + 1] = s * f.y;
+    }
+  }
+}
+
+// One thread per 32-column segment of a row (one packed word).
 __global__ void __launch_bounds__(256)
 ns_identity_kernel(const NsUnit* __restrict__ units, int out_kind, int w_bf16, float eta) {
-  const NsUnit u = units[blockIdx.y];
-  const float s = *u.scale;
-  const int lane = threadIdx.x & 31;
-  if (out_kind == kOutPack1) {
-    const int wpr = (u.cols + 31) >> 5;
-    const int64_t n_words = (int64_t)u.rows * wpr;
-    const int64_t n_out = ((n_words + 3) / 4) * 4;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t w = warp; w < n_out; w += n_warps) {
-      uint32_t word = 0;
-      if (w < n_words) {
-        const int64_t r = w / wpr;
-        const int c = (int)(w - r * wpr) * 32 + lane;
-        bool bit = false;
-        if (c < u.cols) bit = !(s * __bfloat162float(u.x[r * u.ld_x + c]) < 0.f);
-        word = __ballot_sync(0xffffffffu, bit);
-      }
-      if (lane == 0) static_cast<uint32_t*>(u.out)[w] = word;
+  const NsUnit& un = units[blockIdx.y];
+  const int rows = un.rows, cols = un.cols, ld = un.ld_x;
+  const float s = *un.scale;
+  const int wpr = (cols + 31) >> 5;
+  const int64_t n_seg = (int64_t)rows * wpr;
+  const int64_t n_out = out_kind == kOutPack1 ? (n_seg + 3) / 4 * 4 : n_seg;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < n_out;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    if (w >= n_seg) {  // trailing pad words of a packed buffer
+      static_cast<uint32_t*>(un.out)[w] = 0u;
+      continue;
     }
-    return;
-  }
-  const int64_t n = (int64_t)u.rows * u.cols;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = e / u.cols, c = e - r * u.cols;
-    const float v = s * __bfloat162float(u.x[r * u.ld_x + c]);
-    if (out_kind == kOutInt8) {
-      static_cast<int8_t*>(u.out)[e] = v < 0.f ? int8_t(-1) : int8_t(1);
+    const int64_t r = w / wpr;
+    const int c0 = (int)(w - r * wpr) * 32;
+    const int nvalid = min(32, cols - c0);
+    const __nv_bfloat16* xp = un.x + r * ld + c0;
+    float v[32];
+    if (nvalid == 32) {
+      load_x32(xp, s, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = j < nvalid ? s * __bfloat162float(xp[j]) : 0.f;
+    }
+    const int64_t e0 = r * cols + c0;
+    if (out_kind == kOutPack1) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) word |= (j < nvalid && !(v[j] < 0.f)) ? (1u << j) : 0u;
+      static_cast<uint32_t*>(un.out)[w] = word;
+    } else if (out_kind == kOutInt8) {
+      int8_t* o = static_cast<int8_t*>(un.out) + e0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nvalid) o[j] = v[j] < 0.f ? int8_t(-1) : int8_t(1);
     } else if (out_kind == kOutUF32) {
-      static_cast<float*>(u.out)[e] = v;
+      float* o = static_cast<float*>(un.out) + e0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nvalid) o[j] = v[j];
     } else {  // kOutUpdateW
       if (w_bf16) {
-        __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u.out);
-        w[e] = __float2bfloat16_rn(__bfloat162float(w[e]) - eta * v);
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(un.out) + e0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) o[j] = __float2bfloat16_rn(__bfloat162float(o[j]) - eta * v[j]);
       } else {
-        float* w = static_cast<float*>(u.out);
-        w[e] = w[e] - eta * v;
+        float* o = static_cast<float*>(un.out) + e0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) o[j] = o[j] - eta * v[j];
       }
     }
   }
@@ -606,7 +634,9 @@ ns_identity_kernel(const NsUnit* __restrict__ units, int out_kind, int w_bf16, f
 
 cudaError_t launch_ns_identity(const NsUnit* units, int n_units, int64_t max_elems, int out_kind,
                                int w_dtype, float eta, cudaStream_t stream) {
-  dim3 grid((unsigned)grid_for(max_elems, 256, 1024), (unsigned)n_units);
+  // Segments per unit are at most max_elems / 32 + rows; size the x-grid for
+  // the largest unit (grid-stride covers the rest).
+  dim3 grid((unsigned)grid_for(max_elems / 32 + 1, 256, 512), (unsigned)n_units);
   ns_identity_kernel<<<grid, 256, 0, stream>>>(units, out_kind, w_dtype == SIGNMUON_BF16, eta);
   return cudaGetLastError();
 }

@@ -5,7 +5,9 @@
 // item 1: the momentum is orthogonalised toward its polar factor) over every
 // (matrix, worker) unit of a launch:
 //   stage Gram:   A = X X^T            (X^T X for tall X), symmetric output
-//   stage Square: B' = a I + b A + c A A   (A symmetric, so A A = A A^T)
+//   stage Square: B' = a I + A P           (P = b I + c A written by the Gram
+//                                            stage; A, P symmetric, stored in
+//                                            fp16 for the diagonal's sake)
 //   stage Apply:  X' = B' X            (X B' for tall X), i.e. a X + (b A + c A^2) X
 // with, in the last iteration, the entrywise sign fused into the epilogue and
 // written as packed bits or int8 (steps 2-3 of the summary's flow), or the
@@ -143,6 +145,10 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// Same, but the most recent group may still be reading.
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 // Wait until this thread's bulk stores have completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Make this thread's shared-memory writes visible to the async proxy (TMA).
@@ -150,7 +156,15 @@ __device__ __forceinline__ void fence_smem_to_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Byte offset of element (r, c) in a 32x32 bf16 staging block laid out as the
+// 16-bit conversions of the epilogue outputs (round to nearest even).
+__device__ __forceinline__ uint16_t to16(float x, bool half) {
+  return half ? __half_as_ushort(__float2half_rn(x)) : __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, bool half) {
+  return (uint32_t)to16(lo, half) | ((uint32_t)to16(hi, half) << 16);
+}
+
+// Byte offset of element (r, c) in a 32x32 16-bit staging block laid out as the
 // 64-byte TMA swizzle expects: 64-byte rows, 16-byte chunk index XOR-ed with
 // bits 1-2 of the row (the block base is 1 KB aligned).
 __device__ __forceinline__ uint32_t stage_off(int r, int c) {
@@ -267,10 +281,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, int mn_major) {
   return d;
 }
 
-// Instruction descriptor: D fp32, A and B bf16, M = tile_m (128, or 256 for a
-// CTA pair), N = 256.
-__device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn, int tile_m) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+// Instruction descriptor: D fp32, A and B both bf16 (or both fp16), M = tile_m
+// (128, or 256 for a CTA pair), N = 256.
+__device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn, int tile_m, bool fp16) {
+  const uint32_t fmt = fp16 ? 0u : 1u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(tile_m >> 4) << 24);
 }
 
@@ -374,7 +389,7 @@ __device__ __forceinline__ void operand_maps(const NsLaunch& L, const NsUnit* u,
   if (L.stage == kStageGram) {
     ma = xin; mb = xin;
   } else if (L.stage == kStageSquare) {
-    ma = &u->map_a; mb = &u->map_a;
+    ma = &u->map_a; mb = &u->map_p;  // A P, P = bI + cA symmetric (K-major rows)
   } else if (!tall) {
     ma = &u->map_b; mb = xin;
   } else {
@@ -527,7 +542,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       for (int t = first_tile; t < L.total_tiles && ok; t += tile_stride) {
         cursor_seek(L, cur, t);
         const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
-        const uint32_t idesc = instr_desc(T.a_mn, T.b_mn, C::kTileM);
+        // The square stage multiplies the fp16 A and P; all others are bf16.
+        const uint32_t idesc = instr_desc(T.a_mn, T.b_mn, C::kTileM, L.stage == kStageSquare);
         const int nkb = (T.K + kBK - 1) / kBK;
         if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag)) {
           atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
@@ -591,27 +607,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     uint8_t* stg1 = stg0 + kStageBlockBytes;
     const uint32_t stg0_s = smem_addr(stg0), stg1_s = smem_addr(stg1);
     bool stores_pending = false;  // lane 0 of this warp has bulk stores in flight
+    int stage_flip = 0;           // staging block of the next iterate store
     int acc = 0;
     uint32_t acc_phase = 0;
     UnitCursor cur;
     // The unit's fields are copied to registers once per unit: read through
     // a global pointer they would be reloaded after every store (aliasing).
     struct {
-      const __nv_bfloat16* a;
       const CUtensorMap* st_out;  // store map of this stage's bf16 output
+      const CUtensorMap* st_p;    // Gram stage: store map of P = bI + cA
       void* out;
-      int ld_s, cols;
-    } uf = {nullptr, nullptr, nullptr, 0, 0};
+      int cols;
+    } uf = {nullptr, nullptr, nullptr, 0};
     float s = 1.f;
     for (int t = first_tile; t < L.total_tiles; t += tile_stride) {
       if (cursor_seek(L, cur, t)) {
         const NsUnit* un = &L.units[cur.idx];
-        uf.a = un->a;
         uf.st_out = L.stage == kStageGram ? &un->st_a
                   : L.stage == kStageSquare ? &un->st_b
                   : (L.parity ? &un->st_x : &un->st_xalt);
+        uf.st_p = &un->st_p;
         uf.out = un->out;
-        uf.ld_s = un->ld_s;
         uf.cols = un->cols;
         s = L.first ? *un->scale : 1.f;
       }
@@ -626,16 +642,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       const int grow = grow0 + lane;
       const bool row_ok = grow < T.M;
       const bool bf16_out = T.sym || L.out_kind == kOutIterate;
-      // Square stage: prefetch the A tile values of the first chunk.
-      uint4 aux[4];
-      const bool want_aux = (L.stage == kStageSquare) && row_ok;
-      auto aux_ptr = [&](int ch) { return uf.a + (int64_t)grow * uf.ld_s + T.n0 + ch * 32; };
-      auto aux_vec = [&](int ch) { return T.n0 + ch * 32 + 32 <= T.N; };
-      if (want_aux && aux_vec(half * kChunks)) {
-        const uint4* p = reinterpret_cast<const uint4*>(aux_ptr(half * kChunks));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) aux[k] = p[k];
-      }
       // Chunks of this warp's column half that hold valid columns (warp-uniform).
       const int n_ch = max(0, min(kChunks, (T.N - T.n0 - half * kChunks * 32 + 31) / 32));
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
@@ -658,32 +664,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) * s2;
         } else if (L.stage == kStageSquare) {
-          // B' = a I + b A + c A^2: folding a*I here lets the apply product
-          // X' = B' X run without reading X a second time.
-          if (!row_ok) {
+          // B' = a I + A P with P = b I + c A, i.e. a I + b A + c A^2.
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.f;
-          } else if (nvalid == 32) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              float av[8];
-              unpack_bf16x8(aux[k], av);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) v[8 * k + j] = fmaf(L.b, av[j], L.c * __uint_as_float(raw[8 * k + j]));
-            }
-            if (cc + 1 < kChunks && aux_vec(ch + 1)) {
-              const uint4* p = reinterpret_cast<const uint4*>(aux_ptr(ch + 1));
-#pragma unroll
-              for (int k = 0; k < 4; ++k) aux[k] = p[k];
-            }
-          } else {
-            const __nv_bfloat16* p = aux_ptr(ch);
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              v[j] = fmaf(L.b, j < nvalid ? __bfloat162float(p[j]) : 0.f, L.c * __uint_as_float(raw[j]));
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] += (gc0 + j == grow) ? L.a : 0.f;  // diagonal of B'
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) + ((gc0 + j == grow) ? L.a : 0.f);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = s * __uint_as_float(raw[j]);
@@ -692,42 +675,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           // Blocks to write (warp-uniform): a symmetric output stores the
           // blocks above the diagonal together with their transposes, and
           // each diagonal block once (made symmetric); the iterate stores
-          // every block.
+          // every block.  The Gram stage writes two outputs: A, then
+          // P = b I + c A (from the fp32 value of A).
           const bool diag = T.sym && gc0 == grow0;
           const bool mirror = T.sym && gc0 > grow0;
-          if (!T.sym || diag || mirror) {
+          const int n_out = (L.stage == kStageGram) ? 2 : 1;
+          for (int o = 0; o < n_out && (!T.sym || diag || mirror); ++o) {
+            if (o == 1) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = fmaf(L.c, v[j], (gc0 + j == grow) ? L.b : 0.f);
+            }
+            const CUtensorMap* map = o == 0 ? uf.st_out : uf.st_p;
+            // The iterate alternates its two staging blocks, so only the
+            // store before last must have finished reading; symmetric
+            // outputs use both blocks per output.
+            uint8_t* dst = stg0;
+            uint32_t dst_s = stg0_s;
+            if (!T.sym && (stage_flip ^= 1)) { dst = stg1; dst_s = stg1_s; }
             if (stores_pending) {
-              if (lane == 0) bulk_wait_read_all();  // staging free again
+              if (lane == 0) {
+                if (T.sym) bulk_wait_read_all(); else bulk_wait_read_all_but_one();
+              }
               __syncwarp();
             }
+            // The Gram stage's A and P are fp16, everything else bf16.
+            const bool half_out = L.stage == kStageGram;
             if (!diag) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                __nv_bfloat162 h[4];
+                uint32_t w[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) h[j] = __floats2bfloat162_rn(v[8 * k + 2 * j], v[8 * k + 2 * j + 1]);
-                *reinterpret_cast<uint4*>(stg0 + stage_off(lane, 8 * k)) = *reinterpret_cast<const uint4*>(h);
+                for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
+                *reinterpret_cast<uint4*>(dst + stage_off(lane, 8 * k)) = make_uint4(w[0], w[1], w[2], w[3]);
               }
               if (mirror) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                  *reinterpret_cast<__nv_bfloat16*>(stg1 + stage_off(j, lane)) = __float2bfloat16_rn(v[j]);
+                  *reinterpret_cast<uint16_t*>(stg1 + stage_off(j, lane)) = to16(v[j], half_out);
               }
             } else {
               // Diagonal block: row `lane` supplies (lane, j >= lane) and, by
               // symmetry, (j > lane, lane); together the whole block.
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
-                const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
-                if (j >= lane) *reinterpret_cast<__nv_bfloat16*>(stg0 + stage_off(lane, j)) = h;
-                if (j > lane) *reinterpret_cast<__nv_bfloat16*>(stg0 + stage_off(j, lane)) = h;
+                const uint16_t h = to16(v[j], half_out);
+                if (j >= lane) *reinterpret_cast<uint16_t*>(stg0 + stage_off(lane, j)) = h;
+                if (j > lane) *reinterpret_cast<uint16_t*>(stg0 + stage_off(j, lane)) = h;
               }
             }
             fence_smem_to_async();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(uf.st_out, stg0_s, gc0, grow0);
-              if (mirror) tma_store_2d(uf.st_out, stg1_s, grow0, gc0);
+              tma_store_2d(map, dst_s, gc0, grow0);
+              if (mirror) tma_store_2d(map, stg1_s, grow0, gc0);
               bulk_commit();
             }
             stores_pending = true;

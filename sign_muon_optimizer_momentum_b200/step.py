@@ -174,7 +174,7 @@ class SignMuonStep:
         M = self.n_workers
         n_mats = len(self.shapes)
         mom = uploads(self.units * 56) + 2
-        unit_bytes = 1152
+        unit_bytes = 1408
         ns_waves = self._waves(self.shapes, M, self.ws_ns.numel())
         ns = uploads(self.units * unit_bytes) + (3 * self.k if self.k > 0 else 1) * ns_waves
         vote = uploads(n_mats * 64) + uploads(self.units * 8) + 1
@@ -189,12 +189,12 @@ class SignMuonStep:
         def al(x, a):
             return (x + a - 1) // a * a
         units = len(shapes) * M
-        arena = ws_bytes - 256 - al(units * 1152, 1024)
+        arena = ws_bytes - 256 - al(units * 1408, 1024)
         waves, used = 0, arena
         for (r, c) in shapes:
             s = min(r, c)
             lds = al(s, 8)
-            b = 2 * al(s * lds * 2, 1024) + al(r * al(c, 8) * 2, 1024)
+            b = 3 * al(s * lds * 2, 1024) + al(r * al(c, 8) * 2, 1024)
             for _ in range(M):
                 if used + b > arena:
                     waves += 1
