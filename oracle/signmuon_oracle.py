@@ -20,8 +20,8 @@ cited below as "SignMuon summary", by section:
   32x / 4x smaller than fp32);
 * §3 "Theory" (the normalisation bounds the spectral norm of the update
   direction by 1);
-* §4 "nanoGPT" hyper-parameter note (Frobenius scaling; one Newton-Schulz
-  iteration often suffices).
+* §4 "nanoGPT" hyper-parameter note (Frobenius vs spectral scaling; one
+  Newton-Schulz iteration often suffices).
 
 Readings where the summary is silent (each is a stated choice, not a fact of
 the pages): momentum is the EMA ``beta*M + (1-beta)*G``; the Newton-Schulz
@@ -117,6 +117,40 @@ def frobenius_normalize(mom, eps=NORM_EPS):
     """
     m = np.asarray(mom, dtype=np.float64)
     return m / (np.sqrt(np.sum(m * m)) + eps)
+
+
+# ---------------------------------------------------------------------------
+# Spectral scaling of the Newton-Schulz input (SignMuon summary, §4
+# "nanoGPT": the method is robust to Frobenius vs spectral scaling)
+# ---------------------------------------------------------------------------
+def spectral_norm_estimate(m, iters):
+    """Power-iteration estimate of the largest singular value of M.
+
+    The summary names spectral scaling but not how sigma_max is obtained; the
+    reading here is `iters` power iterations on M^T M from the unit start
+    vector v0 = 1/sqrt(n) (n = columns): z = M^T M v, v <- z / ||z||, and
+    sigma_est = sqrt(||z||) from the last step.  For a unit v,
+    ||M^T M v|| <= sigma_max^2, so the estimate never exceeds sigma_max and
+    converges to it as iters grows (for a start vector not orthogonal to the
+    top right singular vector).  A zero matrix gives 0.
+    """
+    m = np.asarray(m, dtype=np.float64)
+    n = m.shape[1]
+    v = np.full(n, 1.0 / np.sqrt(n))
+    z_norm = 0.0
+    for _ in range(max(int(iters), 1)):
+        z = m.T @ (m @ v)
+        z_norm = float(np.sqrt(np.sum(z * z)))
+        if z_norm == 0.0:
+            return 0.0
+        v = z / z_norm
+    return float(np.sqrt(z_norm))
+
+
+def spectral_normalize(mom, iters, eps=NORM_EPS):
+    """X0 = M / (sigma_est + eps) with sigma_est from spectral_norm_estimate."""
+    m = np.asarray(mom, dtype=np.float64)
+    return m / (spectral_norm_estimate(m, iters) + eps)
 
 
 # ---------------------------------------------------------------------------

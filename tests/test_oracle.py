@@ -345,3 +345,54 @@ def test_whole_step_invariants_small():
     z = O.signmuon_step(w, [np.zeros(shape)], [np.zeros(shape)], beta=0.9, eta=0.02,
                         k=3, w_dtype="f32")
     assert np.all(z["u"][0] == 0) and np.all(z["signs"][0] == 1)
+
+
+# --------------------------------------------------------------------------
+# Spectral scaling (power iteration)
+# --------------------------------------------------------------------------
+def test_power_iteration_converges_to_svd_sigma_max():
+    rng = _rng(20)
+    for shape in [(30, 20), (20, 30), (25, 25)]:
+        q1, _ = np.linalg.qr(rng.standard_normal((shape[0], shape[0])))
+        q2, _ = np.linalg.qr(rng.standard_normal((shape[1], shape[1])))
+        r = min(shape)
+        sig = np.concatenate([[3.0, 1.5], np.linspace(1.0, 0.1, r - 2)])
+        m = q1[:, :r] @ np.diag(sig) @ q2[:, :r].T
+        assert abs(O.spectral_norm_estimate(m, 60) - np.linalg.norm(m, 2)) < 1e-12
+        # Never above sigma_max, for any number of iterations.
+        for t in range(1, 8):
+            assert O.spectral_norm_estimate(m, t) <= np.linalg.norm(m, 2) * (1 + 1e-12)
+
+
+def test_power_iteration_closed_forms():
+    # Rank one u v^T: M^T M w = ||u||^2 (v.w) v, so one step from v0 gives
+    # sigma^2 = ||u||^2 ||v|| |v.v0| and every later step is exact, ||u|| ||v||.
+    rng = _rng(21)
+    u, v = rng.standard_normal(7), rng.standard_normal(5)
+    v0 = np.full(5, 1 / math.sqrt(5))
+    assert math.isclose(O.spectral_norm_estimate(np.outer(u, v), 1),
+                        math.sqrt(np.dot(u, u) * np.linalg.norm(v) * abs(np.dot(v, v0))), rel_tol=1e-13)
+    for t in (2, 3):
+        assert math.isclose(O.spectral_norm_estimate(np.outer(u, v), t), np.linalg.norm(u) * np.linalg.norm(v),
+                            rel_tol=1e-13)
+    # Diagonal D from v0 = 1/sqrt(n): after t steps sigma^2 = ||d^(2t)|| / ||d^(2t-2)||.
+    d = np.array([2.0, 1.5, 1.0, 0.5])
+    for t in (1, 2, 5):
+        expected = math.sqrt(np.linalg.norm(d ** (2 * t)) / np.linalg.norm(d ** (2 * t - 2)))
+        assert math.isclose(O.spectral_norm_estimate(np.diag(d), t), expected, rel_tol=1e-13)
+    # Scale equivariance and the zero matrix.
+    m = rng.standard_normal((6, 9))
+    assert math.isclose(O.spectral_norm_estimate(-3.0 * m, 4), 3.0 * O.spectral_norm_estimate(m, 4), rel_tol=1e-13)
+    assert O.spectral_norm_estimate(np.zeros((4, 4)), 3) == 0.0
+    assert np.all(O.spectral_normalize(np.zeros((4, 4)), 3) == 0)
+
+
+def test_spectral_scaling_bounds_normalised_direction():
+    """||X0||_2 = sigma_max / sigma_est >= 1 (slightly above 1 for a partly
+    converged estimate) and equal to 1 up to eps once converged."""
+    rng = _rng(22)
+    m = rng.standard_normal((40, 60))
+    x_conv = O.spectral_normalize(m, 200)
+    assert abs(np.linalg.norm(x_conv, 2) - 1.0) < 1e-6
+    x5 = O.spectral_normalize(m, 5)
+    assert 1.0 - 1e-6 <= np.linalg.norm(x5, 2) < 1.25
