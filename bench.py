@@ -292,7 +292,7 @@ def run_gpu(args, wl):
         return max_over_ranks_value(x, world, dev)
 
     opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
-                       polar=wl.polar, device=dev)
+                       polar=wl.polar, device=dev, norm=args.norm)
     weights = [w.to(dev) for w in syn.initial_weights(wl, rank)]
     signal = [g.to(dev) for g in syn.gradient_signal(wl, rank)]
     n_sets = 2
@@ -421,7 +421,7 @@ def run_gpu(args, wl):
     result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-              "config": dict(workload_config(wl), parallelism=f"replicas{world}",
+              "config": dict(workload_config(wl), parallelism=f"replicas{world}", norm=args.norm,
                              l2=f"inputs larger than L2 ({resident / 2**30:.1f} GiB gradients+momentum resident)"),
               "roofline": roofline, "e2e": e2e,
               "phases_ms": {"momentum": mom_ms, "newton_schulz": ns_ms, "vote_update": vote_ms},
@@ -532,6 +532,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--norm", default="frobenius", choices=["frobenius", "spectral"],
+                    help="scaling of the Newton-Schulz input (spectral: 5 power iterations)")
     args = ap.parse_args()
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
     if args.config == "vote_sweep":

@@ -135,6 +135,27 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
                                        void* stream);
 
 /* ------------------------------------------------------------------------
+ * Step 1a, spectral variant: spectral scaling of the Newton-Schulz input.
+ * Source: SignMuon summary, section 4 "nanoGPT" (the method is robust to
+ * Frobenius vs spectral scaling of the normalisation).
+ *
+ * For every unit, sigma_est is estimated by `iters` power iterations on
+ * X^T X, X = x_bf16[u] ([rows, signmuon_x_ld(cols)] bf16, as written by
+ * signmuon_momentum_norm), from the start vector v0 = 1/sqrt(cols):
+ *   z = X^T X v,  v <- z / ||z||,  sigma_est = sqrt(||z||) of the last step;
+ * then inv_norm[u] <- 1 / (sigma_est + 1e-7), replacing the Frobenius value
+ * so that signmuon_newton_schulz_batched starts from X0 = X / sigma_est.
+ * sigma_est never exceeds the largest singular value of X.  A zero matrix
+ * gives inv_norm = 1e7 (X0 = 0).  1 <= iters <= 1000.  Sums are taken in a
+ * fixed order (bit-reproducible run to run).
+ * workspace: device, >= signmuon_spectral_workspace_bytes(...) bytes.
+ * ---------------------------------------------------------------------- */
+size_t signmuon_spectral_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers);
+signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                       const void* const* x_bf16, int iters, float* inv_norm,
+                                       void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Step 1b-2: k Newton-Schulz iterations, then the entrywise sign.
  * Source: SignMuon summary, section 2 "Core mechanism" item 1 and
  * "Algorithmic flow" steps 1-2 (and step 5 for SIGNMUON_OUT_UPDATE_W).

@@ -40,6 +40,7 @@ EXPORTS = (
     "signmuon_newton_schulz_workspace_bytes", "signmuon_newton_schulz_batched",
     "signmuon_sign_pack", "signmuon_vote_workspace_bytes", "signmuon_vote_update",
     "signmuon_momentum_norm_noalloc", "signmuon_last_error_string",
+    "signmuon_spectral_workspace_bytes", "signmuon_spectral_norm",
 )
 
 
@@ -75,6 +76,8 @@ _SIGS = {
                                             _I, _PP, _I, _PP, _F, _P, _SZ, _P]),
     "signmuon_sign_pack": (_I, [Shape, _I, _P, ctypes.c_int64, _I, _P, _P]),
     "signmuon_vote_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I]),
+    "signmuon_spectral_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I]),
+    "signmuon_spectral_norm": (_I, [ctypes.POINTER(Shape), _I, _I, _PP, _I, _P, _P, _SZ, _P]),
     "signmuon_momentum_norm_noalloc": (_I, [ctypes.POINTER(Shape), _I, _I, _I, _PP, _PP, _F, _PP, _P, _P]),
     "signmuon_vote_update": (_I, [ctypes.POINTER(Shape), _I, _I, _I, _PP, _I, _PP, _F, _PP, _P, _P,
                                   _P, _SZ, _P]),
@@ -157,6 +160,16 @@ def signmuon_momentum_norm(shapes, n_workers, grad_dtype, grad, mom, beta, x_bf1
                                        _ptrs(mom), beta, _ptrs(x_bf16), inv_norm, workspace, ws_bytes,
                                        stream)
     _check("signmuon_momentum_norm", st)
+
+
+def signmuon_spectral_workspace_bytes(shapes, n_workers: int) -> int:
+    return load().signmuon_spectral_workspace_bytes(_shapes(shapes), len(shapes), n_workers)
+
+
+def signmuon_spectral_norm(shapes, n_workers, x_bf16, iters, inv_norm, workspace, ws_bytes, stream=0) -> None:
+    st = load().signmuon_spectral_norm(_shapes(shapes), len(shapes), n_workers, _ptrs(x_bf16), iters, inv_norm,
+                                       workspace, ws_bytes, stream)
+    _check("signmuon_spectral_norm", st)
 
 
 def signmuon_newton_schulz_workspace_bytes(shapes, n_workers: int, minimal: bool = False) -> int:

@@ -228,6 +228,74 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
   return cuda_status(e);
 }
 
+// ------------------------------------------------------------ spectral scaling
+static size_t spec_layout(const signmuon_shape* shapes, int n_mats, int n_workers, size_t* v_floats,
+                          size_t* part_floats) {
+  size_t vf = 0, pf = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const size_t cols4 = align_up((size_t)shapes[i].cols, 4);
+    const size_t n_rb = ((size_t)shapes[i].rows + kSpecRows - 1) / kSpecRows;
+    vf += cols4 * n_workers;
+    pf += n_rb * cols4 * n_workers;
+  }
+  *v_floats = vf;
+  *part_floats = pf;
+  const size_t units = (size_t)n_mats * n_workers;
+  return kWsHeaderBytes + align_up(units * sizeof(SpecUnit), 256) + align_up(vf * 4, 256) + align_up(pf * 4, 256);
+}
+
+size_t signmuon_spectral_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers) {
+  if (validate_shapes(shapes, n_mats) != SIGNMUON_OK || n_workers <= 0) return 0;
+  size_t vf, pf;
+  return spec_layout(shapes, n_mats, n_workers, &vf, &pf);
+}
+
+signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                       const void* const* x_bf16, int iters, float* inv_norm, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+  signmuon_status st = validate_shapes(shapes, n_mats);
+  if (st) return st;
+  if (n_workers <= 0 || n_workers > SIGNMUON_MAX_WORKERS) return SIGNMUON_ERR_INVALID_ARG;
+  if (iters < 1 || iters > 1000) return SIGNMUON_ERR_INVALID_ARG;
+  const int units = n_mats * n_workers;
+  if ((st = validate_ptrs(x_bf16, units))) return st;
+  if (!inv_norm) return SIGNMUON_ERR_INVALID_ARG;
+  if (!aligned16(inv_norm)) return SIGNMUON_ERR_ALIGNMENT;
+  size_t vf, pf;
+  const size_t need = spec_layout(shapes, n_mats, n_workers, &vf, &pf);
+  if ((st = check_workspace(workspace, ws_bytes, need))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<SpecUnit> hu(units);
+  int64_t voff = 0, poff = 0;
+  int blocks = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const int64_t cols4 = (int64_t)align_up((size_t)shapes[i].cols, 4);
+    const int n_rb = (shapes[i].rows + kSpecRows - 1) / kSpecRows;
+    for (int m = 0; m < n_workers; ++m) {
+      SpecUnit& u = hu[i * n_workers + m];
+      memset(&u, 0, sizeof(u));
+      u.x = static_cast<const __nv_bfloat16*>(x_bf16[i * n_workers + m]);
+      u.rows = shapes[i].rows;
+      u.cols = shapes[i].cols;
+      u.ld_x = x_ld_of(u.cols);
+      u.n_rb = n_rb;
+      u.v_off = voff;
+      u.part_off = poff;
+      u.block_begin = blocks;
+      voff += cols4;
+      poff += (int64_t)n_rb * cols4;
+      blocks += n_rb;
+    }
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  SpecUnit* d_units = reinterpret_cast<SpecUnit*>(ws + kWsHeaderBytes);
+  float* vecs = reinterpret_cast<float*>(ws + kWsHeaderBytes + align_up(units * sizeof(SpecUnit), 256));
+  float* parts = vecs + align_up(vf * 4, 256) / 4;
+  cudaError_t e = upload_bytes(d_units, hu.data(), hu.size() * sizeof(SpecUnit), s);
+  if (e == cudaSuccess) e = launch_spectral(d_units, units, blocks, vecs, parts, iters, inv_norm, s);
+  return cuda_status(e);
+}
+
 // ------------------------------------------------------------ Newton-Schulz
 size_t signmuon_newton_schulz_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers,
                                               int minimal) {

@@ -132,6 +132,20 @@ static_assert(sizeof(NsUnit) == 1408, "descriptor size is part of the launch-cou
 static_assert(sizeof(MomUnit) == 56, "descriptor size is part of the launch-count bookkeeping");
 static_assert(sizeof(VoteMat) == 64, "descriptor size is part of the launch-count bookkeeping");
 
+// Spectral-scaling units (power iteration on X^T X).
+struct SpecUnit {
+  const __nv_bfloat16* x;
+  int64_t v_off;        // float offset of this unit's vector v (cols entries)
+  int64_t part_off;     // float offset of its partial sums [n_rb][cols]
+  int32_t rows, cols, ld_x;
+  int32_t n_rb;         // row blocks of kSpecRows rows
+  int32_t block_begin;  // first row block of this unit in the flattened grid
+  int32_t pad_;
+};
+static_assert(sizeof(SpecUnit) == 48, "descriptor size");
+constexpr int kSpecRows = 32;
+constexpr int kSpecSmemCols = 8192;  // v is staged in shared memory up to this many columns (32 KB)
+
 // ---------------------------------------------------------------------------
 // Launch helpers implemented in the .cu files (all enqueue on `stream`).
 // ---------------------------------------------------------------------------
@@ -148,6 +162,8 @@ cudaError_t launch_vote(const VoteMat* mats, int n_mats, int total_blocks, const
 cudaError_t launch_vote_inv(const int64_t* nnz, float* inv, int n_mats, cudaStream_t stream);
 int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words);
 cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream);
+cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, float* vecs, float* parts,
+                            int iters, float* inv_norm, cudaStream_t stream);
 cudaError_t launch_ns_identity(const NsUnit* units, int n_units, int64_t max_elems, int out_kind,
                                int w_dtype, float eta, cudaStream_t stream);
 

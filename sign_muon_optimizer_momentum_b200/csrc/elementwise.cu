@@ -557,6 +557,143 @@ int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words) {
 }
 
 // ---------------------------------------------------------------------------
+// Spectral scaling: sigma_est of each unit's X by power iteration on X^T X
+// from v0 = 1/sqrt(n); inv_norm = 1 / (sigma_est + 1e-7).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int find_spec_unit(const SpecUnit* u, int n, int b) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (u[mid].block_begin <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void spectral_init_kernel(const SpecUnit* __restrict__ units, float* __restrict__ vecs) {
+  const SpecUnit u = units[blockIdx.x];
+  const float v0 = (float)(1.0 / sqrt((double)u.cols));
+  for (int j = threadIdx.x; j < u.cols; j += blockDim.x) vecs[u.v_off + j] = v0;
+}
+
+// One block per 32 rows of one unit: y_r = x_r . v for its rows, then the
+// partial z_j = sum_r y_r x_rj of the block (rows re-read from L1/L2).
+__global__ void __launch_bounds__(256, 4)
+spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const float* __restrict__ vecs,
+                        float* __restrict__ parts) {
+  const int b = blockIdx.x;
+  const SpecUnit u = units[find_spec_unit(units, n_units, b)];
+  const int rb = b - u.block_begin;
+  const int r0 = rb * kSpecRows;
+  const int nrows = min(kSpecRows, u.rows - r0);
+  const float* vg = vecs + u.v_off;
+  __shared__ float ys[kSpecRows];
+  extern __shared__ float4 v_smem4[];  // v staged in shared memory (cols floats)
+  float* vs = reinterpret_cast<float*>(v_smem4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool vec = (u.cols & 7) == 0;
+  const bool staged = u.cols <= kSpecSmemCols;
+  if (staged)
+    for (int j = threadIdx.x; j < u.cols; j += blockDim.x) vs[j] = vg[j];
+  __syncthreads();
+  const float* v = staged ? vs : vg;
+  for (int rr = warp; rr < kSpecRows; rr += 8) {
+    float acc = 0.f;
+    if (rr < nrows) {
+      const __nv_bfloat16* xr = u.x + (int64_t)(r0 + rr) * u.ld_x;
+      if (vec) {
+        for (int j = lane * 8; j < u.cols; j += 256) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(xr + j);
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          const float4 va = *reinterpret_cast<const float4*>(v + j);
+          const float4 vb = *reinterpret_cast<const float4*>(v + j + 4);
+          const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h[q]);
+            acc = fmaf(f.x, vv[2 * q], acc);
+            acc = fmaf(f.y, vv[2 * q + 1], acc);
+          }
+        }
+      } else {
+        for (int j = lane; j < u.cols; j += 32) acc = fmaf(__bfloat162float(xr[j]), v[j], acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) ys[rr] = acc;
+  }
+  __syncthreads();
+  float* part = parts + u.part_off + (int64_t)rb * u.cols;
+  if (vec) {
+    for (int j = threadIdx.x * 8; j < u.cols; j += 256 * 8) {
+      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int rr = 0; rr < nrows; ++rr) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(u.x + (int64_t)(r0 + rr) * u.ld_x + j);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        const float y = ys[rr];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h[q]);
+          z[2 * q] = fmaf(y, f.x, z[2 * q]);
+          z[2 * q + 1] = fmaf(y, f.y, z[2 * q + 1]);
+        }
+      }
+      *reinterpret_cast<float4*>(part + j) = make_float4(z[0], z[1], z[2], z[3]);
+      *reinterpret_cast<float4*>(part + j + 4) = make_float4(z[4], z[5], z[6], z[7]);
+    }
+  } else {
+    for (int j = threadIdx.x; j < u.cols; j += 256) {
+      float z = 0.f;
+      for (int rr = 0; rr < nrows; ++rr) z = fmaf(ys[rr], __bfloat162float(u.x[(int64_t)(r0 + rr) * u.ld_x + j]), z);
+      part[j] = z;
+    }
+  }
+}
+
+// One block per unit: z = sum of the row-block partials (fixed order),
+// v <- z / ||z||; after the last iteration inv_norm = 1 / (sqrt(||z||) + eps).
+__global__ void __launch_bounds__(256)
+spectral_reduce_kernel(const SpecUnit* __restrict__ units, float* __restrict__ vecs, const float* __restrict__ parts,
+                       int last, float* __restrict__ inv_norm) {
+  const SpecUnit u = units[blockIdx.x];
+  float* v = vecs + u.v_off;
+  const float* part = parts + u.part_off;
+  double ss = 0.0;
+  for (int j = threadIdx.x; j < u.cols; j += blockDim.x) {
+    float z = 0.f;
+    for (int rb = 0; rb < u.n_rb; ++rb) z += part[(int64_t)rb * u.cols + j];
+    v[j] = z;
+    ss += (double)z * (double)z;
+  }
+  __shared__ double red[256];
+  red[threadIdx.x] = ss;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  const double zn = sqrt(red[0]);
+  const float scale = zn > 0.0 ? (float)(1.0 / zn) : 0.f;
+  for (int j = threadIdx.x; j < u.cols; j += blockDim.x) v[j] *= scale;
+  if (last && threadIdx.x == 0) inv_norm[blockIdx.x] = (float)(1.0 / (sqrt(zn) + 1e-7));
+}
+
+cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, float* vecs, float* parts,
+                            int iters, float* inv_norm, cudaStream_t stream) {
+  spectral_init_kernel<<<n_units, 256, 0, stream>>>(units, vecs);
+  cudaError_t e = cudaGetLastError();
+  for (int it = 0; it < iters && e == cudaSuccess; ++it) {
+    spectral_rowpass_kernel<<<total_row_blocks, 256, kSpecSmemCols * sizeof(float), stream>>>(units, n_units,
+                                                                                             vecs, parts);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) break;
+    spectral_reduce_kernel<<<n_units, 256, 0, stream>>>(units, vecs, parts, it == iters - 1, inv_norm);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+// ---------------------------------------------------------------------------
 // k = 0: the Newton-Schulz output is X0 = s * X itself (s = inv_norm >= 0), so
 // its sign is the momentum's: the majority-vote Signum baseline.
 // ---------------------------------------------------------------------------

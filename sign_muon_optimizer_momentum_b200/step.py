@@ -54,14 +54,20 @@ class SignMuonStep:
     k:         Newton-Schulz iterations
     variant:   "pack1" (1-bit packed signs) or "int8" (integer-sum vote)
     polar:     run the optional local polar step on the voted matrix
+    norm:      "frobenius" (X0 = M / ||M||_F) or "spectral" (X0 = M / sigma_est,
+               sigma_est from `spectral_iters` power iterations)
     """
 
     def __init__(self, shapes: Sequence[Tuple[int, int]], n_workers: int, k: int, variant: str,
                  beta: float, eta: float, w_dtype: torch.dtype, polar: bool = False,
                  coeffs=NS_QUINTIC, device: Optional[torch.device] = None,
-                 ns_workspace_cap: int = 16 << 30):
+                 ns_workspace_cap: int = 16 << 30, norm: str = "frobenius", spectral_iters: int = 5):
         if variant not in ("pack1", "int8"):
             raise ValueError("variant must be 'pack1' or 'int8'")
+        if norm not in ("frobenius", "spectral"):
+            raise ValueError("norm must be 'frobenius' or 'spectral'")
+        self.norm = norm
+        self.spectral_iters = int(spectral_iters)
         L.load()
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.n_workers = int(n_workers)
@@ -96,6 +102,9 @@ class SignMuonStep:
         self.ws_ns = torch.empty(max(minimal, min(full, ns_workspace_cap)), dtype=torch.uint8, device=dev)
         self.ws_vote = torch.empty(L.signmuon_vote_workspace_bytes(self.shapes, M), dtype=torch.uint8,
                                    device=dev)
+        if self.norm == "spectral":
+            self.ws_spec = torch.empty(L.signmuon_spectral_workspace_bytes(self.shapes, M), dtype=torch.uint8,
+                                       device=dev)
         if self.polar:
             self.vote = [torch.empty((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device=dev)
                          for (r, c) in self.shapes]
@@ -126,6 +135,10 @@ class SignMuonStep:
                                  [m.data_ptr() for m in self.mom], self.beta,
                                  [x.data_ptr() for x in self.x], self.inv_norm.data_ptr(),
                                  self.ws_mom.data_ptr(), self.ws_mom.numel(), stream)
+        if self.norm == "spectral":
+            L.signmuon_spectral_norm(self.shapes, self.n_workers, [x.data_ptr() for x in self.x],
+                                     self.spectral_iters, self.inv_norm.data_ptr(), self.ws_spec.data_ptr(),
+                                     self.ws_spec.numel(), stream)
 
     def newton_schulz(self, stream: int, out_mode: Optional[int] = None, outs=None) -> None:
         if out_mode is None:
@@ -174,6 +187,8 @@ class SignMuonStep:
         M = self.n_workers
         n_mats = len(self.shapes)
         mom = uploads(self.units * 56) + 2
+        if self.norm == "spectral":
+            mom += uploads(self.units * 48) + 1 + 2 * self.spectral_iters
         unit_bytes = 1408
         ns_waves = self._waves(self.shapes, M, self.ws_ns.numel())
         ns = uploads(self.units * unit_bytes) + (3 * self.k if self.k > 0 else 1) * ns_waves

@@ -105,6 +105,12 @@ def test_argument_validation_returns_status(lib):
     assert _err(L.signmuon_sign_pack, (4, 8), 3, fake, 8, 0, fake) == 1      # bad dtype
     assert _err(L.signmuon_sign_pack, (4, 8), 0, odd, 8, 0, fake) == 2
     assert _err(L.signmuon_sign_pack, (0, 8), 0, fake, 8, 0, fake) == 1
+    # Spectral scaling.
+    sp = L.signmuon_spectral_norm
+    assert _err(sp, shp, 1, [fake], 0, fake, fake, 1 << 20) == 1          # iters < 1
+    assert _err(sp, shp, 1, [odd], 3, fake, fake, 1 << 20) == 2
+    assert _err(sp, shp, 1, [fake], 3, fake, fake, 64) == 4
+    assert _err(sp, shp, 0, [fake], 3, fake, fake, 1 << 20) == 1
     # Vote.
     vu = L.signmuon_vote_update
     assert _err(vu, shp, 0, 0, [], 0, [fake], 0.01, None, 0, 0, fake, 1 << 20) == 1

@@ -556,3 +556,183 @@ def test_signum_majority_vote_step_bit_exact(variant, w_dtype, M):
             assert np.array_equal(f64(weights[i]), w[i]), (beta, wl_b.shapes[i])
             for m in range(M):
                 assert np.array_equal(f64(opt.mom[i * M + m]), moms[i][m])
+
+
+# ---------------------------------------------------------------------------
+# spectral scaling (power iteration)
+# ---------------------------------------------------------------------------
+SPEC_CASES = [([(256, 256)], 2, 5), ([(128, 384), (384, 128)], 2, 3), ([(64, 147), (33, 20)], 3, 1),
+              ([(768, 2304), (3072, 768)], 1, 5), ([(1, 1), (1, 40), (40, 1)], 2, 2)]
+
+
+def gpu_spectral(shapes, M, xs, inv, iters):
+    w = ws(L.signmuon_spectral_workspace_bytes(shapes, M))
+    L.signmuon_spectral_norm(shapes, M, [x.data_ptr() for x in xs], iters, inv.data_ptr(), w.data_ptr(), w.numel(),
+                             stream())
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("shapes,M,iters", SPEC_CASES)
+def test_spectral_norm_matches_oracle(shapes, M, iters):
+    grads, moms = seeded_state(shapes, M, 17)
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9, torch.float32)
+    gpu_spectral(shapes, M, xs, inv, iters)
+    for u in range(len(xs)):
+        m, _ = oracle_u(moms[u], grads[u], 0.9, 0)
+        # Same bf16 input as the kernel (rounded by the oracle itself): only
+        # the summation order differs.
+        ref_bf = 1.0 / (O.spectral_norm_estimate(O.round_to_bf16(m), iters) + O.NORM_EPS)
+        assert math.isclose(inv[u].item(), ref_bf, rel_tol=2e-4), (shapes[u // M], inv[u].item(), ref_bf)
+        ref = 1.0 / (O.spectral_norm_estimate(m, iters) + O.NORM_EPS)
+        assert math.isclose(inv[u].item(), ref, rel_tol=5e-3)
+
+
+def test_spectral_zero_matrix_and_ns_parity():
+    shapes, M, iters, k = [(96, 300), (300, 96)], 2, 5, 5
+    z = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
+    xs, inv = gpu_momentum(shapes, M, z, [torch.zeros_like(t) for t in z], 0.9, torch.float32)
+    gpu_spectral(shapes, M, xs, inv, iters)
+    assert torch.allclose(inv, torch.full_like(inv, 1e7))
+    grads, moms = seeded_state(shapes, M, 19)
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9, torch.float32)
+    gpu_spectral(shapes, M, xs, inv, iters)
+    us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, us)
+    for u in range(len(xs)):
+        m, _ = oracle_u(moms[u], grads[u], 0.9, 0)
+        ref = O.newton_schulz(O.spectral_normalize(m, iters), k)
+        got = f64(us[u])
+        assert rel_fro(got, ref) <= NS_TOL
+        big = np.abs(ref) > 1e-3
+        assert np.mean(np.sign(got[big]) == np.sign(ref[big])) >= SIGN_AGREE
+
+
+def test_spectral_step_runs_and_is_deterministic():
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    wl = syn.Workload("spec", ((96, 160), (160, 96)), 3, 3, "pack1", "bf16", g_noise_std=2.0)
+    results = []
+    for _ in range(2):
+        opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, torch.bfloat16,
+                           norm="spectral", spectral_iters=4)
+        weights = [w.cuda() for w in syn.initial_weights(wl, 0)]
+        signal = syn.gradient_signal(wl, 0)
+        grads = [syn.worker_gradient(wl, signal[i], i, m, 0, 0).cuda() for i in range(2) for m in range(3)]
+        opt.step(weights, grads)
+        torch.cuda.synchronize()
+        results.append([w.clone() for w in weights])
+    for a, b in zip(*results):
+        assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads (sampled outputs), in the launch configuration bench.py times
+# ---------------------------------------------------------------------------
+@pytest.mark.slow
+def test_resnet50_full_size_sampled_parity():
+    """ResNet-50 shapes at full size (54 matrices, M = 4, k = 1, int8 vote):
+    momentum of every unit bit-exact, Newton-Schulz of a sample of units
+    within tolerance, and the vote + update of sampled matrices bit-exact
+    wherever the oracle's vote is not marginal."""
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    wl = syn.WORKLOADS["resnet50"]
+    M = wl.n_workers
+    opt = SignMuonStep(wl.shapes, M, wl.ns_iters, wl.variant, wl.beta, wl.eta, torch.float32)
+    w0 = syn.initial_weights(wl, 0)
+    weights = [w.cuda() for w in w0]
+    signal = syn.gradient_signal(wl, 0)
+    grads = [syn.worker_gradient(wl, signal[i], i, m, 0, 0) for i in range(len(wl.shapes)) for m in range(M)]
+    opt.step(weights, [g.cuda() for g in grads])
+    torch.cuda.synchronize()
+    beta = float(np.float32(wl.beta))
+    for u, g in enumerate(grads):
+        assert np.array_equal(f64(opt.mom[u]), O.momentum_update(np.zeros(g.shape), f64(g), beta))
+    for i in (0, 7, 20, 40, 53):   # 64x147, 128x1152-class, 1024x256, 512x2048-class, 2048x1000
+        r, c = wl.shapes[i]
+        ref_signs = []
+        for m in range(M):
+            mom = O.momentum_update(np.zeros((r, c)), f64(grads[i * M + m]), beta)
+            U = O.newton_schulz(O.frobenius_normalize(mom), wl.ns_iters)
+            s_gpu = opt.signs[i * M + m].cpu().numpy()
+            big = np.abs(U) > 1e-3
+            if big.sum():
+                assert np.mean(s_gpu[big] == O.sign_entries(U)[big]) >= SIGN_AGREE
+            ref_signs.append(O.sign_entries(U))
+        ref_w = O.apply_update(f64(w0[i]), wl.eta, O.majority_vote(ref_signs), "f32")
+        same = f64(weights[i]) == ref_w
+        total = sum(s.astype(np.int64) for s in ref_signs)
+        marginal = np.abs(total) <= 2
+        assert np.all(same | marginal), (wl.shapes[i], np.mean(same))
+
+
+@pytest.mark.slow
+def test_square4096_batch_full_size_sampled():
+    """32 x 4096^2, M = 16, k = 5, 1-bit vote and local polar step, at full
+    size: sampled momentum bit-exact, sampled Newton-Schulz signs against the
+    fp64 oracle, and the vote matrix and polar update consistent with the
+    step's own packed signs (majority count, Frobenius scale, bounded
+    update)."""
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    wl = syn.WORKLOADS["square4096x32"]
+    M = wl.n_workers
+    dt = torch.bfloat16
+    opt = SignMuonStep(wl.shapes, M, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt, polar=True)
+    weights = [w.cuda() for w in syn.initial_weights(wl, 0, device="cpu")]
+    w_before = weights[3].clone()
+    signal = [g.cuda() for g in syn.gradient_signal(wl, 0, device="cuda")]
+    grads = [torch.empty(s, dtype=dt, device="cuda") for s in wl.shapes for _ in range(M)]
+    for i in range(len(wl.shapes)):
+        for m in range(M):
+            syn.worker_gradient(wl, signal[i], i, m, 0, 0, out=grads[i * M + m])
+    opt.step(weights, grads)
+    torch.cuda.synchronize()
+    beta = float(np.float32(wl.beta))
+    u = 3 * M + 5
+    mom = O.momentum_update(np.zeros((4096, 4096)), f64(grads[u]), beta)
+    assert np.array_equal(f64(opt.mom[u]), mom)
+    U = O.newton_schulz(O.frobenius_normalize(mom), wl.ns_iters)
+    s_gpu = unpack_words(opt.signs[u].cpu().numpy().view(np.uint32), 4096, 4096)
+    big = np.abs(U) > 1e-3
+    assert np.mean(s_gpu[big] == O.sign_entries(U)[big]) >= SIGN_AGREE
+    # The vote matrix of matrix 3 is the majority of the step's own signs.
+    count = sum((unpack_words(opt.signs[3 * M + m].cpu().numpy().view(np.uint32), 4096, 4096) == 1)
+                .astype(np.int64) for m in range(M))
+    vote = np.sign(2 * count - M)
+    assert np.array_equal(f64(opt.vote[3])[:, :4096], vote)
+    assert opt.nnz[3].item() == np.count_nonzero(vote)
+    # Polar update: ||V / sqrt(nnz)||_2 <= 1, so every entry of U_V is at most
+    # phi's maximum 1.2024 in magnitude, and |dW| <= eta * 1.2024 plus the
+    # bf16 rounding of W (at most 1 ulp <= |W| 2^-7).
+    dw = f64(weights[3]) - f64(w_before)
+    assert np.isfinite(dw).all()
+    assert np.all(np.abs(dw) <= wl.eta * 1.2024 + np.abs(f64(w_before)) * 2.0 ** -7 + 1e-30)
+    assert np.count_nonzero(dw) > 0
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("M", [16, 64])
+def test_vote_sweep_1b_params_sampled_bit_exact(M):
+    """The vote sweep at 2^30 parameters (fp32 W, eta = 0.01): the updated
+    weights at 4096 sampled positions equal the oracle's vote and update of
+    the same seeded int8 signs, bit for bit."""
+    P = 1 << 30
+    shape = (P // 1024, 1024)
+    rng = np.random.default_rng(M)
+    idx = torch.from_numpy(rng.choice(P, 4096, replace=False)).cuda()
+    words = L.signmuon_packed_words(shape)
+    packed, sampled = [], []
+    for m, s8 in syn.vote_sweep_signs(P, M, seed=3, device="cuda"):
+        buf = torch.empty(words, dtype=torch.int32, device="cuda")
+        L.signmuon_sign_pack(shape, L.SIGNMUON_F32, s8.float().data_ptr(), 1024, 0, buf.data_ptr(), stream())
+        torch.cuda.synchronize()
+        packed.append(buf)
+        sampled.append(s8[idx].cpu().numpy())
+        del s8
+    w = syn.gaussian(shape, 0.02, "cuda", "W", 3, 0)
+    w_s = w.view(-1)[idx].cpu().numpy()
+    wk = ws(L.signmuon_vote_workspace_bytes([shape], M))
+    L.signmuon_vote_update([shape], M, False, [t.data_ptr() for t in packed], L.SIGNMUON_F32, [w.data_ptr()], 0.01,
+                           None, 0, 0, wk.data_ptr(), wk.numel(), stream())
+    torch.cuda.synchronize()
+    v = O.majority_vote([s[None, :] for s in sampled])[0]
+    ref = O.apply_update(w_s.astype(np.float64), 0.01, v, "f32")
+    assert np.array_equal(w.view(-1)[idx].cpu().double().numpy(), ref)
