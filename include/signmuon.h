@@ -191,6 +191,43 @@ signmuon_status signmuon_newton_schulz_batched(
     size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Step 1b-2 split in two: plan once, run every step.
+ * Same computation as signmuon_newton_schulz_batched (which is exactly
+ * plan followed by run); the split only moves per-call host work off the
+ * step: encoding ten TMA tensor maps per unit and uploading the unit table
+ * (1408 bytes per unit) happen once, in plan, instead of on every call.
+ * An optimizer whose buffers persist from step to step plans once and then
+ * calls run each step.
+ *
+ * plan: caller-owned HOST memory of signmuon_newton_schulz_plan_bytes(...)
+ *   bytes, 8-byte aligned; plan() fills it, run() only reads it.  The plan
+ *   records the device addresses of x_bf16, inv_norm, out (or w) and the
+ *   workspace: all of them must stay allocated, and hold the same shapes,
+ *   for as long as the plan is run.  After any of them moves, plan again.
+ * plan() validates and documents its arguments as signmuon_newton_schulz_
+ *   batched does, then writes the unit table into `workspace` with work
+ *   enqueued on `stream`; run() enqueues the k iterations on `stream`, which
+ *   must be ordered after that upload (the same stream, or synchronised).
+ * run() reads inv_norm and x_bf16 at the time it executes (stream order),
+ *   so each step's momentum kernel may refill them in place.
+ * Two runs of plans that share a workspace must not overlap in time (they
+ *   share the A / B' / P buffers); a later plan() on the same workspace
+ *   overwrites the unit table of an earlier one, invalidating it.
+ * Errors: SIGNMUON_ERR_INVALID_ARG for a NULL plan, a plan buffer smaller
+ *   than plan_bytes, a plan not filled by a successful plan(), or k outside
+ *   [0, 64]; the other codes as for signmuon_newton_schulz_batched.  A failed
+ *   plan() leaves the plan unusable (run() rejects it).
+ * ---------------------------------------------------------------------- */
+size_t signmuon_newton_schulz_plan_bytes(int n_mats, int n_workers);
+signmuon_status signmuon_newton_schulz_plan(
+    const signmuon_shape* shapes, int n_mats, int n_workers, void* const* x_bf16,
+    const float* inv_norm, signmuon_ns_out out_mode, void* const* out, signmuon_dtype w_dtype,
+    void* const* w, void* workspace, size_t ws_bytes, void* plan, size_t plan_bytes,
+    void* stream);
+signmuon_status signmuon_newton_schulz_run(const void* plan, int k, float a, float b, float c,
+                                           float eta, void* stream);
+
+/* ------------------------------------------------------------------------
  * Step 2-3 standalone: entrywise sign of a matrix, packed or int8.
  * Source: SignMuon summary, section 2 "Algorithmic flow", steps 2-3 and
  * "Communication efficiency" (1 bit per entry, or 8 bits with int8).

@@ -38,6 +38,7 @@ EXPORTS = (
     "signmuon_status_string", "signmuon_abi_version", "signmuon_x_ld", "signmuon_packed_words",
     "signmuon_device_error", "signmuon_momentum_workspace_bytes", "signmuon_momentum_norm",
     "signmuon_newton_schulz_workspace_bytes", "signmuon_newton_schulz_batched",
+    "signmuon_newton_schulz_plan_bytes", "signmuon_newton_schulz_plan", "signmuon_newton_schulz_run",
     "signmuon_sign_pack", "signmuon_vote_workspace_bytes", "signmuon_vote_update",
     "signmuon_momentum_norm_noalloc", "signmuon_last_error_string",
     "signmuon_spectral_workspace_bytes", "signmuon_spectral_norm",
@@ -74,6 +75,10 @@ _SIGS = {
     "signmuon_newton_schulz_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I, _I]),
     "signmuon_newton_schulz_batched": (_I, [ctypes.POINTER(Shape), _I, _I, _PP, _P, _I, _F, _F, _F,
                                             _I, _PP, _I, _PP, _F, _P, _SZ, _P]),
+    "signmuon_newton_schulz_plan_bytes": (_SZ, [_I, _I]),
+    "signmuon_newton_schulz_plan": (_I, [ctypes.POINTER(Shape), _I, _I, _PP, _P, _I, _PP, _I, _PP, _P, _SZ,
+                                         _P, _SZ, _P]),
+    "signmuon_newton_schulz_run": (_I, [_P, _I, _F, _F, _F, _F, _P]),
     "signmuon_sign_pack": (_I, [Shape, _I, _P, ctypes.c_int64, _I, _P, _P]),
     "signmuon_vote_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I]),
     "signmuon_spectral_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I]),
@@ -183,6 +188,30 @@ def signmuon_newton_schulz_batched(shapes, n_workers, x_bf16, inv_norm, k, a, b,
                                                inv_norm, k, a, b, c, out_mode, _ptrs(out), w_dtype,
                                                _ptrs(w), eta, workspace, ws_bytes, stream)
     _check("signmuon_newton_schulz_batched", st)
+
+
+def signmuon_newton_schulz_plan_bytes(n_mats: int, n_workers: int) -> int:
+    return load().signmuon_newton_schulz_plan_bytes(n_mats, n_workers)
+
+
+def signmuon_newton_schulz_plan(shapes, n_workers, x_bf16, inv_norm, out_mode, out, w_dtype, w,
+                                workspace, ws_bytes, stream=0, plan=None):
+    """Fills `plan` (a host buffer; a new one of the needed size when None)
+    and returns it; pass it to signmuon_newton_schulz_run."""
+    nbytes = signmuon_newton_schulz_plan_bytes(len(shapes), n_workers)
+    if plan is None:
+        plan = (ctypes.c_uint64 * max(1, -(-nbytes // 8)))()
+    st = load().signmuon_newton_schulz_plan(_shapes(shapes), len(shapes), n_workers, _ptrs(x_bf16), inv_norm,
+                                            out_mode, _ptrs(out), w_dtype, _ptrs(w), workspace, ws_bytes,
+                                            ctypes.addressof(plan), ctypes.sizeof(plan), stream)
+    _check("signmuon_newton_schulz_plan", st)
+    return plan
+
+
+def signmuon_newton_schulz_run(plan, k, a, b, c, eta, stream=0) -> None:
+    st = load().signmuon_newton_schulz_run(ctypes.addressof(plan) if plan is not None else None, k, a, b, c,
+                                           eta, stream)
+    _check("signmuon_newton_schulz_run", st)
 
 
 def signmuon_sign_pack(shape, u_dtype, u, ld_u, int8_out, out, stream=0) -> None:

@@ -309,15 +309,35 @@ size_t signmuon_newton_schulz_workspace_bytes(const signmuon_shape* shapes, int 
   return kWsHeaderBytes + ns_desc_bytes(units) + arena;
 }
 
-signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int n_mats, int n_workers,
-                                               void* const* x_bf16, const float* inv_norm, int k, float a,
-                                               float b, float c, signmuon_ns_out out_mode, void* const* out,
-                                               signmuon_dtype w_dtype, void* const* w, float eta,
-                                               void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// A Newton-Schulz plan: the wave schedule of one set of units whose unit
+// table (tensor maps, buffer addresses, tile numbering) already sits in the
+// workspace.  It lives in caller-owned host memory (plan_bytes() bytes).
+struct NsPlanHeader {
+  uint64_t magic;
+  uint8_t* workspace;
+  int64_t max_elems;
+  int32_t n_units, n_waves, out_mode, w_dtype;
+};
+struct NsPlanWave {
+  int32_t u0, nu;
+  int32_t total[3], pair[3];
+};
+constexpr uint64_t kNsPlanMagic = 0x314e4c50534e4d53ull;  // "SMNSPLN1"
+constexpr size_t kNsPlanHeaderBytes = (sizeof(NsPlanHeader) + 63) / 64 * 64;
+
+size_t ns_plan_bytes(int units) { return kNsPlanHeaderBytes + (size_t)units * sizeof(NsPlanWave); }
+inline NsPlanWave* plan_waves(void* plan) { return reinterpret_cast<NsPlanWave*>(static_cast<uint8_t*>(plan) + kNsPlanHeaderBytes); }
+
+signmuon_status ns_validate_buffers(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                    void* const* x_bf16, const float* inv_norm, signmuon_ns_out out_mode,
+                                    void* const* out, signmuon_dtype w_dtype, void* const* w) {
   signmuon_status st = validate_shapes(shapes, n_mats);
   if (st) return st;
   if (n_workers <= 0 || n_workers > SIGNMUON_MAX_WORKERS) return SIGNMUON_ERR_INVALID_ARG;
-  if (k < 0 || k > 64) return SIGNMUON_ERR_INVALID_ARG;
   if (out_mode != SIGNMUON_OUT_PACK1 && out_mode != SIGNMUON_OUT_INT8 && out_mode != SIGNMUON_OUT_UPDATE_W &&
       out_mode != SIGNMUON_OUT_U_F32)
     return SIGNMUON_ERR_INVALID_ARG;
@@ -332,10 +352,20 @@ signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int
   } else {
     if ((st = validate_ptrs(out, units))) return st;
   }
+  return SIGNMUON_OK;
+}
+
+// Encodes the unit table, uploads it into the workspace (stream-ordered on s)
+// and fills the plan.  Arguments are validated by the caller.
+signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_workers, void* const* x_bf16,
+                             const float* inv_norm, signmuon_ns_out out_mode, void* const* out,
+                             signmuon_dtype w_dtype, void* const* w, void* workspace, size_t ws_bytes,
+                             void* plan, cudaStream_t s) {
+  const int units = n_mats * n_workers;
   const size_t need_min = signmuon_newton_schulz_workspace_bytes(shapes, n_mats, n_workers, 1);
-  if ((st = check_workspace(workspace, ws_bytes, need_min))) return st;
+  signmuon_status st = check_workspace(workspace, ws_bytes, need_min);
+  if (st) return st;
   if (!encode_fn()) return SIGNMUON_ERR_UNSUPPORTED;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   NsUnit* d_units = reinterpret_cast<NsUnit*>(ws + kWsHeaderBytes);
@@ -386,11 +416,6 @@ signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int
     }
   }
   wave_begin.push_back(units);
-  // Per wave and stage, pick the tile mode with the least padded work (the
-  // CTA-pair mode is preferred unless it pads more than 15 % extra), then
-  // number the tiles; prefixes restart at each wave (a launch covers one
-  // wave).
-  std::vector<int> wave_pair((wave_begin.size() - 1) * 3, 0);
   // SIGNMUON_NS_TILE_MODE=single|pair forces one tile mode (used by the tests
   // to compare the two modes on the same inputs); unset = automatic.
   int forced_mode = -1;
@@ -398,63 +423,132 @@ signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int
     if (!strcmp(m, "single")) forced_mode = 0;
     else if (!strcmp(m, "pair")) forced_mode = 1;
   }
-  for (size_t wv = 0; wv + 1 < wave_begin.size(); ++wv) {
+  // Per wave and stage, pick the tile mode with the least padded work (the
+  // CTA-pair mode is preferred unless it pads more than 15 % extra), then
+  // number the tiles; prefixes restart at each wave (a launch covers one
+  // wave).
+  NsPlanHeader* hdr = static_cast<NsPlanHeader*>(plan);
+  NsPlanWave* waves = plan_waves(plan);
+  const int n_waves = (int)wave_begin.size() - 1;
+  for (int wv = 0; wv < n_waves; ++wv) {
+    NsPlanWave& W = waves[wv];
+    W.u0 = wave_begin[wv];
+    W.nu = wave_begin[wv + 1] - W.u0;
     for (int stg = 0; stg < 3; ++stg) {
       double single_area = 0, pair_area = 0;
-      for (int ui = wave_begin[wv]; ui < wave_begin[wv + 1]; ++ui) {
+      for (int ui = W.u0; ui < W.u0 + W.nu; ++ui) {
         single_area += (double)ns_tiles(hu[ui].rows, hu[ui].cols, stg, 0) * 128.0 * kBN;
         pair_area += (double)ns_tiles(hu[ui].rows, hu[ui].cols, stg, 1) * 256.0 * kBN;
       }
       int pair = pair_area <= 1.15 * single_area ? 1 : 0;
       if (forced_mode >= 0) pair = forced_mode;
-      wave_pair[wv * 3 + stg] = pair;
+      W.pair[stg] = pair;
       int pre = 0;
-      for (int ui = wave_begin[wv]; ui < wave_begin[wv + 1]; ++ui) {
+      for (int ui = W.u0; ui < W.u0 + W.nu; ++ui) {
         hu[ui].tile_begin[stg] = pre;
         hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg, pair);
         pre += hu[ui].tile_count[stg];
       }
+      W.total[stg] = pre;
     }
   }
   cudaError_t e = upload_bytes(d_units, hu.data(), hu.size() * sizeof(NsUnit), s);
   if (e != cudaSuccess) return cuda_status(e);
+  hdr->magic = kNsPlanMagic;
+  hdr->workspace = ws;
+  hdr->max_elems = max_elems;
+  hdr->n_units = units;
+  hdr->n_waves = n_waves;
+  hdr->out_mode = (int32_t)out_mode;
+  hdr->w_dtype = (int32_t)w_dtype;
+  return SIGNMUON_OK;
+}
 
-  for (size_t wv = 0; wv + 1 < wave_begin.size(); ++wv) {
-    const int u0 = wave_begin[wv], nu = wave_begin[wv + 1] - u0;
+signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, float eta, cudaStream_t s) {
+  const NsPlanHeader* hdr = static_cast<const NsPlanHeader*>(plan);
+  const NsPlanWave* waves = reinterpret_cast<const NsPlanWave*>(static_cast<const uint8_t*>(plan) + kNsPlanHeaderBytes);
+  NsUnit* d_units = reinterpret_cast<NsUnit*>(hdr->workspace + kWsHeaderBytes);
+  cudaError_t e = cudaSuccess;
+  for (int wv = 0; wv < hdr->n_waves; ++wv) {
+    const NsPlanWave& W = waves[wv];
     if (k == 0) {
-      e = launch_ns_identity(d_units + u0, nu, max_elems, (int)out_mode, (int)w_dtype, eta, s);
+      e = launch_ns_identity(d_units + W.u0, W.nu, hdr->max_elems, hdr->out_mode, hdr->w_dtype, eta, s);
       if (e != cudaSuccess) return cuda_status(e);
       continue;
-    }
-    int total[3] = {0, 0, 0};
-    for (int stg = 0; stg < 3; ++stg) {
-      const NsUnit& lastu = hu[u0 + nu - 1];
-      total[stg] = lastu.tile_begin[stg] + lastu.tile_count[stg];
     }
     for (int it = 0; it < k; ++it) {
       NsLaunch L;
       memset(&L, 0, sizeof(L));
-      L.units = d_units + u0;
-      L.n_units = nu;
+      L.units = d_units + W.u0;
+      L.n_units = W.nu;
       L.parity = it & 1;
       L.first = it == 0;
       L.a = a;
       L.b = b;
       L.c = c;
       L.eta = eta;
-      L.w_dtype = (int)w_dtype;
-      L.err = reinterpret_cast<uint32_t*>(ws);
+      L.w_dtype = hdr->w_dtype;
+      L.err = reinterpret_cast<uint32_t*>(hdr->workspace);
       for (int stg = 0; stg < 3; ++stg) {
         L.stage = stg;
-        L.total_tiles = total[stg];
-        L.pair = wave_pair[wv * 3 + stg];
-        L.out_kind = (stg == kStageApply && it == k - 1) ? (int)out_mode : (int)kOutIterate;
+        L.total_tiles = W.total[stg];
+        L.pair = W.pair[stg];
+        L.out_kind = (stg == kStageApply && it == k - 1) ? hdr->out_mode : (int)kOutIterate;
         e = launch_ns_gemm(L, s);
         if (e != cudaSuccess) return cuda_status(e);
       }
     }
   }
   return SIGNMUON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t signmuon_newton_schulz_plan_bytes(int n_mats, int n_workers) {
+  if (n_mats <= 0 || n_workers <= 0 || n_workers > SIGNMUON_MAX_WORKERS) return 0;
+  return ns_plan_bytes(n_mats * n_workers);
+}
+
+signmuon_status signmuon_newton_schulz_plan(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                            void* const* x_bf16, const float* inv_norm,
+                                            signmuon_ns_out out_mode, void* const* out, signmuon_dtype w_dtype,
+                                            void* const* w, void* workspace, size_t ws_bytes, void* plan,
+                                            size_t plan_bytes, void* stream) {
+  signmuon_status st = ns_validate_buffers(shapes, n_mats, n_workers, x_bf16, inv_norm, out_mode, out, w_dtype, w);
+  if (st) return st;
+  if (!plan) return SIGNMUON_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(plan) & 7u) return SIGNMUON_ERR_ALIGNMENT;
+  if (plan_bytes < ns_plan_bytes(n_mats * n_workers)) return SIGNMUON_ERR_INVALID_ARG;
+  static_cast<NsPlanHeader*>(plan)->magic = 0;  // invalid until fully built
+  return ns_make_plan(shapes, n_mats, n_workers, x_bf16, inv_norm, out_mode, out, w_dtype, w, workspace,
+                      ws_bytes, plan, static_cast<cudaStream_t>(stream));
+}
+
+signmuon_status signmuon_newton_schulz_run(const void* plan, int k, float a, float b, float c, float eta,
+                                           void* stream) {
+  if (!plan) return SIGNMUON_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(plan) & 7u) return SIGNMUON_ERR_ALIGNMENT;
+  if (static_cast<const NsPlanHeader*>(plan)->magic != kNsPlanMagic) return SIGNMUON_ERR_INVALID_ARG;
+  if (k < 0 || k > 64) return SIGNMUON_ERR_INVALID_ARG;
+  return ns_run_plan(plan, k, a, b, c, eta, static_cast<cudaStream_t>(stream));
+}
+
+signmuon_status signmuon_newton_schulz_batched(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                               void* const* x_bf16, const float* inv_norm, int k, float a,
+                                               float b, float c, signmuon_ns_out out_mode, void* const* out,
+                                               signmuon_dtype w_dtype, void* const* w, float eta,
+                                               void* workspace, size_t ws_bytes, void* stream) {
+  signmuon_status st = ns_validate_buffers(shapes, n_mats, n_workers, x_bf16, inv_norm, out_mode, out, w_dtype, w);
+  if (st) return st;
+  if (k < 0 || k > 64) return SIGNMUON_ERR_INVALID_ARG;
+  std::vector<uint64_t> plan((ns_plan_bytes(n_mats * n_workers) + 7) / 8);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = ns_make_plan(shapes, n_mats, n_workers, x_bf16, inv_norm, out_mode, out, w_dtype, w, workspace,
+                         ws_bytes, plan.data(), s)))
+    return st;
+  return ns_run_plan(plan.data(), k, a, b, c, eta, s);
 }
 
 // ------------------------------------------------------------------ sign pack

@@ -382,6 +382,14 @@ __device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, i
   return T;
 }
 
+// Pair mode, Gram stage, diagonal tile: each CTA's B rows (n0 + 128 rank ..)
+// are its A rows (m0 + 128 rank ..) of the same operand, so B is read from
+// the A buffer and not loaded.
+template <bool kPair>
+__device__ __forceinline__ bool diag_b_from_a(const NsLaunch& L, const Tile& T) {
+  return kPair && L.stage == kStageGram && T.m0 == T.n0;
+}
+
 // Tensor maps of the two operands of a unit's tile.
 __device__ __forceinline__ void operand_maps(const NsLaunch& L, const NsUnit* u, bool tall, const CUtensorMap*& ma,
                                              const CUtensorMap*& mb) {
@@ -494,6 +502,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         const int nkb = (T.K + kBK - 1) / kBK;
         const int a_row0 = T.m0 + (int)rank * C::kRowsA;
         const int b_row0 = T.n0 + (int)rank * C::kRowsB;
+        const bool b_from_a = diag_b_from_a<kPair>(L, T);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(smem_addr(&empty_bar[stage]), phase ^ 1, abort_flag)) {
             atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutProducer);
@@ -503,8 +512,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           }
           const uint32_t own_full = smem_addr(&full_bar[stage]);
           // Pair mode: both CTAs' copies complete on the even CTA's barrier,
-          // which the even CTA arms for both.
-          if (rank == 0) mbar_arrive_expect_tx(own_full, (kPair ? 2 : 1) * C::kStageBytes);
+          // which the even CTA arms for both.  On a diagonal tile of a
+          // symmetric product each CTA's B half is its A half (the same rows
+          // of the same matrix), so only A is loaded.
+          const int stage_bytes = b_from_a ? C::kStageA : C::kStageBytes;
+          if (rank == 0) mbar_arrive_expect_tx(own_full, (kPair ? 2 : 1) * stage_bytes);
           const uint32_t fb = kPair ? map_to_rank(own_full, 0) : own_full;
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
           const uint32_t sb = sa + C::kStageA;
@@ -519,6 +531,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           }
 #pragma unroll
           for (int j = 0; j < C::kRowsB / kBoxRows; ++j) {
+            if (b_from_a) break;
             const int mn = b_row0 + j * kBoxRows;
             if constexpr (kPair)
               tma_load_2d_pair(sb + j * kBoxBytes, mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
@@ -544,6 +557,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
         // The square stage multiplies the fp16 A and P; all others are bf16.
         const uint32_t idesc = instr_desc(T.a_mn, T.b_mn, C::kTileM, L.stage == kStageSquare);
+        const bool b_from_a = diag_b_from_a<kPair>(L, T);
         const int nkb = (T.K + kBK - 1) / kBK;
         if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag)) {
           atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
@@ -561,7 +575,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           }
           tc_fence_after();
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
-          const uint32_t sb = sa + C::kStageA;
+          const uint32_t sb = b_from_a ? sa : sa + C::kStageA;
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
             const uint32_t aoff = T.a_mn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);

@@ -6,7 +6,8 @@ one GPU, so that the exchange of step 3 becomes the local M-way reduction of
 the vote kernel:
 
   1. signmuon_momentum_norm          momentum, bf16 copy, Frobenius norm
-  2. signmuon_newton_schulz_batched  k iterations, sign fused into the last
+  2. signmuon_newton_schulz_run      k iterations, sign fused into the last
+                                     (planned once by signmuon_newton_schulz_plan)
   3-4. signmuon_vote_update          majority vote + W <- W - eta * vote
   5. (polar) vote matrix -> one Newton-Schulz iteration -> W update
 
@@ -97,6 +98,8 @@ class SignMuonStep:
         self.inv_norm = torch.empty(self.units, dtype=torch.float32, device=dev)
         self.ws_mom = torch.empty(L.signmuon_momentum_workspace_bytes(self.shapes, M), dtype=torch.uint8,
                                   device=dev)
+        self._ns_plan = self._polar_plan = None
+        self._ns_plan_key = self._polar_plan_key = None
         full = L.signmuon_newton_schulz_workspace_bytes(self.shapes, M)
         minimal = L.signmuon_newton_schulz_workspace_bytes(self.shapes, M, minimal=True)
         self.ws_ns = torch.empty(max(minimal, min(full, ns_workspace_cap)), dtype=torch.uint8, device=dev)
@@ -144,11 +147,18 @@ class SignMuonStep:
         if out_mode is None:
             out_mode = L.SIGNMUON_OUT_PACK1 if self.variant == "pack1" else L.SIGNMUON_OUT_INT8
         outs = self.signs if outs is None else outs
+        optrs = [o.data_ptr() for o in outs]
+        # The unit table (tensor maps, buffer addresses) is built once per set
+        # of output buffers; every later call only launches the iterations.
+        key = (out_mode, tuple(optrs))
+        if self._ns_plan_key != key:
+            self._ns_plan = L.signmuon_newton_schulz_plan(
+                self.shapes, self.n_workers, [x.data_ptr() for x in self.x], self.inv_norm.data_ptr(),
+                out_mode, optrs, L.SIGNMUON_F32, None, self.ws_ns.data_ptr(), self.ws_ns.numel(), stream,
+                plan=self._ns_plan)
+            self._ns_plan_key = key
         a, b, c = self.coeffs
-        L.signmuon_newton_schulz_batched(self.shapes, self.n_workers, [x.data_ptr() for x in self.x],
-                                         self.inv_norm.data_ptr(), self.k, a, b, c, out_mode,
-                                         [o.data_ptr() for o in outs], L.SIGNMUON_F32, None, 0.0,
-                                         self.ws_ns.data_ptr(), self.ws_ns.numel(), stream)
+        L.signmuon_newton_schulz_run(self._ns_plan, self.k, a, b, c, 0.0, stream)
 
     def vote_update(self, weights: Sequence[torch.Tensor], stream: int) -> None:
         wptr = [_check_buf(w, s, self.w_dtype, f"weight[{i}]")
@@ -164,11 +174,15 @@ class SignMuonStep:
                                None, self.eta, [v.data_ptr() for v in self.vote], self.nnz.data_ptr(),
                                self.vote_inv.data_ptr(), self.ws_vote.data_ptr(), self.ws_vote.numel(),
                                stream)
+        key = tuple(wptr)
+        if self._polar_plan_key != key:
+            self._polar_plan = L.signmuon_newton_schulz_plan(
+                self.shapes, 1, [v.data_ptr() for v in self.vote], self.vote_inv.data_ptr(),
+                L.SIGNMUON_OUT_UPDATE_W, None, _dtype_code(self.w_dtype), wptr, self.ws_polar.data_ptr(),
+                self.ws_polar.numel(), stream, plan=self._polar_plan)
+            self._polar_plan_key = key
         a, b, c = self.coeffs
-        L.signmuon_newton_schulz_batched(self.shapes, 1, [v.data_ptr() for v in self.vote],
-                                         self.vote_inv.data_ptr(), 1, a, b, c, L.SIGNMUON_OUT_UPDATE_W,
-                                         None, _dtype_code(self.w_dtype), wptr, self.eta,
-                                         self.ws_polar.data_ptr(), self.ws_polar.numel(), stream)
+        L.signmuon_newton_schulz_run(self._polar_plan, 1, a, b, c, self.eta, stream)
 
     def step(self, weights: Sequence[torch.Tensor], grads: Sequence[torch.Tensor]) -> None:
         """One optimizer step: updates `weights` (one tensor per matrix) in place
@@ -181,7 +195,9 @@ class SignMuonStep:
         self.vote_update(weights, stream)
 
     def kernel_launches_per_step(self) -> int:
-        """Number of libsignmuon kernels one step enqueues (descriptor uploads included)."""
+        """Number of libsignmuon kernels one step enqueues once the Newton-Schulz
+        plans exist (from the second step on; the momentum and vote unit tables
+        are still uploaded every step)."""
         def uploads(nbytes):
             return max(1, -(-nbytes // (32768 - 512)))
         M = self.n_workers
@@ -189,14 +205,13 @@ class SignMuonStep:
         mom = uploads(self.units * 56) + 2
         if self.norm == "spectral":
             mom += uploads(self.units * 48) + 1 + 2 * self.spectral_iters
-        unit_bytes = 1408
         ns_waves = self._waves(self.shapes, M, self.ws_ns.numel())
-        ns = uploads(self.units * unit_bytes) + (3 * self.k if self.k > 0 else 1) * ns_waves
+        ns = (3 * self.k if self.k > 0 else 1) * ns_waves
         vote = uploads(n_mats * 64) + uploads(self.units * 8) + 1
         total = mom + ns + vote
         if self.polar:
             total += 1  # 1/sqrt(nnz) kernel (the nnz clear is a memset, not a kernel)
-            total += uploads(n_mats * unit_bytes) + 3 * self._waves(self.shapes, 1, self.ws_polar.numel())
+            total += 3 * self._waves(self.shapes, 1, self.ws_polar.numel())
         return total
 
     @staticmethod

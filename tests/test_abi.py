@@ -100,6 +100,25 @@ def test_argument_validation_returns_status(lib):
     # UPDATE_W needs one worker and weights.
     assert _err(ns, shp, 2, [fake, fake], fake, 1, a, b, c, 2, None, 0, [fake], 0.1, fake, 1 << 30) == 1
     assert _err(ns, shp, 1, [fake], fake, 1, a, b, c, 2, None, 0, None, 0.1, fake, 1 << 30) == 1
+    # Newton-Schulz plan / run.
+    assert L.signmuon_newton_schulz_plan_bytes(0, 1) == 0
+    assert L.signmuon_newton_schulz_plan_bytes(1, 128) == 0
+    assert L.signmuon_newton_schulz_plan_bytes(2, 3) >= 6 * 32
+    plan = (ctypes.c_uint64 * 64)()
+    pl = L.load().signmuon_newton_schulz_plan
+    sh = (L.Shape * 1)(L.Shape(4, 8))
+    xp = (ctypes.c_void_p * 1)(fake)
+    op = (ctypes.c_void_p * 1)(fake)
+    args = [sh, 1, 1, xp, fake, 0, op, 0, None, fake, 1 << 30]
+    assert pl(*args, None, 512, None) == 1                              # no plan buffer
+    assert pl(*args, ctypes.addressof(plan), 8, None) == 1               # plan buffer too small
+    assert pl(*args, ctypes.addressof(plan) + 4, 500, None) == 2         # misaligned plan buffer
+    assert pl(sh, 1, 1, xp, fake, 7, op, 0, None, fake, 1 << 30, ctypes.addressof(plan), 512, None) == 1
+    assert pl(*args[:-1], 64, ctypes.addressof(plan), 512, None) == 4    # workspace too small
+    run = L.load().signmuon_newton_schulz_run
+    assert run(None, 1, a, b, c, 0.0, None) == 1
+    assert run(ctypes.addressof(plan), 1, a, b, c, 0.0, None) == 1        # never filled (rejected plan)
+    assert _err(L.signmuon_newton_schulz_run, plan, 1, a, b, c, 0.0) == 1
     # Sign pack.
     assert _err(L.signmuon_sign_pack, (4, 8), 0, fake, 4, 0, fake) == 1      # ld < cols
     assert _err(L.signmuon_sign_pack, (4, 8), 3, fake, 8, 0, fake) == 1      # bad dtype

@@ -314,6 +314,57 @@ def test_newton_schulz_waves_match_single_wave():
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("minimal_ws", [False, True])
+def test_newton_schulz_plan_run_matches_batched(minimal_ws):
+    """plan + run (run repeated, then a re-plan onto other outputs) gives
+    bit-identical results to the one-shot entry point."""
+    shapes, M, k = [(128, 256), (256, 128), (200, 200), (64, 147)], 3, 2
+    grads, moms = seeded_state(shapes, M, 21)
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9,
+                           torch.float32)
+    saved = [x.clone() for x in xs]
+
+    def restore():
+        for x, sv in zip(xs, saved):
+            x.copy_(sv)
+
+    def new_outs():
+        return [torch.full(shapes[u // M], float("nan"), device="cuda") for u in range(len(xs))]
+
+    ref = new_outs()
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, ref, minimal_ws=minimal_ws)
+    w = ws(L.signmuon_newton_schulz_workspace_bytes(shapes, M, minimal=minimal_ws))
+    xp = [x.data_ptr() for x in xs]
+    for _ in range(2):
+        outs = new_outs()
+        restore()
+        plan = L.signmuon_newton_schulz_plan(shapes, M, xp, inv.data_ptr(), L.SIGNMUON_OUT_U_F32,
+                                             [o.data_ptr() for o in outs], L.SIGNMUON_F32, None, w.data_ptr(),
+                                             w.numel(), stream())
+        for _ in range(2):  # the same plan, twice in a row
+            restore()
+            for o in outs:
+                o.fill_(float("nan"))
+            L.signmuon_newton_schulz_run(plan, k, A, B, C, 0.0, stream())
+            torch.cuda.synchronize()
+            assert_no_device_error(w)
+            for a, b in zip(ref, outs):
+                assert torch.equal(a, b)
+    # k = 0 through the same plan equals the one-shot k = 0.
+    restore()
+    ref0 = new_outs()
+    gpu_ns(shapes, M, xs, inv, 0, L.SIGNMUON_OUT_U_F32, ref0, minimal_ws=minimal_ws)
+    restore()
+    outs = new_outs()
+    plan = L.signmuon_newton_schulz_plan(shapes, M, xp, inv.data_ptr(), L.SIGNMUON_OUT_U_F32,
+                                         [o.data_ptr() for o in outs], L.SIGNMUON_F32, None, w.data_ptr(),
+                                         w.numel(), stream())
+    L.signmuon_newton_schulz_run(plan, 0, A, B, C, 0.0, stream())
+    torch.cuda.synchronize()
+    for a, b in zip(ref0, outs):
+        assert torch.equal(a, b)
+
+
 def test_newton_schulz_k0_and_zero_input():
     shapes, M = [(40, 72), (72, 40)], 2
     grads, moms = seeded_state(shapes, M, 11)
