@@ -45,15 +45,20 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-KERNEL_SOURCES = ("sign_muon_optimizer_momentum_b200/csrc/ns_gemm.cu",
-                  "sign_muon_optimizer_momentum_b200/csrc/elementwise.cu",
-                  "sign_muon_optimizer_momentum_b200/csrc/common.cuh")
+# The sources that decide each kernel's memory traffic (code and launch
+# configuration); a traffic figure is used only while they are unchanged.
+_CSRC = "sign_muon_optimizer_momentum_b200/csrc/"
+KERNEL_SOURCES = {
+    "ns_gemm_kernel": (_CSRC + "ns_gemm.cu", _CSRC + "common.cuh", _CSRC + "api.cu"),
+    "momentum_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh", _CSRC + "api.cu"),
+    "vote_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh", _CSRC + "api.cu"),
+}
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel):
     import hashlib
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()[:16]
 
@@ -68,7 +73,7 @@ def captured_traffic(kernel, workload):
         entries = json.load(open(p))
     except ValueError:
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel)
     for e in entries:
         if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_hash") == src:
             return e.get("bytes_per_launch")
@@ -439,7 +444,8 @@ def run_gpu(args, wl):
 
 def run_vote_sweep(args):
     """Vote + update alone (the bandwidth-bound row): P params as (P/1024, 1024)
-    fp32 W, M packed sign buffers with P(+1) ~ U(0,1) per entry."""
+    W (fp32 by default, or bf16), M packed sign buffers with P(+1) ~ U(0,1)
+    per entry."""
     import torch
     from sign_muon_optimizer_momentum_b200 import _lib as L
     from sign_muon_optimizer_momentum_b200 import build as _build
@@ -469,13 +475,16 @@ def run_vote_sweep(args):
         torch.cuda.synchronize()
         signs.append(buf)
         del s8
-    w = syn.gaussian(shape, 0.02, dev, "W", rank, 0)
+    w_bf16 = args.sweep_w_dtype == "bf16"
+    w = syn.gaussian(shape, 0.02, dev, "W", rank, 0, dtype=torch.bfloat16 if w_bf16 else torch.float32)
+    w_code = L.SIGNMUON_BF16 if w_bf16 else L.SIGNMUON_F32
+    w_bytes = 2 if w_bf16 else 4
     wsz = L.signmuon_vote_workspace_bytes([shape], M)
     wsb = torch.zeros(wsz, dtype=torch.uint8, device=dev)
     sp = [t.data_ptr() for t in signs]
 
     def step():
-        L.signmuon_vote_update([shape], M, False, sp, L.SIGNMUON_F32, [w.data_ptr()], 0.01, None, 0, 0,
+        L.signmuon_vote_update([shape], M, False, sp, w_code, [w.data_ptr()], 0.01, None, 0, 0,
                                wsb.data_ptr(), wsz, stream.cuda_stream)
 
     for _ in range(args.warmup):
@@ -499,18 +508,19 @@ def run_vote_sweep(args):
         ms = t.item()
     clk = clocks.stop() if clocks else None
     per = ms / args.steps
-    bytes_per = P * (M / 8 + 8)
+    bytes_per = P * (M / 8 + 2 * w_bytes)
     pk = peaks()
     gbs = bytes_per / (per / 1e3) / 1e9
     res = {"metric": METRIC, "value": P * M * world / (per / 1e3), "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
-           "config": {"workload": "vote_sweep", "params": P, "workers": M, "w_dtype": "f32", "eta": 0.01,
+           "config": {"workload": "vote_sweep", "params": P, "workers": M, "w_dtype": args.sweep_w_dtype, "eta": 0.01,
                       "l2": f"inputs larger than L2 ({bytes_per / 2**30:.2f} GiB per step)"},
            "roofline": {"bound": "hbm", "kernel": "vote_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
                         "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
-                        "traffic": captured_traffic("vote_kernel", f"vote_sweep_P{P}_M{M}"),
-                        "note": f"algorithmic {M}/8 + 8 B/param (packed signs read, fp32 W read+write)"},
+                        "traffic": captured_traffic("vote_kernel", f"vote_sweep_P{P}_M{M}_{args.sweep_w_dtype}"),
+                        "note": f"algorithmic {M}/8 + {2 * w_bytes} B/param (packed signs read, "
+                                f"{args.sweep_w_dtype} W read+write)"},
            "gpu_launches": 3 * args.steps, "clocks": clk}
     if world > 1:
         import torch.distributed as dist
@@ -529,6 +539,8 @@ def main():
                     help="keep only the first N matrices of the workload (small profiling cases)")
     ap.add_argument("--sweep-params", type=int, default=1 << 30)
     ap.add_argument("--sweep-workers", type=int, default=16)
+    ap.add_argument("--sweep-w-dtype", default="f32", choices=["f32", "bf16"],
+                    help="weight dtype of the vote sweep")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -604,7 +604,7 @@ signmuon_status signmuon_vote_update(const signmuon_shape* shapes, int n_mats, i
     v.n_words = (int64_t)v.rows * v.wpr;
     v.ld_x = x_ld_of(v.cols);
     v.block_begin = blocks;
-    v.block_count = vote_blocks_for(int8_in != 0, v.cols, v.n, v.n_words);
+    v.block_count = vote_blocks_for(int8_in != 0, w_dtype == SIGNMUON_BF16, vote_out, v.cols, v.n, v.n_words);
     v.sign_ptr_offset = i * n_workers;
     blocks += v.block_count;
   }
@@ -612,8 +612,13 @@ signmuon_status signmuon_vote_update(const signmuon_shape* shapes, int n_mats, i
   VoteMat* d_mats = reinterpret_cast<VoteMat*>(ws + kWsHeaderBytes);
   const void** d_table =
       reinterpret_cast<const void**>(ws + kWsHeaderBytes + align_up((size_t)n_mats * sizeof(VoteMat), 256));
-  cudaError_t e = upload_bytes(d_mats, hm.data(), hm.size() * sizeof(VoteMat), s);
-  if (e == cudaSuccess) e = upload_bytes(d_table, signs, (size_t)units * sizeof(void*), s);
+  // The matrix table and the sign-pointer table are adjacent in the
+  // workspace: one upload writes both.
+  const size_t table_off = align_up((size_t)n_mats * sizeof(VoteMat), 256);
+  std::vector<uint8_t> staged(table_off + (size_t)units * sizeof(void*), 0);
+  memcpy(staged.data(), hm.data(), hm.size() * sizeof(VoteMat));
+  memcpy(staged.data() + table_off, signs, (size_t)units * sizeof(void*));
+  cudaError_t e = upload_bytes(d_mats, staged.data(), staged.size(), s);
   if (e == cudaSuccess && vote_out) e = cudaMemsetAsync(nnz, 0, (size_t)n_mats * sizeof(int64_t), s);
   if (e == cudaSuccess)
     e = launch_vote(d_mats, n_mats, blocks, d_table, n_workers, int8_in != 0, w_dtype == SIGNMUON_BF16, eta,

@@ -160,7 +160,7 @@ cudaError_t launch_vote(const VoteMat* mats, int n_mats, int total_blocks, const
                         int n_workers, int int8_in, int w_bf16, float eta, int vote_out,
                         unsigned long long* nnz, cudaStream_t stream);
 cudaError_t launch_vote_inv(const int64_t* nnz, float* inv, int n_mats, cudaStream_t stream);
-int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words);
+int vote_blocks_for(int int8_in, int w_bf16, int vote_out, int cols, int64_t n, int64_t n_words);
 cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream);
 cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, float* vecs, float* parts,
                             int iters, float* inv_norm, cudaStream_t stream);

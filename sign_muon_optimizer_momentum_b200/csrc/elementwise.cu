@@ -8,6 +8,8 @@
 //   * the k = 0 Newton-Schulz output path (U = X0).
 #include <cstring>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace signmuon {
@@ -321,6 +323,63 @@ __device__ __forceinline__ int vote_of(uint32_t gt, uint32_t tie, int j) {
   return ((gt >> j) & 1) ? 1 : (((tie >> j) & 1) ? 0 : -1);
 }
 
+// The step -eta * vote for bit j of the (gt, tie) masks: -eta for +1, +eta
+// for -1 and -0 for a tie (w + -0 == w bit for bit, signed zeros included).
+__device__ __forceinline__ float vote_step(uint32_t gt, uint32_t tie, int j, float eta) {
+  const float d = ((gt >> j) & 1u) ? -eta : eta;
+  return ((tie >> j) & 1u) ? -0.f : d;
+}
+
+// Single-rounding bf16 result for a sum s = fl32(w + d) that fell on a bf16
+// rounding midpoint (see upd_bf16): the exact error of the fp32 addition
+// decides the direction.
+__device__ __noinline__ float bf16_midpoint_fix(float w, float d, float s) {
+  const float bb = __fsub_rn(s, w);
+  const float err = __fadd_rn(__fsub_rn(w, __fsub_rn(s, bb)), __fsub_rn(d, bb));
+  if (err == 0.f) return s;  // a true tie: the conversion rounds to even
+  const uint32_t hi = __float_as_uint(s) & 0xFFFF0000u;
+  const bool away = (err > 0.f) == (s > 0.f);
+  return __uint_as_float(away ? hi + 0x10000u : hi);
+}
+
+// W <- W - eta * vote on 8 bf16 weights (one 16-byte vector) whose votes are
+// bits sh .. sh+7 of (gt, tie), each rounded once.  The sums are formed in
+// fp32; the rare midpoint case is checked for the vector as a whole.
+__device__ __forceinline__ void update8_bf16(uint4& raw, uint32_t gt, uint32_t tie, int sh, float eta) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(&raw);
+  float w[8], sum[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    w[2 * q] = __uint_as_float(r[q] << 16);
+    w[2 * q + 1] = __uint_as_float(r[q] & 0xFFFF0000u);
+  }
+  bool mid = false;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sum[j] = __fadd_rn(w[j], vote_step(gt, tie, sh + j, eta));
+    mid |= (__float_as_uint(sum[j]) & 0xFFFFu) == 0x8000u;
+  }
+  if (mid) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if ((__float_as_uint(sum[j]) & 0xFFFFu) == 0x8000u)
+        sum[j] = bf16_midpoint_fix(w[j], vote_step(gt, tie, sh + j, eta), sum[j]);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(sum[2 * q], sum[2 * q + 1]);
+    r[q] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
+// W <- W - eta * vote on 4 fp32 weights with votes at bits sh .. sh+3.
+__device__ __forceinline__ void update4_f32(float4& x, uint32_t gt, uint32_t tie, int sh, float eta) {
+  x.x = __fadd_rn(x.x, vote_step(gt, tie, sh + 0, eta));
+  x.y = __fadd_rn(x.y, vote_step(gt, tie, sh + 1, eta));
+  x.z = __fadd_rn(x.z, vote_step(gt, tie, sh + 2, eta));
+  x.w = __fadd_rn(x.w, vote_step(gt, tie, sh + 3, eta));
+}
+
 __device__ __forceinline__ int find_vote_mat(const VoteMat* mats, int n, int b) {
   int lo = 0, hi = n - 1;
   while (lo < hi) {
@@ -341,82 +400,141 @@ constexpr int kVoteInt8PerThread = 16;
 constexpr int kVoteInt8PerBlock = kVoteThreads * kVoteInt8PerThread;   // 4096
 constexpr int kVoteGeneralWordsPerBlock = kVoteThreads;
 
-__device__ __forceinline__ void count_word(const void* const* __restrict__ tab, int m_workers, int64_t w,
-                                           BitCount& bc) {
+// Counts kWords words of every worker's signs together (their loads are
+// independent and in flight at once).  Words with ok[k] false count zeros.
+template <int kWords>
+__device__ __forceinline__ void count_words(const void* const* __restrict__ tab, int m_workers,
+                                            const int64_t* w, const bool* ok, BitCount* bc) {
 #pragma unroll
-  for (int p = 0; p < 7; ++p) bc.p[p] = 0;
+  for (int k = 0; k < kWords; ++k)
+#pragma unroll
+    for (int p = 0; p < 7; ++p) bc[k].p[p] = 0;
   int m = 0;
   for (; m + 8 <= m_workers; m += 8) {
-    uint32_t x[8];
+    uint32_t x[kWords][8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = __ldg(static_cast<const uint32_t*>(tab[m + j]) + w);
-    uint32_t t2a, t2b, t4a, t4b, t8;
-    csa(t2a, bc.p[0], bc.p[0], x[0], x[1]);
-    csa(t2b, bc.p[0], bc.p[0], x[2], x[3]);
-    csa(t4a, bc.p[1], bc.p[1], t2a, t2b);
-    csa(t2a, bc.p[0], bc.p[0], x[4], x[5]);
-    csa(t2b, bc.p[0], bc.p[0], x[6], x[7]);
-    csa(t4b, bc.p[1], bc.p[1], t2a, t2b);
-    csa(t8, bc.p[2], bc.p[2], t4a, t4b);
-    ripple(bc, t8, 3);
-  }
-  for (; m < m_workers; ++m) ripple(bc, __ldg(static_cast<const uint32_t*>(tab[m]) + w), 0);
-}
-
-__device__ void vote_packed_fast(const VoteMat& mt, const void* const* __restrict__ tab, int m_workers,
-                                 int lb, int w_bf16, float eta, int vote_out,
-                                 unsigned long long* nnz_out) {
-  const int lane = threadIdx.x & 31;
-  const int64_t w = (int64_t)lb * kVoteThreads + threadIdx.x;  // word of this thread
-  uint32_t gt = 0, tie = 0;
-  if (w < mt.n_words) {
-    BitCount bc;
-    count_word(tab, m_workers, w, bc);
-    vote_masks(bc, m_workers, gt, tie);
-  }
-  // The warp's 32 words cover weights [p0, p0 + 1024): 256 groups of 4.
-  const int64_t p0 = (w - lane) * 32;
-  unsigned long long nz = 0;
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t* src = static_cast<const uint32_t*>(tab[m + j]);
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int g4 = it * 32 + lane;    // group of 4 weights within the warp chunk
-    const int src = g4 >> 3;          // lane holding the word of this group
-    const uint32_t gw = __shfl_sync(0xffffffffu, gt, src);
-    const uint32_t tw = __shfl_sync(0xffffffffu, tie, src);
-    const int sh = (g4 & 7) * 4;
-    const int64_t p = p0 + (int64_t)g4 * 4;
-    if (p >= mt.n) continue;  // n is a multiple of 32: a group is all-in or all-out
-    int v[4];
+      for (int k = 0; k < kWords; ++k) x[k][j] = ok[k] ? __ldg(src + w[k]) : 0u;
+    }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = vote_of(gw, tw, sh + j);
-    if (vote_out) {
-      __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(mt.vote);
-      __nv_bfloat162 h[2];
-      h[0] = __floats2bfloat162_rn((float)v[0], (float)v[1]);
-      h[1] = __floats2bfloat162_rn((float)v[2], (float)v[3]);
-      *reinterpret_cast<uint2*>(vo + p) = *reinterpret_cast<const uint2*>(h);
-      nz += (v[0] != 0) + (v[1] != 0) + (v[2] != 0) + (v[3] != 0);
-    } else if (w_bf16) {
-      __nv_bfloat16* wp = static_cast<__nv_bfloat16*>(mt.w);
-      uint2 raw = *reinterpret_cast<const uint2*>(wp + p);
-      __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&raw);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) e[j] = upd_bf16(e[j], eta, v[j]);
-      *reinterpret_cast<uint2*>(wp + p) = raw;
-    } else {
-      float* wp = static_cast<float*>(mt.w);
-      float4 x = *reinterpret_cast<const float4*>(wp + p);
-      x.x = upd_f32(x.x, eta, v[0]);
-      x.y = upd_f32(x.y, eta, v[1]);
-      x.z = upd_f32(x.z, eta, v[2]);
-      x.w = upd_f32(x.w, eta, v[3]);
-      *reinterpret_cast<float4*>(wp + p) = x;
+    for (int k = 0; k < kWords; ++k) {
+      BitCount& b = bc[k];
+      uint32_t t2a, t2b, t4a, t4b, t8;
+      csa(t2a, b.p[0], b.p[0], x[k][0], x[k][1]);
+      csa(t2b, b.p[0], b.p[0], x[k][2], x[k][3]);
+      csa(t4a, b.p[1], b.p[1], t2a, t2b);
+      csa(t2a, b.p[0], b.p[0], x[k][4], x[k][5]);
+      csa(t2b, b.p[0], b.p[0], x[k][6], x[k][7]);
+      csa(t4b, b.p[1], b.p[1], t2a, t2b);
+      csa(t8, b.p[2], b.p[2], t4a, t4b);
+      ripple(b, t8, 3);
     }
   }
-  if (vote_out) {
+  for (; m < m_workers; ++m) {
+    const uint32_t* src = static_cast<const uint32_t*>(tab[m]);
+#pragma unroll
+    for (int k = 0; k < kWords; ++k) ripple(bc[k], ok[k] ? __ldg(src + w[k]) : 0u, 0);
+  }
+}
+
+enum VoteMode { kVoteF32 = 0, kVoteBf16 = 1, kVoteOut = 2 };
+
+// Words per thread of the packed fast path, per mode: a bf16 thread moves
+// half the W bytes of an fp32 one per word, so it takes two words to keep as
+// many bytes in flight.
+template <int kMode>
+struct PackedWords { static constexpr int value = kMode == kVoteBf16 ? 2 : 1; };
+
+template <int kMode>
+__device__ void vote_packed_fast(const VoteMat& mt, const void* const* __restrict__ tab, int m_workers,
+                                 int lb, float eta, unsigned long long* nnz_out) {
+  constexpr int kWords = PackedWords<kMode>::value;
+  const int lane = threadIdx.x & 31;
+  // Word k of this thread; the warp's 32 words k cover weights
+  // [p0[k], p0[k] + 1024).  n is a multiple of 32, so a group of 4 or 8
+  // weights inside one word is all-in or all-out.  W moves in 16-byte vectors.
+  // (Issuing the W loads before the sign loads measured slower: the extra
+  // live registers cost more occupancy than the overlap gains.)
+  int64_t wd[kWords], p0[kWords];
+  bool ok[kWords];
+#pragma unroll
+  for (int k = 0; k < kWords; ++k) {
+    wd[k] = ((int64_t)lb * kWords + k) * kVoteThreads + threadIdx.x;
+    p0[k] = (wd[k] - lane) * 32;
+    ok[k] = wd[k] < mt.n_words;
+  }
+  constexpr int kVec = kMode == kVoteBf16 ? 8 : 4;   // weights per vector
+  constexpr int kIters = 1024 / 32 / kVec;           // vectors per thread and word
+  using Vec = typename std::conditional<kMode == kVoteBf16, uint4, float4>::type;
+  uint32_t gt[kWords], tie[kWords];
+  {
+    BitCount bc[kWords];
+    count_words<kWords>(tab, m_workers, wd, ok, bc);
+#pragma unroll
+    for (int k = 0; k < kWords; ++k) {
+      vote_masks(bc[k], m_workers, gt[k], tie[k]);
+      if (!ok[k]) gt[k] = tie[k] = 0;
+    }
+  }
+  Vec vec[kMode == kVoteOut ? 1 : kWords][kMode == kVoteOut ? 1 : kIters];
+  if constexpr (kMode != kVoteOut) {
+#pragma unroll
+    for (int k = 0; k < kWords; ++k) {
+      const Vec* wp = reinterpret_cast<const Vec*>(static_cast<const uint8_t*>(mt.w)) + p0[k] / kVec;
+#pragma unroll
+      for (int it = 0; it < kIters; ++it)
+        if (p0[k] + (int64_t)(it * 32 + lane) * kVec < mt.n) vec[k][it] = wp[it * 32 + lane];
+    }
+  }
+  if constexpr (kMode == kVoteOut) {
+    unsigned long long nz = 0;
+    __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(mt.vote);
+#pragma unroll
+    for (int k = 0; k < kWords; ++k) {
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int g4 = it * 32 + lane;  // group of 4 weights within the warp chunk
+        const uint32_t gw = __shfl_sync(0xffffffffu, gt[k], g4 >> 3);
+        const uint32_t tw = __shfl_sync(0xffffffffu, tie[k], g4 >> 3);
+        const int sh = (g4 & 7) * 4;
+        const int64_t p = p0[k] + (int64_t)g4 * 4;
+        if (p >= mt.n) continue;
+        int v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = vote_of(gw, tw, sh + j);
+        __nv_bfloat162 h[2];
+        h[0] = __floats2bfloat162_rn((float)v[0], (float)v[1]);
+        h[1] = __floats2bfloat162_rn((float)v[2], (float)v[3]);
+        *reinterpret_cast<uint2*>(vo + p) = *reinterpret_cast<const uint2*>(h);
+        nz += (v[0] != 0) + (v[1] != 0) + (v[2] != 0) + (v[3] != 0);
+      }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xffffffffu, nz, o);
     if (lane == 0 && nz) atomicAdd(nnz_out, nz);
+  } else {
+    // Vector g = it*32 + lane of word k holds weights [p0[k] + kVec g, +kVec),
+    // counted in word (kVec g) / 32 of the warp chunk, i.e. by lane g / (32 / kVec).
+#pragma unroll
+    for (int k = 0; k < kWords; ++k) {
+      Vec* wp = reinterpret_cast<Vec*>(static_cast<uint8_t*>(mt.w)) + p0[k] / kVec;
+#pragma unroll
+      for (int it = 0; it < kIters; ++it) {
+        const int g = it * 32 + lane;
+        const uint32_t gw = __shfl_sync(0xffffffffu, gt[k], g / (32 / kVec));
+        const uint32_t tw = __shfl_sync(0xffffffffu, tie[k], g / (32 / kVec));
+        const int sh = (g % (32 / kVec)) * kVec;
+        if (p0[k] + (int64_t)g * kVec >= mt.n) continue;
+        Vec& x = vec[k][it];
+        if constexpr (kMode == kVoteBf16)
+          update8_bf16(x, gw, tw, sh, eta);
+        else
+          update4_f32(x, gw, tw, sh, eta);
+        wp[g] = x;
+      }
+    }
   }
 }
 
@@ -459,76 +577,122 @@ __device__ void vote_packed_general(const VoteMat& mt, const void* const* __rest
 }
 
 // int8 path: 16 weights per thread; per-byte sums with SIMD byte adds
-// (|sum| <= M <= 127 fits a signed byte), vote = sign(sum).
-__device__ void vote_int8(const VoteMat& mt, const void* const* __restrict__ tab, int m_workers,
-                          int lb, int w_bf16, float eta, int vote_out,
-                          unsigned long long* nnz_out) {
+// (|sum| <= M <= 127 fits a signed byte), vote = sign(sum).  A warp covers
+// 512 consecutive weights; when all of them are in the matrix the update
+// reads and writes W in warp-contiguous 16-byte vectors, each thread taking
+// the votes of its vector from the thread that counted them (one shuffle of
+// a word holding 16 "positive" bits and 16 "zero" bits).
+template <int kMode>
+__device__ void vote_int8(const VoteMat& mt, const void* const* __restrict__ tab, int m_workers, int lb,
+                          float eta, unsigned long long* nnz_out) {
+  const int lane = threadIdx.x & 31;
   const int64_t e0 = ((int64_t)lb * kVoteThreads + threadIdx.x) * kVoteInt8PerThread;
+  const int64_t q0 = e0 - (int64_t)lane * kVoteInt8PerThread;  // first weight of the warp
+  // Vector path: the warp's 512 weights all lie in the matrix (warp-uniform).
+  const bool vec_path = kMode != kVoteOut && q0 + 32 * kVoteInt8PerThread <= mt.n;
+  constexpr int kVec = kMode == kVoteBf16 ? 8 : 4;   // weights per 16-byte vector
+  constexpr int kIters = kVoteInt8PerThread / kVec;   // vectors per thread
+  using Vec = typename std::conditional<kMode == kVoteBf16, uint4, float4>::type;
+  Vec vec[kMode == kVoteOut ? 1 : kIters];
+  Vec* wp = nullptr;
+  if constexpr (kMode != kVoteOut) {
+    // W loads first: they do not depend on the counts.
+    wp = reinterpret_cast<Vec*>(static_cast<uint8_t*>(mt.w)) + q0 / kVec;
+    if (vec_path) {
+#pragma unroll
+      for (int it = 0; it < kIters; ++it) vec[it] = wp[it * 32 + lane];
+    }
+  }
+  uint32_t code = 0;  // bit j: vote j is +1; bit 16 + j: vote j is 0
+  if (e0 + 16 <= mt.n) {
+    uint32_t acc[4] = {0, 0, 0, 0};
+    for (int m = 0; m < m_workers; ++m) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(tab[m]) + e0));
+      acc[0] = __vadd4(acc[0], x.x);
+      acc[1] = __vadd4(acc[1], x.y);
+      acc[2] = __vadd4(acc[2], x.z);
+      acc[3] = __vadd4(acc[3], x.w);
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int s = (int)(int8_t)((acc[j >> 2] >> ((j & 3) * 8)) & 0xff);
+      code |= (s > 0 ? 1u << j : 0u) | (s == 0 ? 1u << (16 + j) : 0u);
+    }
+  } else {
+    for (int j = 0; j < 16; ++j) {
+      int s = 0;
+      if (e0 + j < mt.n)
+        for (int m = 0; m < m_workers; ++m) s += static_cast<const int8_t*>(tab[m])[e0 + j];
+      code |= (s > 0 ? 1u << j : 0u) | (s == 0 ? 1u << (16 + j) : 0u);
+    }
+  }
+  auto vote_in = [](uint32_t cw, int j) { return ((cw >> j) & 1) ? 1 : (((cw >> (16 + j)) & 1) ? 0 : -1); };
+  if constexpr (kMode != kVoteOut) {
+    if (vec_path) {
+      // Vector g = it*32 + lane holds weights [q0 + kVec g, +kVec), counted
+      // by thread g / (16 / kVec).
+#pragma unroll
+      for (int it = 0; it < kIters; ++it) {
+        const int g = it * 32 + lane;
+        const uint32_t cw = __shfl_sync(0xffffffffu, code, g / (16 / kVec));
+        const int sh = (g % (16 / kVec)) * kVec;
+        if constexpr (kMode == kVoteBf16)
+          update8_bf16(vec[it], cw, cw >> 16, sh, eta);
+        else
+          update4_f32(vec[it], cw, cw >> 16, sh, eta);
+        wp[g] = vec[it];
+      }
+      return;
+    }
+  }
+  // Scalar path: the vote-out mode and the last (partial) warp of a matrix.
   unsigned long long nz = 0;
   if (e0 < mt.n) {
-    int v[16];
-    if (e0 + 16 <= mt.n) {
-      uint32_t acc[4] = {0, 0, 0, 0};
-      for (int m = 0; m < m_workers; ++m) {
-        const uint4 x = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(tab[m]) + e0));
-        acc[0] = __vadd4(acc[0], x.x);
-        acc[1] = __vadd4(acc[1], x.y);
-        acc[2] = __vadd4(acc[2], x.z);
-        acc[3] = __vadd4(acc[3], x.w);
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int s = (int)(int8_t)((acc[j >> 2] >> ((j & 3) * 8)) & 0xff);
-        v[j] = (s > 0) - (s < 0);
-      }
-    } else {
-      for (int j = 0; j < 16; ++j) {
-        int s = 0;
-        if (e0 + j < mt.n)
-          for (int m = 0; m < m_workers; ++m) s += static_cast<const int8_t*>(tab[m])[e0 + j];
-        v[j] = (s > 0) - (s < 0);
-      }
-    }
     const bool full = (e0 + 16 <= mt.n);
     for (int j = 0; j < 16; ++j) {
       const int64_t e = e0 + j;
       if (!full && e >= mt.n) break;
-      if (vote_out) {
+      const int v = vote_in(code, j);
+      if constexpr (kMode == kVoteOut) {
         const int64_t r = e / mt.cols, c = e - r * mt.cols;
-        static_cast<__nv_bfloat16*>(mt.vote)[r * mt.ld_x + c] = __float2bfloat16_rn((float)v[j]);
-        nz += (v[j] != 0);
-      } else if (w_bf16) {
-        __nv_bfloat16* wp = static_cast<__nv_bfloat16*>(mt.w);
-        wp[e] = upd_bf16(wp[e], eta, v[j]);
+        static_cast<__nv_bfloat16*>(mt.vote)[r * mt.ld_x + c] = __float2bfloat16_rn((float)v);
+        nz += (v != 0);
+      } else if constexpr (kMode == kVoteBf16) {
+        __nv_bfloat16* w = static_cast<__nv_bfloat16*>(mt.w);
+        w[e] = upd_bf16(w[e], eta, v);
       } else {
-        float* wp = static_cast<float*>(mt.w);
-        wp[e] = upd_f32(wp[e], eta, v[j]);
+        float* w = static_cast<float*>(mt.w);
+        w[e] = upd_f32(w[e], eta, v);
       }
     }
   }
-  if (vote_out) {
+  if constexpr (kMode == kVoteOut) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xffffffffu, nz, o);
-    if ((threadIdx.x & 31) == 0 && nz) atomicAdd(nnz_out, nz);
+    if (lane == 0 && nz) atomicAdd(nnz_out, nz);
   }
 }
 
-__global__ void __launch_bounds__(kVoteThreads)
+// One instantiation per mode (fp32 update, bf16 update, vote out), so that
+// each uses only the registers its own path needs.
+template <int kMode>
+struct VoteMinBlocks { static constexpr int value = 4; };
+
+template <int kMode>
+__global__ void __launch_bounds__(kVoteThreads, VoteMinBlocks<kMode>::value)
 vote_kernel(const VoteMat* __restrict__ mats, int n_mats, const void* const* __restrict__ table,
-            int n_workers, int int8_in, int w_bf16, float eta, int vote_out,
-            unsigned long long* __restrict__ nnz) {
+            int n_workers, int int8_in, float eta, unsigned long long* __restrict__ nnz) {
   const int b = blockIdx.x;
   const int i = find_vote_mat(mats, n_mats, b);
   const VoteMat mt = mats[i];
   const int lb = b - mt.block_begin;
   const void* const* tab = table + mt.sign_ptr_offset;
-  if (int8_in) {
-    vote_int8(mt, tab, n_workers, lb, w_bf16, eta, vote_out, nnz + i);
-  } else if ((mt.cols & 31) == 0) {
-    vote_packed_fast(mt, tab, n_workers, lb, w_bf16, eta, vote_out, nnz + i);
-  } else {
-    vote_packed_general(mt, tab, n_workers, lb, w_bf16, eta, vote_out, nnz + i);
-  }
+  if (int8_in)
+    vote_int8<kMode>(mt, tab, n_workers, lb, eta, nnz + i);
+  else if ((mt.cols & 31) == 0)
+    vote_packed_fast<kMode>(mt, tab, n_workers, lb, eta, nnz + i);
+  else
+    vote_packed_general(mt, tab, n_workers, lb, kMode == kVoteBf16, eta, kMode == kVoteOut, nnz + i);
 }
 
 __global__ void vote_inv_kernel(const int64_t* __restrict__ nnz, float* __restrict__ inv, int n) {
@@ -540,8 +704,15 @@ cudaError_t launch_vote(const VoteMat* mats, int n_mats, int total_blocks, const
                         int n_workers, int int8_in, int w_bf16, float eta, int vote_out,
                         unsigned long long* nnz, cudaStream_t stream) {
   if (total_blocks <= 0) return cudaSuccess;
-  vote_kernel<<<total_blocks, kVoteThreads, 0, stream>>>(mats, n_mats, sign_table, n_workers, int8_in,
-                                                        w_bf16, eta, vote_out, nnz);
+  if (vote_out)
+    vote_kernel<kVoteOut><<<total_blocks, kVoteThreads, 0, stream>>>(mats, n_mats, sign_table, n_workers,
+                                                                     int8_in, eta, nnz);
+  else if (w_bf16)
+    vote_kernel<kVoteBf16><<<total_blocks, kVoteThreads, 0, stream>>>(mats, n_mats, sign_table, n_workers,
+                                                                      int8_in, eta, nnz);
+  else
+    vote_kernel<kVoteF32><<<total_blocks, kVoteThreads, 0, stream>>>(mats, n_mats, sign_table, n_workers,
+                                                                     int8_in, eta, nnz);
   return cudaGetLastError();
 }
 
@@ -550,9 +721,14 @@ cudaError_t launch_vote_inv(const int64_t* nnz, float* inv, int n_mats, cudaStre
   return cudaGetLastError();
 }
 
-int vote_blocks_for(int int8_in, int cols, int64_t n, int64_t n_words) {
+int vote_blocks_for(int int8_in, int w_bf16, int vote_out, int cols, int64_t n, int64_t n_words) {
   if (int8_in) return (int)((n + kVoteInt8PerBlock - 1) / kVoteInt8PerBlock);
-  if ((cols & 31) == 0) return (int)((n_words + kVoteWordsPerBlock - 1) / kVoteWordsPerBlock);
+  if ((cols & 31) == 0) {
+    const int64_t per_block = (int64_t)kVoteWordsPerBlock * (vote_out ? PackedWords<kVoteOut>::value
+                                                             : w_bf16 ? PackedWords<kVoteBf16>::value
+                                                                      : PackedWords<kVoteF32>::value);
+    return (int)((n_words + per_block - 1) / per_block);
+  }
   return (int)((n_words + kVoteGeneralWordsPerBlock - 1) / kVoteGeneralWordsPerBlock);
 }
 

@@ -207,7 +207,7 @@ class SignMuonStep:
             mom += uploads(self.units * 48) + 1 + 2 * self.spectral_iters
         ns_waves = self._waves(self.shapes, M, self.ws_ns.numel())
         ns = (3 * self.k if self.k > 0 else 1) * ns_waves
-        vote = uploads(n_mats * 64) + uploads(self.units * 8) + 1
+        vote = uploads(-(-n_mats * 64 // 256) * 256 + self.units * 8) + 1
         total = mom + ns + vote
         if self.polar:
             total += 1  # 1/sqrt(nnz) kernel (the nnz clear is a memset, not a kernel)

@@ -541,15 +541,17 @@ def test_vote_update_bf16_single_rounding_on_midpoint(int8_in):
     """eta = 2^-9 + 2^-30 puts the fp32 difference 1 - eta exactly on the bf16
     midpoint 1 - 2^-9 although the exact difference lies below it: a
     double-rounded update would give 1.0, the single rounding 0.99609375."""
-    shape, M = (4, 64), 1
+    # 16 x 64 = 1024 weights: two full 512-weight warps of the int8 path and
+    # one 1024-weight warp chunk of the packed path (the vector paths).
+    shape, M = (16, 64), 1
     eta = float(np.float32(2.0 ** -9 + 2.0 ** -30))
     assert eta == 2.0 ** -9 + 2.0 ** -30
     w0 = torch.ones(shape, dtype=torch.bfloat16)
-    w0[1] = -1.0
-    w0[2] = 2.0
-    w0[3] = syn.gaussian((64,), 1.0, "cpu", "mid", dtype=torch.bfloat16)
+    w0[1::4] = -1.0
+    w0[2::4] = 2.0
+    w0[3::4] = syn.gaussian((4, 64), 1.0, "cpu", "mid", dtype=torch.bfloat16)
     signs = torch.ones(shape, dtype=torch.int8)
-    signs[1] = -1
+    signs[1::4] = -1
     dev = [signs.cuda()] if int8_in else _packed_device([signs], shape)
     w = w0.cuda()
     wk = ws(L.signmuon_vote_workspace_bytes([shape], M))
@@ -558,6 +560,32 @@ def test_vote_update_bf16_single_rounding_on_midpoint(int8_in):
     torch.cuda.synchronize()
     ref = O.apply_update(f64(w0), eta, signs.numpy(), "bf16")
     assert ref[0, 0] == 0.99609375
+    assert np.array_equal(f64(w), ref)
+
+
+@pytest.mark.parametrize("int8_in", [False, True])
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
+def test_vote_tie_leaves_weights_bit_identical(int8_in, w_dtype):
+    """A tied vote (even M, equal split) leaves W bit for bit, signed zeros
+    included; the other entries follow the oracle."""
+    shape, M = (16, 64), 2
+    w0 = syn.gaussian(shape, 1.0, "cpu", "tie", dtype=w_dtype)
+    w0[0, :32] = 0.0
+    w0[0, 32:] = -0.0
+    s0 = torch.ones(shape, dtype=torch.int8)
+    s1 = -torch.ones(shape, dtype=torch.int8)   # every entry ties ...
+    s1[8:] = 1                                  # ... except the lower half (+1)
+    dev = [s0.cuda(), s1.cuda()] if int8_in else _packed_device([s0, s1], shape)
+    w = w0.cuda()
+    wk = ws(L.signmuon_vote_workspace_bytes([shape], M))
+    code = L.SIGNMUON_BF16 if w_dtype == torch.bfloat16 else L.SIGNMUON_F32
+    L.signmuon_vote_update([shape], M, int8_in, [d.data_ptr() for d in dev], code, [w.data_ptr()], 0.01,
+                           None, 0, 0, wk.data_ptr(), wk.numel(), stream())
+    torch.cuda.synchronize()
+    ibits = torch.int16 if w_dtype == torch.bfloat16 else torch.int32
+    assert torch.equal(w[:8].cpu().view(ibits), w0[:8].view(ibits))
+    ref = O.apply_update(f64(w0), 0.01, O.majority_vote([s0.numpy(), s1.numpy()]),
+                         "bf16" if w_dtype == torch.bfloat16 else "f32")
     assert np.array_equal(f64(w), ref)
 
 
