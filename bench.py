@@ -45,13 +45,13 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-# The sources that decide each kernel's memory traffic (code and launch
-# configuration); a traffic figure is used only while they are unchanged.
+# The sources of each kernel; a captured traffic figure is used only while
+# they are unchanged.
 _CSRC = "sign_muon_optimizer_momentum_b200/csrc/"
 KERNEL_SOURCES = {
-    "ns_gemm_kernel": (_CSRC + "ns_gemm.cu", _CSRC + "common.cuh", _CSRC + "api.cu"),
-    "momentum_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh", _CSRC + "api.cu"),
-    "vote_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh", _CSRC + "api.cu"),
+    "ns_gemm_kernel": (_CSRC + "ns_gemm.cu", _CSRC + "common.cuh"),
+    "momentum_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
+    "vote_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
 }
 
 
@@ -277,6 +277,7 @@ def run_gpu(args, wl):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = world > 1 or args.exchange
     if world > 1:
         import datetime
         torch.cuda.set_device(local)
@@ -284,6 +285,15 @@ def run_gpu(args, wl):
                                 device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
+        if args.exchange:
+            import datetime
+            import socket
+            sk = socket.socket()
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+            sk.close()
+            dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", 0))
     _build.build()
     dev = torch.device("cuda", torch.cuda.current_device())
     dt = syn.torch_dtype(wl.w_dtype)
@@ -296,8 +306,18 @@ def run_gpu(args, wl):
     def max_over_ranks(x):
         return max_over_ranks_value(x, world, dev)
 
-    opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
-                       polar=wl.polar, device=dev, norm=args.norm)
+    if args.exchange:
+        # One group of n_workers workers per GPU; the signs of all GPUs are
+        # exchanged (1-bit all-gather for packed workloads, int8 SUM
+        # all-reduce for int8 ones) and every GPU votes over all of them.
+        from sign_muon_optimizer_momentum_b200.distributed import SignMuonDistStep
+        if args.norm != "frobenius":
+            raise SystemExit("--exchange supports the Frobenius scaling only")
+        opt = SignMuonDistStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
+                               polar=wl.polar, device=dev)
+    else:
+        opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
+                           polar=wl.polar, device=dev, norm=args.norm)
     weights = [w.to(dev) for w in syn.initial_weights(wl, rank)]
     signal = [g.to(dev) for g in syn.gradient_signal(wl, rank)]
     n_sets = 2
@@ -426,15 +446,20 @@ def run_gpu(args, wl):
     result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-              "config": dict(workload_config(wl), parallelism=f"replicas{world}", norm=args.norm,
+              "config": dict(workload_config(wl), norm=args.norm,
+                             parallelism=(f"dp{world}-{'allgather' if wl.variant == 'pack1' else 'allreduce'}"
+                                          if args.exchange else f"replicas{world}"),
                              l2=f"inputs larger than L2 ({resident / 2**30:.1f} GiB gradients+momentum resident)"),
               "roofline": roofline, "e2e": e2e,
               "phases_ms": {"momentum": mom_ms, "newton_schulz": ns_ms, "vote_update": vote_ms},
               "gpu_launches": opt.kernel_launches_per_step() * args.steps,
               "clocks": clk}
+    if args.exchange:
+        result["config"]["vote_workers"] = world * wl.n_workers
+        result["config"]["exchange_bytes_per_step"] = opt.exchange_bytes_per_step()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl)
-    if world > 1:
+    if pg:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
@@ -521,7 +546,7 @@ def run_vote_sweep(args):
                         "traffic": captured_traffic("vote_kernel", f"vote_sweep_P{P}_M{M}_{args.sweep_w_dtype}"),
                         "note": f"algorithmic {M}/8 + {2 * w_bytes} B/param (packed signs read, "
                                 f"{args.sweep_w_dtype} W read+write)"},
-           "gpu_launches": 3 * args.steps, "clocks": clk}
+           "gpu_launches": 2 * args.steps, "clocks": clk}
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -546,6 +571,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--norm", default="frobenius", choices=["frobenius", "spectral"],
                     help="scaling of the Newton-Schulz input (spectral: 5 power iterations)")
+    ap.add_argument("--exchange", action="store_true",
+                    help="each GPU runs the workload's workers and the signs of all GPUs are exchanged "
+                         "(1-bit all-gather or int8 SUM all-reduce, NCCL) before one vote over all workers; "
+                         "default: independent replicas")
     args = ap.parse_args()
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
     if args.config == "vote_sweep":

@@ -35,7 +35,9 @@
  *   words (the row-major words, rounded up to a multiple of 4).
  * - int8 sign buffers: row-major int8 in {-1, +1}, row stride cols.
  * - sign(0) = sign(-0) = +1 and a NaN maps to +1 (the test is "u < 0").
- * - Every buffer pointer must be 16-byte aligned (SIGNMUON_ERR_ALIGNMENT).
+ * - Every buffer pointer must be 16-byte aligned (SIGNMUON_ERR_ALIGNMENT),
+ *   except the inv_norm input of the Newton-Schulz calls (one float per
+ *   unit, 4-byte aligned: it may point into a larger per-unit array).
  * - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *   enqueued asynchronously; no entry point synchronises the host except
  *   signmuon_device_error.

@@ -97,6 +97,9 @@ def test_argument_validation_returns_status(lib):
     assert _err(ns, shp, 1, [odd], fake, 1, a, b, c, 0, [fake], 0, None, 0.0, fake, 1 << 30) == 2
     assert _err(ns, shp, 1, [fake], fake, 1, a, b, c, 0, [fake], 0, None, 0.0, fake, 64) == 4
     assert _err(ns, shp, 1, [fake], fake, 1, a, b, c, 0, [fake], 0, None, 0.0, fake + 16, 1 << 30) == 2
+    # inv_norm needs 4-byte alignment only (one float per unit).
+    assert _err(ns, shp, 1, [fake], fake + 2, 1, a, b, c, 0, [fake], 0, None, 0.0, fake, 1 << 30) == 2
+    assert _err(ns, shp, 1, [fake], fake + 4, 1, a, b, c, 0, [fake], 0, None, 0.0, fake, 64) == 4
     # UPDATE_W needs one worker and weights.
     assert _err(ns, shp, 2, [fake, fake], fake, 1, a, b, c, 2, None, 0, [fake], 0.1, fake, 1 << 30) == 1
     assert _err(ns, shp, 1, [fake], fake, 1, a, b, c, 2, None, 0, None, 0.1, fake, 1 << 30) == 1
