@@ -25,6 +25,9 @@ import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+# stdout carries exactly one JSON line: NCCL's own messages (its version banner
+# at communicator setup among them) go to stderr unless the caller chose a file.
+os.environ.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
