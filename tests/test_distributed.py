@@ -127,6 +127,38 @@ def test_gloo_exchange_two_ranks(variant):
     assert res == {0: True, 1: True}
 
 
+def _dropout_worker(rank, world, port, out):
+    import datetime
+    import time
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out[rank] = "left"                       # drops out before the exchange
+        return
+    lay = D.exchange_layout(SHAPES, 1, 1, "pack1")
+    local = torch.zeros(lay.group_len[0], dtype=torch.int32)
+    gathered = torch.zeros(world * lay.group_len[0], dtype=torch.int32)
+    t0 = time.time()
+    try:
+        D.exchange("pack1", local, gathered)
+        out[rank] = "no error"
+    except Exception as e:                       # the missing rank surfaces as an error
+        out[rank] = f"error after {time.time() - t0:.1f}s: {type(e).__name__}"
+
+
+def test_gloo_exchange_with_a_dropped_rank_raises():
+    """A rank that leaves before the exchange makes the collective fail on the
+    others within the group's timeout (an exception, not a hang)."""
+    import torch.multiprocessing as mp
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_dropout_worker, args=(2, _free_port(), out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[1] == "left"
+    assert res[0].startswith("error after"), res[0]
+
+
 # ---------------------------------------------------------------------------
 # GPU
 # ---------------------------------------------------------------------------

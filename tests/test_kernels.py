@@ -492,6 +492,60 @@ def test_polar_workload_small_runs():
         assert not torch.equal(w.cpu(), w_init)
 
 
+def test_polar_replans_when_weight_buffers_move():
+    """The polar step's plan records the weight addresses: stepping new
+    weight tensors (same values) must update those, not the old ones."""
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    wl = syn.Workload("mini_polar2", ((128, 256), (256, 128)), 3, 1, "pack1", "f32", g_noise_std=2.0,
+                      polar=True)
+    signal = syn.gradient_signal(wl, 0)
+
+    def grads(t):
+        return [syn.worker_gradient(wl, signal[i], i, m, t, 0).cuda()
+                for i in range(len(wl.shapes)) for m in range(wl.n_workers)]
+
+    def run(move):
+        opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, torch.float32,
+                           polar=True)
+        w = [x.cuda() for x in syn.initial_weights(wl, 0)]
+        opt.step(w, grads(0))
+        if move:
+            old = w
+            w = [x.clone() for x in old]
+            for x in old:
+                x.fill_(7.0)                      # must stay untouched from here on
+        opt.step(w, grads(1))
+        torch.cuda.synchronize()
+        if move:
+            assert all(bool((x == 7.0).all()) for x in old)
+        return [x.cpu() for x in w]
+
+    for a, b in zip(run(False), run(True)):
+        assert torch.equal(a, b)
+
+
+def test_nan_gradient_gives_all_plus_signs():
+    """A NaN anywhere in one worker's gradient makes its normalised momentum
+    (and U) NaN everywhere; sign(NaN) is +1 (bit = !(u < 0)), as in the
+    oracle.  The other workers are unaffected."""
+    shapes, M = [(64, 96)], 3
+    grads, moms = seeded_state(shapes, M, 17)
+    grads[1][5, 7] = float("nan")
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9, torch.float32)
+    packed = [torch.zeros(L.signmuon_packed_words(shapes[0]), dtype=torch.int32, device="cuda") for _ in range(M)]
+    gpu_ns(shapes, M, xs, inv, 2, L.SIGNMUON_OUT_PACK1, packed)
+    r, c = shapes[0]
+    for m in range(M):
+        _, u = oracle_u(moms[m], grads[m], 0.9, 2)
+        got = unpack_words(packed[m].cpu().numpy().view(np.uint32), r, c)
+        if m == 1:
+            assert np.isnan(u).all()
+            assert (got == 1).all()
+        else:
+            big = np.abs(u) > 1e-3
+            assert np.mean(got[big] == O.sign_entries(u)[big]) >= SIGN_AGREE
+
+
 @pytest.mark.slow
 def test_nanogpt_full_size_sampled_parity():
     """The nanoGPT-small workload at full size (48 matrices, M = 8, k = 5,
