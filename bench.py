@@ -314,8 +314,8 @@ def run_gpu(args, wl):
         # exchanged (1-bit all-gather for packed workloads, int8 SUM
         # all-reduce for int8 ones) and every GPU votes over all of them.
         from sign_muon_optimizer_momentum_b200.distributed import SignMuonDistStep
-        if args.norm != "frobenius":
-            raise SystemExit("--exchange supports the Frobenius scaling only")
+        if args.norm != "frobenius" or args.graph:
+            raise SystemExit("--exchange runs eagerly with the Frobenius scaling only")
         opt = SignMuonDistStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
                                polar=wl.polar, device=dev)
     else:
@@ -350,9 +350,26 @@ def run_gpu(args, wl):
         if ev is not None:
             ev[3].record(stream)
 
+    graphs = None
+    if args.graph:
+        # One CUDA graph per gradient set: each replay is a whole step.
+        graphs = [opt.capture(weights, grad_sets[t]) for t in range(n_sets)]
+
     for t in range(args.warmup):
-        one_step(t)
+        if graphs:
+            graphs[t % n_sets].replay()
+        else:
+            one_step(t)
     barrier()
+
+    if graphs:
+        # Phases from the captured kernels cannot be told apart on the host:
+        # they are taken from eager steps (same kernels), the step time from
+        # the replays.
+        ph_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(args.steps)]
+        for t in range(args.steps):
+            one_step(t, ph_ev[t])
+        barrier()
 
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
@@ -363,10 +380,15 @@ def run_gpu(args, wl):
     barrier()
     start.record(stream)
     for t in range(args.steps):
-        one_step(t, ns_ev[t])
+        if graphs:
+            graphs[t % n_sets].replay()
+        else:
+            one_step(t, ns_ev[t])
     stop.record(stream)
     barrier()
     ms = max_over_ranks(start.elapsed_time(stop))
+    if graphs:
+        ns_ev = ph_ev
     mom_ms = sum(e[0].elapsed_time(e[1]) for e in ns_ev) / args.steps
     ns_ms = sum(e[1].elapsed_time(e[2]) for e in ns_ev) / args.steps
     vote_ms = sum(e[2].elapsed_time(e[3]) for e in ns_ev) / args.steps
@@ -457,6 +479,7 @@ def run_gpu(args, wl):
               "phases_ms": {"momentum": mom_ms, "newton_schulz": ns_ms, "vote_update": vote_ms},
               "gpu_launches": opt.kernel_launches_per_step() * args.steps,
               "clocks": clk}
+    result["config"]["launch"] = "cuda_graph" if graphs else "eager"
     if args.exchange:
         result["config"]["vote_workers"] = world * wl.n_workers
         result["config"]["exchange_bytes_per_step"] = opt.exchange_bytes_per_step()
@@ -574,6 +597,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--norm", default="frobenius", choices=["frobenius", "spectral"],
                     help="scaling of the Newton-Schulz input (spectral: 5 power iterations)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step as one CUDA graph replay (captured with SignMuonStep.capture)")
     ap.add_argument("--exchange", action="store_true",
                     help="each GPU runs the workload's workers and the signs of all GPUs are exchanged "
                          "(1-bit all-gather or int8 SUM all-reduce, NCCL) before one vote over all workers; "

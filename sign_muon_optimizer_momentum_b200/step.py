@@ -144,12 +144,16 @@ class SignMuonStep:
                                      self.ws_spec.numel(), stream)
 
     def newton_schulz(self, stream: int, out_mode: Optional[int] = None, outs=None) -> None:
-        if out_mode is None:
-            out_mode = L.SIGNMUON_OUT_PACK1 if self.variant == "pack1" else L.SIGNMUON_OUT_INT8
-        outs = self.signs if outs is None else outs
-        optrs = [o.data_ptr() for o in outs]
+        self._ns_plan_for(stream, out_mode, outs)
+        a, b, c = self.coeffs
+        L.signmuon_newton_schulz_run(self._ns_plan, self.k, a, b, c, 0.0, stream)
+
+    def _ns_plan_for(self, stream: int, out_mode: Optional[int], outs) -> None:
         # The unit table (tensor maps, buffer addresses) is built once per set
         # of output buffers; every later call only launches the iterations.
+        if out_mode is None:
+            out_mode = L.SIGNMUON_OUT_PACK1 if self.variant == "pack1" else L.SIGNMUON_OUT_INT8
+        optrs = [o.data_ptr() for o in (self.signs if outs is None else outs)]
         key = (out_mode, tuple(optrs))
         if self._ns_plan_key != key:
             self._ns_plan = L.signmuon_newton_schulz_plan(
@@ -157,8 +161,15 @@ class SignMuonStep:
                 out_mode, optrs, L.SIGNMUON_F32, None, self.ws_ns.data_ptr(), self.ws_ns.numel(), stream,
                 plan=self._ns_plan)
             self._ns_plan_key = key
-        a, b, c = self.coeffs
-        L.signmuon_newton_schulz_run(self._ns_plan, self.k, a, b, c, 0.0, stream)
+
+    def _polar_plan_for(self, wptr, stream: int) -> None:
+        key = tuple(wptr)
+        if self._polar_plan_key != key:
+            self._polar_plan = L.signmuon_newton_schulz_plan(
+                self.shapes, 1, [v.data_ptr() for v in self.vote], self.vote_inv.data_ptr(),
+                L.SIGNMUON_OUT_UPDATE_W, None, _dtype_code(self.w_dtype), wptr, self.ws_polar.data_ptr(),
+                self.ws_polar.numel(), stream, plan=self._polar_plan)
+            self._polar_plan_key = key
 
     def vote_update(self, weights: Sequence[torch.Tensor], stream: int) -> None:
         wptr = [_check_buf(w, s, self.w_dtype, f"weight[{i}]")
@@ -174,15 +185,37 @@ class SignMuonStep:
                                None, self.eta, [v.data_ptr() for v in self.vote], self.nnz.data_ptr(),
                                self.vote_inv.data_ptr(), self.ws_vote.data_ptr(), self.ws_vote.numel(),
                                stream)
-        key = tuple(wptr)
-        if self._polar_plan_key != key:
-            self._polar_plan = L.signmuon_newton_schulz_plan(
-                self.shapes, 1, [v.data_ptr() for v in self.vote], self.vote_inv.data_ptr(),
-                L.SIGNMUON_OUT_UPDATE_W, None, _dtype_code(self.w_dtype), wptr, self.ws_polar.data_ptr(),
-                self.ws_polar.numel(), stream, plan=self._polar_plan)
-            self._polar_plan_key = key
+        self._polar_plan_for(wptr, stream)
         a, b, c = self.coeffs
         L.signmuon_newton_schulz_run(self._polar_plan, 1, a, b, c, self.eta, stream)
+
+    def prepare(self, weights: Sequence[torch.Tensor]) -> None:
+        """Builds the Newton-Schulz plans (and the local polar step's plan for
+        these weight tensors) without running a step, on the current stream."""
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        self._ns_plan_for(stream, None, None)
+        if self.polar:
+            wptr = [_check_buf(w, s, self.w_dtype, f"weight[{i}]")
+                    for i, (w, s) in enumerate(zip(weights, self.shapes))]
+            self._polar_plan_for(wptr, stream)
+
+    def capture(self, weights: Sequence[torch.Tensor], grads: Sequence[torch.Tensor]) -> "torch.cuda.CUDAGraph":
+        """Captures one step over these weight and gradient tensors into a CUDA
+        graph: graph.replay() then runs a whole step (every kernel of it, the
+        descriptor uploads included) with one launch from the host, on the
+        values the tensors hold at that time.  The tensors must stay allocated
+        and in place while the graph is used.  Capturing runs nothing."""
+        if len(weights) != len(self.shapes) or len(grads) != self.units:
+            raise ValueError("expected one weight per matrix and one gradient per (matrix, worker)")
+        self.prepare(weights)
+        cur = torch.cuda.current_stream(self.device)
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(cur)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self.step(weights, grads)
+        cur.wait_stream(side)
+        return graph
 
     def step(self, weights: Sequence[torch.Tensor], grads: Sequence[torch.Tensor]) -> None:
         """One optimizer step: updates `weights` (one tensor per matrix) in place

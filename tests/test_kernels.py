@@ -524,6 +524,36 @@ def test_polar_replans_when_weight_buffers_move():
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("polar,norm", [(False, "frobenius"), (True, "frobenius"), (False, "spectral")])
+def test_graph_replay_equals_eager_steps(polar, norm):
+    """SignMuonStep.capture: replaying the captured step equals calling step()
+    (weights and momentum bit for bit), with new gradient values every step."""
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    wl = syn.Workload("graph", ((64, 96), (256, 256), (300, 128)), 3, 2, "pack1", "bf16", g_noise_std=2.0,
+                      polar=polar)
+    dt = torch.bfloat16
+    signal = syn.gradient_signal(wl, 0)
+    gvals = [[syn.worker_gradient(wl, signal[i], i, m, t, 0).cuda() for i in range(3) for m in range(3)]
+             for t in range(3)]
+    results = []
+    for use_graph in (False, True):
+        opt = SignMuonStep(wl.shapes, 3, 2, "pack1", 0.9, 0.02, dt, polar=polar, norm=norm)
+        w = [x.cuda() for x in syn.initial_weights(wl, 0)]
+        g = [torch.empty_like(x) for x in gvals[0]]
+        graph = opt.capture(w, g) if use_graph else None
+        for t in range(3):
+            for dst, src in zip(g, gvals[t]):
+                dst.copy_(src)
+            if graph is not None:
+                graph.replay()
+            else:
+                opt.step(w, g)
+        torch.cuda.synchronize()
+        results.append(([x.cpu() for x in w], [m.cpu() for m in opt.mom]))
+    for a, b in zip(results[0][0] + results[0][1], results[1][0] + results[1][1]):
+        assert torch.equal(a, b)
+
+
 def test_nan_gradient_gives_all_plus_signs():
     """A NaN anywhere in one worker's gradient makes its normalised momentum
     (and U) NaN everywhere; sign(NaN) is +1 (bit = !(u < 0)), as in the
