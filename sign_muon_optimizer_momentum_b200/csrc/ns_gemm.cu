@@ -754,18 +754,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             const int wpr = (uf.cols + 31) >> 5;
             static_cast<uint32_t*>(uf.out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
           } else if (L.out_kind == kOutInt8) {
+            // A lane writes 32 bytes of its row, in the widest stores the
+            // row's alignment allows (the row starts at grow * cols bytes;
+            // gc0 is a multiple of 32).
             int8_t* o = static_cast<int8_t*>(uf.out) + (int64_t)grow * uf.cols + gc0;
+            uint32_t pk[8];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+              uint32_t x = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) x |= (uint32_t)((v[4 * w + j] < 0.f) ? 0xFFu : 0x01u) << (8 * j);
+              pk[w] = x;
+            }
             if (nvalid == 32 && (uf.cols & 15) == 0) {
-              uint32_t pk[8];
-#pragma unroll
-              for (int w = 0; w < 8; ++w) {
-                uint32_t x = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) x |= (uint32_t)((v[4 * w + j] < 0.f) ? 0xFFu : 0x01u) << (8 * j);
-                pk[w] = x;
-              }
               reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
               reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            } else if (nvalid == 32 && (uf.cols & 7) == 0) {
+#pragma unroll
+              for (int w = 0; w < 4; ++w) reinterpret_cast<uint2*>(o)[w] = make_uint2(pk[2 * w], pk[2 * w + 1]);
+            } else if (nvalid == 32 && (uf.cols & 3) == 0) {
+#pragma unroll
+              for (int w = 0; w < 8; ++w) reinterpret_cast<uint32_t*>(o)[w] = pk[w];
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -783,17 +792,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                 if (j < nvalid) o[j] = v[j];
             }
           } else {  // kOutUpdateW: W <- W - eta * U
+            // 16-byte vectors when the row is aligned for them; the loads
+            // are all issued before the stores.
             const int64_t off = (int64_t)grow * uf.cols + gc0;
             if (L.w_dtype == SIGNMUON_BF16) {
               __nv_bfloat16* w = static_cast<__nv_bfloat16*>(uf.out) + off;
+              if (nvalid == 32 && (uf.cols & 7) == 0) {
+                uint4 raw[4];
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nvalid) w[j] = __float2bfloat16_rn(fmaf(-L.eta, v[j], __bfloat162float(w[j])));
+                for (int q4 = 0; q4 < 4; ++q4) raw[q4] = reinterpret_cast<const uint4*>(w)[q4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&raw[q4]);
+#pragma unroll
+                  for (int j = 0; j < 8; ++j)
+                    e[j] = __float2bfloat16_rn(fmaf(-L.eta, v[8 * q4 + j], __bfloat162float(e[j])));
+                  reinterpret_cast<uint4*>(w)[q4] = raw[q4];
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nvalid) w[j] = __float2bfloat16_rn(fmaf(-L.eta, v[j], __bfloat162float(w[j])));
+              }
             } else {
               float* w = static_cast<float*>(uf.out) + off;
+              if (nvalid == 32 && (uf.cols & 3) == 0) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);
+                for (int h = 0; h < 2; ++h) {  // two halves of 16 weights (register pressure)
+                  float4 x[4];
+#pragma unroll
+                  for (int q4 = 0; q4 < 4; ++q4) x[q4] = reinterpret_cast<const float4*>(w)[4 * h + q4];
+#pragma unroll
+                  for (int q4 = 0; q4 < 4; ++q4) {
+                    const int j = 16 * h + 4 * q4;
+                    x[q4].x = fmaf(-L.eta, v[j + 0], x[q4].x);
+                    x[q4].y = fmaf(-L.eta, v[j + 1], x[q4].y);
+                    x[q4].z = fmaf(-L.eta, v[j + 2], x[q4].z);
+                    x[q4].w = fmaf(-L.eta, v[j + 3], x[q4].w);
+                    reinterpret_cast<float4*>(w)[4 * h + q4] = x[q4];
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);
+              }
             }
           }
         }

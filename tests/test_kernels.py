@@ -270,7 +270,9 @@ def test_newton_schulz_matches_oracle(shapes, M, k):
 def test_newton_schulz_fused_outputs_are_signs_of_u():
     """The packed and int8 epilogues write exactly the signs of the fp32 U the
     same launch configuration produces (sign(0) = +1)."""
-    shapes, M, k = [(96, 300), (300, 96), (64, 147)], 2, 2
+    # cols % 16 == 0, % 8 == 0, % 4 == 0 and odd: every store width of the
+    # int8 epilogue, wide and tall.
+    shapes, M, k = [(96, 300), (300, 96), (64, 147), (200, 1000), (1000, 104)], 2, 2
     grads, moms = seeded_state(shapes, M, 7)
     xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.cuda() for m in moms], 0.9,
                            torch.float32)
@@ -391,14 +393,15 @@ def test_newton_schulz_k0_and_zero_input():
 def test_polar_step_update(w_dtype):
     """Vote-out, then one Newton-Schulz iteration on the voted matrix fused with
     W <- W - eta * U_V (the optional local polar step)."""
-    shapes, M, eta = [(256, 256), (128, 384)], 4, 0.02
+    # Aligned rows (vector update) and ragged ones (cols % 8 != 0, odd).
+    shapes, M, eta = [(256, 256), (128, 384), (100, 147), (72, 300)], 4, 0.02
     all_signs = [_signs(s, M, seed=20 + i) for i, s in enumerate(shapes)]
     flat = []
     for s_list, shp in zip(all_signs, shapes):
         flat += _packed_device(s_list, shp)
     votes = [torch.zeros((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device="cuda") for r, c in shapes]
-    nnz = torch.zeros(2, dtype=torch.int64, device="cuda")
-    inv = torch.zeros(4, dtype=torch.float32, device="cuda")
+    nnz = torch.zeros(len(shapes), dtype=torch.int64, device="cuda")
+    inv = torch.zeros(len(shapes), dtype=torch.float32, device="cuda")
     wk = ws(L.signmuon_vote_workspace_bytes(shapes, M))
     L.signmuon_vote_update(shapes, M, False, [x.data_ptr() for x in flat], L.SIGNMUON_F32, None, eta,
                            [v.data_ptr() for v in votes], nnz.data_ptr(), inv.data_ptr(), wk.data_ptr(),
