@@ -128,6 +128,17 @@ int ns_tiles(int rows, int cols, int stage, int pair) {
 
 size_t ns_desc_bytes(int n_units) { return align_up((size_t)n_units * sizeof(NsUnit), 1024); }
 
+// Bytes of the tile records of every unit in every stage, for whichever tile
+// mode a wave picks (the larger count of the two).
+size_t ns_rec_bytes(const signmuon_shape* shapes, int n_mats, int n_workers) {
+  size_t n = 0;
+  for (int i = 0; i < n_mats; ++i)
+    for (int stg = 0; stg < 3; ++stg)
+      n += (size_t)n_workers * std::max(ns_tiles(shapes[i].rows, shapes[i].cols, stg, 0),
+                                         ns_tiles(shapes[i].rows, shapes[i].cols, stg, 1));
+  return align_up(n * sizeof(NsTileRec), 1024);
+}
+
 }  // namespace
 
 extern "C" {
@@ -306,7 +317,7 @@ size_t signmuon_newton_schulz_workspace_bytes(const signmuon_shape* shapes, int 
     const size_t b = ns_unit_bytes(shapes[i]).total;
     arena = minimal ? std::max(arena, b) : arena + b * n_workers;
   }
-  return kWsHeaderBytes + ns_desc_bytes(units) + arena;
+  return kWsHeaderBytes + ns_desc_bytes(units) + ns_rec_bytes(shapes, n_mats, n_workers) + arena;
 }
 
 }  // extern "C"
@@ -319,12 +330,14 @@ namespace {
 struct NsPlanHeader {
   uint64_t magic;
   uint8_t* workspace;
+  const float* scales;  // inv_norm
   int64_t max_elems;
   int32_t n_units, n_waves, out_mode, w_dtype;
 };
 struct NsPlanWave {
   int32_t u0, nu;
   int32_t total[3], pair[3];
+  int64_t rec0[3];  // first tile record of each stage (index into the record table)
 };
 constexpr uint64_t kNsPlanMagic = 0x314e4c50534e4d53ull;  // "SMNSPLN1"
 constexpr size_t kNsPlanHeaderBytes = (sizeof(NsPlanHeader) + 63) / 64 * 64;
@@ -371,8 +384,10 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   NsUnit* d_units = reinterpret_cast<NsUnit*>(ws + kWsHeaderBytes);
-  uint8_t* arena = ws + kWsHeaderBytes + ns_desc_bytes(units);
-  const size_t arena_bytes = ws_bytes - kWsHeaderBytes - ns_desc_bytes(units);
+  NsTileRec* d_recs = reinterpret_cast<NsTileRec*>(ws + kWsHeaderBytes + ns_desc_bytes(units));
+  const size_t tables = kWsHeaderBytes + ns_desc_bytes(units) + ns_rec_bytes(shapes, n_mats, n_workers);
+  uint8_t* arena = ws + tables;
+  const size_t arena_bytes = ws_bytes - tables;
 
   // Plan waves: consecutive units whose buffers fit the arena together.
   std::vector<NsUnit> hu(units);
@@ -432,6 +447,7 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
   NsPlanHeader* hdr = static_cast<NsPlanHeader*>(plan);
   NsPlanWave* waves = plan_waves(plan);
   const int n_waves = (int)wave_begin.size() - 1;
+  std::vector<NsTileRec> recs;
   for (int wv = 0; wv < n_waves; ++wv) {
     NsPlanWave& W = waves[wv];
     W.u0 = wave_begin[wv];
@@ -446,18 +462,24 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
       if (forced_mode >= 0) pair = forced_mode;
       W.pair[stg] = pair;
       int pre = 0;
+      W.rec0[stg] = (int64_t)recs.size();
       for (int ui = W.u0; ui < W.u0 + W.nu; ++ui) {
         hu[ui].tile_begin[stg] = pre;
         hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg, pair);
         pre += hu[ui].tile_count[stg];
+        for (int li = 0; li < hu[ui].tile_count[stg]; ++li)
+          recs.push_back(NsTileRec{ui - W.u0, li, hu[ui].rows, hu[ui].cols});
       }
       W.total[stg] = pre;
     }
   }
+  if (recs.size() * sizeof(NsTileRec) > ns_rec_bytes(shapes, n_mats, n_workers)) return SIGNMUON_ERR_WORKSPACE;
   cudaError_t e = upload_bytes(d_units, hu.data(), hu.size() * sizeof(NsUnit), s);
+  if (e == cudaSuccess) e = upload_bytes(d_recs, recs.data(), recs.size() * sizeof(NsTileRec), s);
   if (e != cudaSuccess) return cuda_status(e);
   hdr->magic = kNsPlanMagic;
   hdr->workspace = ws;
+  hdr->scales = inv_norm;
   hdr->max_elems = max_elems;
   hdr->n_units = units;
   hdr->n_waves = n_waves;
@@ -470,6 +492,8 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
   const NsPlanHeader* hdr = static_cast<const NsPlanHeader*>(plan);
   const NsPlanWave* waves = reinterpret_cast<const NsPlanWave*>(static_cast<const uint8_t*>(plan) + kNsPlanHeaderBytes);
   NsUnit* d_units = reinterpret_cast<NsUnit*>(hdr->workspace + kWsHeaderBytes);
+  const NsTileRec* d_recs =
+      reinterpret_cast<const NsTileRec*>(hdr->workspace + kWsHeaderBytes + ns_desc_bytes(hdr->n_units));
   cudaError_t e = cudaSuccess;
   for (int wv = 0; wv < hdr->n_waves; ++wv) {
     const NsPlanWave& W = waves[wv];
@@ -482,6 +506,7 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
       NsLaunch L;
       memset(&L, 0, sizeof(L));
       L.units = d_units + W.u0;
+      L.scales = hdr->scales + W.u0;
       L.n_units = W.nu;
       L.parity = it & 1;
       L.first = it == 0;
@@ -493,6 +518,7 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
       L.err = reinterpret_cast<uint32_t*>(hdr->workspace);
       for (int stg = 0; stg < 3; ++stg) {
         L.stage = stg;
+        L.recs = d_recs + W.rec0[stg];
         L.total_tiles = W.total[stg];
         L.pair = W.pair[stg];
         L.out_kind = (stg == kStageApply && it == k - 1) ? hdr->out_mode : (int)kOutIterate;

@@ -90,8 +90,20 @@ struct alignas(64) NsUnit {
 };
 static_assert(sizeof(NsUnit) % 64 == 0, "NsUnit must keep 64-byte alignment");
 
+// One tile of a Newton-Schulz launch, laid out on the host in launch order,
+// so that a CTA learns its next tile's unit and geometry from one 16-byte
+// load issued a tile ahead (no search over the unit table).
+struct NsTileRec {
+  int32_t unit;   // index into the launch's unit table
+  int32_t li;     // tile index within the unit (the tile_of numbering)
+  int32_t rows, cols;
+};
+static_assert(sizeof(NsTileRec) == 16, "tile records are read as one 16-byte load");
+
 struct NsLaunch {
   const NsUnit* units;
+  const NsTileRec* recs;  // total_tiles records of this launch's stage
+  const float* scales;    // scales[u] = 1 / norm of unit u (first iteration)
   int n_units;
   int stage;        // NsStage
   int parity;       // 0: X_in = x, X_out = xalt; 1: the reverse

@@ -310,35 +310,24 @@ struct GemmCfg {
 // b, b + grid, b + 2 grid, ...  Every role walks the same sequence with its
 // own cursor, so a unit's record is read once per unit, not once per tile.
 // ---------------------------------------------------------------------------
-struct UnitCursor {
-  int idx = -1;    // current unit
-  int begin = 0;   // its first tile
-  int end = 0;     // one past its last tile
-  int rows = 0, cols = 0;
-};
-
-// Moves the cursor to the unit holding tile t (t never decreases).  Returns
-// true when the unit changed.
-__device__ __forceinline__ bool cursor_seek(const NsLaunch& L, UnitCursor& c, int t) {
-  if (c.idx >= 0 && t < c.end) return false;
-  int lo = c.idx < 0 ? 0 : c.idx + 1;
-  if (c.idx >= 0 && lo < L.n_units && t < L.units[lo].tile_begin[L.stage] + L.units[lo].tile_count[L.stage]) {
-    // common case: the next unit
-  } else {
-    int hi = L.n_units - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (L.units[mid].tile_begin[L.stage] <= t) lo = mid; else hi = mid - 1;
-    }
+// Tile records of one CTA's tiles t0, t0 + stride, ...: the record of the
+// tile after the current one is loaded while the current one is processed.
+struct RecStream {
+  NsTileRec next;
+  __device__ __forceinline__ void start(const NsLaunch& L, int t0) {
+    if (t0 < L.total_tiles) next = load(L, t0);
   }
-  const NsUnit& u = L.units[lo];
-  c.idx = lo;
-  c.begin = u.tile_begin[L.stage];
-  c.end = c.begin + u.tile_count[L.stage];
-  c.rows = u.rows;
-  c.cols = u.cols;
-  return true;
-}
+  // The record of tile t; issues the load of tile t + stride's.
+  __device__ __forceinline__ NsTileRec advance(const NsLaunch& L, int t, int stride) {
+    const NsTileRec cur = next;
+    if (t + stride < L.total_tiles) next = load(L, t + stride);
+    return cur;
+  }
+  static __device__ __forceinline__ NsTileRec load(const NsLaunch& L, int t) {
+    const int4 v = __ldg(reinterpret_cast<const int4*>(L.recs + t));
+    return NsTileRec{v.x, v.y, v.z, v.w};
+  }
+};
 
 struct Tile {
   int M, N, K;
@@ -489,16 +478,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      UnitCursor cur;
+      RecStream rs;
+      rs.start(L, first_tile);
+      int cur_unit = -1;
       const CUtensorMap* ma = nullptr;
       const CUtensorMap* mb = nullptr;
       for (int t = first_tile; t < L.total_tiles && ok; t += tile_stride) {
-        if (cursor_seek(L, cur, t)) {
-          operand_maps(L, &L.units[cur.idx], cur.rows > cur.cols, ma, mb);
+        const NsTileRec rec = rs.advance(L, t, tile_stride);
+        if (rec.unit != cur_unit) {
+          cur_unit = rec.unit;
+          operand_maps(L, &L.units[rec.unit], rec.rows > rec.cols, ma, mb);
           tensormap_acquire(ma);
           tensormap_acquire(mb);
         }
-        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
+        const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
         const int nkb = (T.K + kBK - 1) / kBK;
         const int a_row0 = T.m0 + (int)rank * C::kRowsA;
         const int b_row0 = T.n0 + (int)rank * C::kRowsB;
@@ -551,10 +544,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      UnitCursor cur;
+      RecStream rs;
+      rs.start(L, first_tile);
       for (int t = first_tile; t < L.total_tiles && ok; t += tile_stride) {
-        cursor_seek(L, cur, t);
-        const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
+        const NsTileRec rec = rs.advance(L, t, tile_stride);
+        const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
         // The square stage multiplies the fp16 A and P; all others are bf16.
         const uint32_t idesc = instr_desc(T.a_mn, T.b_mn, C::kTileM, L.stage == kStageSquare);
         const bool b_from_a = diag_b_from_a<kPair>(L, T);
@@ -624,9 +618,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     int stage_flip = 0;           // staging block of the next iterate store
     int acc = 0;
     uint32_t acc_phase = 0;
-    UnitCursor cur;
+    RecStream rs;
+    rs.start(L, first_tile);
+    int cur_unit = -1;
     // The unit's fields are copied to registers once per unit: read through
     // a global pointer they would be reloaded after every store (aliasing).
+    // Their loads are issued before the wait for the accumulator.
     struct {
       const CUtensorMap* st_out;  // store map of this stage's bf16 output
       const CUtensorMap* st_p;    // Gram stage: store map of P = bI + cA
@@ -635,17 +632,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     } uf = {nullptr, nullptr, nullptr, 0};
     float s = 1.f;
     for (int t = first_tile; t < L.total_tiles; t += tile_stride) {
-      if (cursor_seek(L, cur, t)) {
-        const NsUnit* un = &L.units[cur.idx];
+      const NsTileRec rec = rs.advance(L, t, tile_stride);
+      if (rec.unit != cur_unit) {
+        cur_unit = rec.unit;
+        const NsUnit* un = &L.units[rec.unit];
         uf.st_out = L.stage == kStageGram ? &un->st_a
                   : L.stage == kStageSquare ? &un->st_b
                   : (L.parity ? &un->st_x : &un->st_xalt);
         uf.st_p = &un->st_p;
         uf.out = un->out;
-        uf.cols = un->cols;
-        s = L.first ? *un->scale : 1.f;
+        uf.cols = rec.cols;
+        s = L.first ? __ldg(L.scales + rec.unit) : 1.f;
       }
-      const Tile T = tile_of(L.stage, cur.rows, cur.cols, t - cur.begin, C::kTileM);
+      const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
       if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag)) {
         atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutEpilogue);
         *abort_flag = 1;

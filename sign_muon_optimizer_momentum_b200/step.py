@@ -249,15 +249,21 @@ class SignMuonStep:
 
     @staticmethod
     def _waves(shapes, M, ws_bytes) -> int:
+        """Waves the library splits the units into for this workspace size
+        (its buffers per unit: A, P, B' and an X copy, 1 KB aligned)."""
         def al(x, a):
             return (x + a - 1) // a * a
-        units = len(shapes) * M
-        arena = ws_bytes - 256 - al(units * 1408, 1024)
+
+        def unit_bytes(r, c):
+            s = min(r, c)
+            return 3 * al(s * al(s, 8) * 2, 1024) + al(r * al(c, 8) * 2, 1024)
+        # The minimal workspace is the tables plus the largest unit's buffers.
+        tables = (L.signmuon_newton_schulz_workspace_bytes(shapes, M, minimal=True)
+                  - max(unit_bytes(r, c) for r, c in shapes))
+        arena = ws_bytes - tables
         waves, used = 0, arena
         for (r, c) in shapes:
-            s = min(r, c)
-            lds = al(s, 8)
-            b = 3 * al(s * lds * 2, 1024) + al(r * al(c, 8) * 2, 1024)
+            b = unit_bytes(r, c)
             for _ in range(M):
                 if used + b > arena:
                     waves += 1
