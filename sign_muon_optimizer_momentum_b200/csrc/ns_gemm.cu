@@ -59,10 +59,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -129,8 +125,17 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Arrivals that order execution only, with no memory release: an epilogue
+// thread signals that it has finished reading an accumulator (its
+// tcgen05.ld waited on, then tcgen05.fence::before_thread_sync).  The MMA
+// thread reads nothing the epilogue wrote, so a release -- which would
+// first wait for the epilogue's outstanding global stores to become
+// visible across the cluster -- is not needed.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Bulk tensor store of a 32x32 block from shared memory (async proxy).
@@ -842,9 +847,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       }
       tc_fence_before();
       if constexpr (kPair)
-        mbar_arrive_cluster(map_to_rank(smem_addr(&tempty_bar[acc]), 0));  // the even CTA's barrier
+        mbar_arrive_relaxed_cluster(map_to_rank(smem_addr(&tempty_bar[acc]), 0));  // the even CTA's barrier
       else
-        mbar_arrive(smem_addr(&tempty_bar[acc]));
+        mbar_arrive_relaxed(smem_addr(&tempty_bar[acc]));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
     // All of this warp's bulk stores must complete before the CTA exits.
