@@ -471,6 +471,15 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
           recs.push_back(NsTileRec{ui - W.u0, li, hu[ui].rows, hu[ui].cols});
       }
       W.total[stg] = pre;
+      // Launch order: longest reduction first (the Gram's K is the long
+      // side, the other stages' the short one), so that the round-robin
+      // assignment of tiles to CTAs ends on short tiles; a stable sort keeps
+      // each unit's tiles together.
+      auto k_of = [stg](const NsTileRec& r) {
+        return stg == kStageGram ? std::max(r.rows, r.cols) : std::min(r.rows, r.cols);
+      };
+      std::stable_sort(recs.begin() + W.rec0[stg], recs.end(),
+                       [&](const NsTileRec& x, const NsTileRec& y) { return k_of(x) > k_of(y); });
     }
   }
   if (recs.size() * sizeof(NsTileRec) > ns_rec_bytes(shapes, n_mats, n_workers)) return SIGNMUON_ERR_WORKSPACE;

@@ -84,8 +84,8 @@ struct alignas(64) NsUnit {
   void* out;             // final output (packed / int8 / fp32 U / W)
   const float* scale;    // &inv_norm[u]
   int32_t rows, cols, ld_x, ld_s;
-  int32_t tile_begin[3];  // prefix of tiles over the launch's units, per stage
-  int32_t tile_count[3];
+  int32_t tile_begin[3];  // host bookkeeping: first tile of the unit in unit order, per stage
+  int32_t tile_count[3];  //   and its tile count (the kernels read the tile records)
   int32_t pad_[2];
 };
 static_assert(sizeof(NsUnit) % 64 == 0, "NsUnit must keep 64-byte alignment");

@@ -310,10 +310,9 @@ struct GemmCfg {
 };
 
 // ---------------------------------------------------------------------------
-// Tile scheduling.  Tiles of a launch are numbered unit by unit (each unit's
-// tiles are consecutive, prefix in NsUnit::tile_begin); CTA b takes tiles
-// b, b + grid, b + 2 grid, ...  Every role walks the same sequence with its
-// own cursor, so a unit's record is read once per unit, not once per tile.
+// Tile scheduling.  The host lists a launch's tiles as records (unit, tile
+// within the unit, shape), longest reduction first; CTA (pair) b takes
+// records b, b + grid, b + 2 grid, ...  Every role walks the same sequence.
 // ---------------------------------------------------------------------------
 // Tile records of one CTA's tiles t0, t0 + stride, ...: the record of the
 // tile after the current one is loaded while the current one is processed.
