@@ -126,6 +126,15 @@ int ns_tiles(int rows, int cols, int stage, int pair) {
   return n;
 }
 
+// SMs of the current device (148 on B200; 148 if the query fails).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    return 148;
+  return n;
+}
+
 size_t ns_desc_bytes(int n_units) { return align_up((size_t)n_units * sizeof(NsUnit), 1024); }
 
 // Bytes of the tile records of every unit in every stage, for whichever tile
@@ -471,15 +480,21 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
           recs.push_back(NsTileRec{ui - W.u0, li, hu[ui].rows, hu[ui].cols});
       }
       W.total[stg] = pre;
-      // Launch order: longest reduction first (the Gram's K is the long
-      // side, the other stages' the short one), so that the round-robin
-      // assignment of tiles to CTAs ends on short tiles; a stable sort keeps
-      // each unit's tiles together.
-      auto k_of = [stg](const NsTileRec& r) {
-        return stg == kStageGram ? std::max(r.rows, r.cols) : std::min(r.rows, r.cols);
-      };
-      std::stable_sort(recs.begin() + W.rec0[stg], recs.end(),
-                       [&](const NsTileRec& x, const NsTileRec& y) { return k_of(x) > k_of(y); });
+      // Launch order.  With few tiles per CTA (pair) the round-robin
+      // assignment leaves CTAs unevenly loaded when tiles differ in length:
+      // then the longest reductions go first (the Gram's K is the long side,
+      // the other stages' the short one) so that the launch ends on short
+      // tiles.  With many tiles per CTA the unit order stays, which keeps
+      // the tiles running at the same time on few units (L2 reuse of their
+      // operands).  The sort is stable: a unit's tiles stay together.
+      const int workers = pair ? sm_count() / 2 : sm_count();
+      if (W.total[stg] < 8 * workers) {
+        auto k_of = [stg](const NsTileRec& r) {
+          return stg == kStageGram ? std::max(r.rows, r.cols) : std::min(r.rows, r.cols);
+        };
+        std::stable_sort(recs.begin() + W.rec0[stg], recs.end(),
+                         [&](const NsTileRec& x, const NsTileRec& y) { return k_of(x) > k_of(y); });
+      }
     }
   }
   if (recs.size() * sizeof(NsTileRec) > ns_rec_bytes(shapes, n_mats, n_workers)) return SIGNMUON_ERR_WORKSPACE;

@@ -311,8 +311,9 @@ struct GemmCfg {
 
 // ---------------------------------------------------------------------------
 // Tile scheduling.  The host lists a launch's tiles as records (unit, tile
-// within the unit, shape), longest reduction first; CTA (pair) b takes
-// records b, b + grid, b + 2 grid, ...  Every role walks the same sequence.
+// within the unit, shape) -- in unit order, or longest reduction first when
+// each CTA gets few tiles; CTA (pair) b takes records b, b + grid,
+// b + 2 grid, ...  Every role walks the same sequence.
 // ---------------------------------------------------------------------------
 // Tile records of one CTA's tiles t0, t0 + stride, ...: the record of the
 // tile after the current one is loaded while the current one is processed.
