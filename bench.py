@@ -452,13 +452,22 @@ def run_gpu(args, wl):
             flops_note = "Newton-Schulz call of the step"
         achieved = flops / (ns_ms / 1e3) / 1e12
         dense = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters, True) / (ns_ms / 1e3) / 1e12
+        # The kernel runs inside the timed steps back to back: over a timed
+        # region of half a second or more the GPU sits at its power cap, the
+        # condition of the sustained bf16 peak; shorter regions compare with
+        # the burst peak.
+        sustained = ms >= 500.0
+        peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
         roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved,
-                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                     "traffic": captured_traffic("ns_gemm_kernel", wl.name),
                     "note": f"{flops_note}: {flops / 1e12:.3f} TFLOP algorithmic (symmetric-aware: 3s^2l + s^3 "
                             f"per iteration and unit) per step over {ns_ms:.3f} ms (CUDA events, mean of "
-                            f"{args.steps} timed steps); dense-equivalent {dense:.1f} TFLOP/s; peak = "
-                            f"{pk['source']} burst bf16 cuBLAS (sustained {pk['bf16_tflops_sustained']})"}
+                            f"{args.steps} timed steps, {ms / 1e3:.2f} s of timed work); dense-equivalent "
+                            f"{dense:.1f} TFLOP/s; peak = {pk['source']} "
+                            f"{'sustained' if sustained else 'burst'} bf16 cuBLAS (burst {pk['bf16_tflops']}, "
+                            f"sustained {pk['bf16_tflops_sustained']}); frac of burst "
+                            f"{achieved / pk['bf16_tflops']:.3f}"}
     else:
         # k = 0 (majority-vote Signum): the momentum pass dominates.
         gbytes = wl.params * wl.n_workers * ((2 if wl.w_dtype == "bf16" else 4) + 8 + 2)
