@@ -56,13 +56,28 @@ cudaError_t upload_bytes(void* dst_device, const void* src_host, size_t bytes,
 // ---------------------------------------------------------------------------
 // Momentum
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int find_block_unit(const MomUnit* units, int n_units, int b) {
-  int lo = 0, hi = n_units - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (units[mid].block_begin <= b) lo = mid; else hi = mid - 1;
+// Index of the last entry i in [0, n) with begin(i) <= b, for increasing
+// begin() with begin(0) == 0: the table entry that owns block b.  Called by
+// whole warps: each round loads 32 entries in parallel and picks one by
+// ballot, so a table of n entries costs ceil(log32 n) load latencies instead
+// of the log2 n dependent loads of a binary search.
+template <typename Begin>
+__device__ __forceinline__ int find_owner(int n, int b, Begin begin) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, count = n;
+  while (count > 1) {
+    const int step = (count + 31) / 32;  // entries per lane's slot
+    const bool le = lane * step < count && begin(lo + lane * step) <= b;
+    const unsigned m = __ballot_sync(0xffffffffu, le);
+    const int l = 31 - __clz(m);         // last slot starting at or before b (slot 0 always does)
+    lo += l * step;
+    count = min(step, count - l * step);
   }
   return lo;
+}
+
+__device__ __forceinline__ int find_block_unit(const MomUnit* units, int n_units, int b) {
+  return find_owner(n_units, b, [&](int i) { return __ldg(&units[i].block_begin); });
 }
 
 __device__ __forceinline__ float load_grad(const void* g, int64_t i, int bf16) {
@@ -381,12 +396,7 @@ __device__ __forceinline__ void update4_f32(float4& x, uint32_t gt, uint32_t tie
 }
 
 __device__ __forceinline__ int find_vote_mat(const VoteMat* mats, int n, int b) {
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (mats[mid].block_begin <= b) lo = mid; else hi = mid - 1;
-  }
-  return lo;
+  return find_owner(n, b, [&](int i) { return __ldg(&mats[i].block_begin); });
 }
 
 // Packed fast path (cols % 32 == 0): packed word w covers W[32w, 32w+32).
@@ -737,12 +747,7 @@ int vote_blocks_for(int int8_in, int w_bf16, int vote_out, int cols, int64_t n, 
 // from v0 = 1/sqrt(n); inv_norm = 1 / (sigma_est + 1e-7).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int find_spec_unit(const SpecUnit* u, int n, int b) {
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (u[mid].block_begin <= b) lo = mid; else hi = mid - 1;
-  }
-  return lo;
+  return find_owner(n, b, [&](int i) { return __ldg(&u[i].block_begin); });
 }
 
 __global__ void spectral_init_kernel(const SpecUnit* __restrict__ units, float* __restrict__ vecs) {
@@ -777,6 +782,8 @@ spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const f
     if (rr < nrows) {
       const __nv_bfloat16* xr = u.x + (int64_t)(r0 + rr) * u.ld_x;
       if (vec) {
+        // Unrolled so that several 16-byte loads of the row are in flight.
+#pragma unroll 4
         for (int j = lane * 8; j < u.cols; j += 256) {
           const uint4 raw = *reinterpret_cast<const uint4*>(xr + j);
           const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -803,6 +810,7 @@ spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const f
   if (vec) {
     for (int j = threadIdx.x * 8; j < u.cols; j += 256 * 8) {
       float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
       for (int rr = 0; rr < nrows; ++rr) {
         const uint4 raw = *reinterpret_cast<const uint4*>(u.x + (int64_t)(r0 + rr) * u.ld_x + j);
         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
