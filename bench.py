@@ -7,8 +7,10 @@ workload: momentum + Frobenius norm, k Newton-Schulz iterations with the sign
 fused into the last one, and the majority vote fused with the update (plus
 the local polar step when the workload has it).  The metric is
 params * workers / s (whole job); inputs are resident in HBM and larger than
-L2.  With N > 1 (torchrun) every rank runs an independent replica: the path
-has no exchange step because the M workers are buffers on one GPU.
+L2.  With N > 1 (torchrun) every rank runs an independent replica by default:
+the M workers are buffers on one GPU, so the step has no exchange; with
+--exchange every rank runs the workload's workers and the signs of all ranks
+are exchanged (NCCL) before one vote over all of them.
 
 Rank 0 prints one JSON line.  `--impl reference` times the CPU fp64 oracle on
 a bounded sample of the same workload instead.
@@ -469,14 +471,18 @@ def run_gpu(args, wl):
                             f"sustained {pk['bf16_tflops_sustained']}); frac of burst "
                             f"{achieved / pk['bf16_tflops']:.3f}"}
     else:
-        # k = 0 (majority-vote Signum): the momentum pass dominates.
-        gbytes = wl.params * wl.n_workers * ((2 if wl.w_dtype == "bf16" else 4) + 8 + 2)
+        # k = 0 (majority-vote Signum): the momentum pass dominates.  Fused
+        # (the momentum kernel writes the signs) or momentum + bf16 copy.
+        fused = getattr(opt, "fused_sign", False)
+        out_b = (1 / 8 if wl.variant == "pack1" else 1) if fused else 2
+        gbytes = wl.params * wl.n_workers * ((2 if wl.w_dtype == "bf16" else 4) + 8 + out_b)
         achieved = gbytes / (mom_ms / 1e3) / 1e9
+        out_what = ("packed sign" if wl.variant == "pack1" else "int8 sign") if fused else "bf16 copy"
         roofline = {"bound": "hbm", "kernel": "momentum_kernel", "achieved": achieved, "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                     "traffic": captured_traffic("momentum_kernel", wl.name),
                     "note": f"momentum call: {gbytes / 1e9:.3f} GB algorithmic (gradient read, fp32 momentum "
-                            f"read+write, bf16 copy write) per step over {mom_ms:.3f} ms"}
+                            f"read+write, {out_what} write) per step over {mom_ms:.3f} ms"}
     result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

@@ -137,6 +137,35 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
                                        void* stream);
 
 /* ------------------------------------------------------------------------
+ * Steps 1a-2 for k = 0 (the majority-vote Signum / SignSGD baseline),
+ * fused: the momentum update and the signs of X0 = M / (||M||_F + 1e-7)
+ * in one pass, without the bf16 copy of M.
+ * Source: SignMuon summary, section 4 (the Signum / SignSGD baselines the
+ * summary compares against) and section 2 "Algorithmic flow" steps 1-3.
+ *
+ * mom[u] and inv_norm[u] are updated exactly as by signmuon_momentum_norm.
+ * signs[u] receives sign(X0) (+1 for 0, -0 and NaN), which is sign(mom[u])
+ * when the norm is finite and +1 everywhere when it is not (X0 is then NaN
+ * or zero in every entry):
+ *   int8_out == 0: packed words (signmuon_packed_words words per unit, bit
+ *                  j of word w in row r = entry (r, 32w + j), 1 = +1); every
+ *                  cols must be a multiple of 32 (else SIGNMUON_ERR_UNSUPPORTED,
+ *                  and signmuon_momentum_norm + signmuon_newton_schulz_batched
+ *                  with k = 0 serve); trailing pad words are not written.
+ *   int8_out != 0: int8 [rows, cols], any shape.
+ * The signs equal those of signmuon_newton_schulz_batched with k = 0 except
+ * for |M| below about 5e-41, where that path's bf16 copy of M (or its
+ * product with inv_norm) underflows to -0; this call reads the fp32 momentum
+ * itself and keeps those signs, as the fp64 definition does.
+ * Arguments, alignment and workspace as for signmuon_momentum_norm.
+ * ---------------------------------------------------------------------- */
+signmuon_status signmuon_momentum_sign(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                       signmuon_dtype grad_dtype, const void* const* grad,
+                                       float* const* mom, float beta, int int8_out,
+                                       void* const* signs, float* inv_norm, void* workspace,
+                                       size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Step 1a, spectral variant: spectral scaling of the Newton-Schulz input.
  * Source: SignMuon summary, section 4 "nanoGPT" (the method is robust to
  * Frobenius vs spectral scaling of the normalisation).

@@ -41,7 +41,7 @@ EXPORTS = (
     "signmuon_newton_schulz_plan_bytes", "signmuon_newton_schulz_plan", "signmuon_newton_schulz_run",
     "signmuon_sign_pack", "signmuon_vote_workspace_bytes", "signmuon_vote_update",
     "signmuon_momentum_norm_noalloc", "signmuon_last_error_string",
-    "signmuon_spectral_workspace_bytes", "signmuon_spectral_norm",
+    "signmuon_spectral_workspace_bytes", "signmuon_spectral_norm", "signmuon_momentum_sign",
 )
 
 
@@ -72,6 +72,7 @@ _SIGS = {
     "signmuon_momentum_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I]),
     "signmuon_momentum_norm": (_I, [ctypes.POINTER(Shape), _I, _I, _I, _PP, _PP, _F, _PP, _P, _P,
                                     _SZ, _P]),
+    "signmuon_momentum_sign": (_I, [ctypes.POINTER(Shape), _I, _I, _I, _PP, _PP, _F, _I, _PP, _P, _P, _SZ, _P]),
     "signmuon_newton_schulz_workspace_bytes": (_SZ, [ctypes.POINTER(Shape), _I, _I, _I]),
     "signmuon_newton_schulz_batched": (_I, [ctypes.POINTER(Shape), _I, _I, _PP, _P, _I, _F, _F, _F,
                                             _I, _PP, _I, _PP, _F, _P, _SZ, _P]),
@@ -175,6 +176,14 @@ def signmuon_spectral_norm(shapes, n_workers, x_bf16, iters, inv_norm, workspace
     st = load().signmuon_spectral_norm(_shapes(shapes), len(shapes), n_workers, _ptrs(x_bf16), iters, inv_norm,
                                        workspace, ws_bytes, stream)
     _check("signmuon_spectral_norm", st)
+
+
+def signmuon_momentum_sign(shapes, n_workers, grad_dtype, grad, mom, beta, int8_out, signs, inv_norm, workspace,
+                           ws_bytes, stream=0) -> None:
+    st = load().signmuon_momentum_sign(_shapes(shapes), len(shapes), n_workers, grad_dtype, _ptrs(grad),
+                                       _ptrs(mom), beta, int(bool(int8_out)), _ptrs(signs), inv_norm, workspace,
+                                       ws_bytes, stream)
+    _check("signmuon_momentum_sign", st)
 
 
 def signmuon_newton_schulz_workspace_bytes(shapes, n_workers: int, minimal: bool = False) -> int:

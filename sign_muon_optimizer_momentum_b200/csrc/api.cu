@@ -203,10 +203,13 @@ size_t signmuon_momentum_workspace_bytes(const signmuon_shape* shapes, int n_mat
   return kWsHeaderBytes + align_up((size_t)units * sizeof(MomUnit), 256) + align_up((size_t)blocks * 4, 256);
 }
 
-signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats, int n_workers,
-                                       signmuon_dtype grad_dtype, const void* const* grad, float* const* mom,
-                                       float beta, void* const* x_bf16, float* inv_norm, void* workspace,
-                                       size_t ws_bytes, void* stream) {
+// Momentum update with one of three outputs (kernel modes): the bf16 copy of
+// M (0), or the signs of X0 = M / norm packed (1) or int8 (2).  Arguments
+// other than the outputs are validated here.
+static signmuon_status momentum_run(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                    signmuon_dtype grad_dtype, const void* const* grad, float* const* mom,
+                                    float beta, void* const* out, int out_mode, float* inv_norm, void* workspace,
+                                    size_t ws_bytes, void* stream) {
   signmuon_status st = validate_shapes(shapes, n_mats);
   if (st) return st;
   if (n_workers <= 0 || n_workers > SIGNMUON_MAX_WORKERS) return SIGNMUON_ERR_INVALID_ARG;
@@ -214,7 +217,7 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
   const int units = n_mats * n_workers;
   if ((st = validate_ptrs(grad, units))) return st;
   if ((st = validate_ptrs(reinterpret_cast<const void* const*>(mom), units))) return st;
-  if ((st = validate_ptrs(reinterpret_cast<const void* const*>(x_bf16), units))) return st;
+  if ((st = validate_ptrs(reinterpret_cast<const void* const*>(out), units))) return st;
   if (!inv_norm) return SIGNMUON_ERR_INVALID_ARG;
   if (!aligned16(inv_norm)) return SIGNMUON_ERR_ALIGNMENT;
   if ((st = check_workspace(workspace, ws_bytes, signmuon_momentum_workspace_bytes(shapes, n_mats, n_workers))))
@@ -228,7 +231,7 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
       MomUnit& u = mu[i * n_workers + m];
       u.grad = grad[i * n_workers + m];
       u.mom = mom[i * n_workers + m];
-      u.x = static_cast<__nv_bfloat16*>(x_bf16[i * n_workers + m]);
+      u.x = static_cast<__nv_bfloat16*>(out[i * n_workers + m]);
       u.rows = shapes[i].rows;
       u.cols = shapes[i].cols;
       u.n = (int64_t)u.rows * u.cols;
@@ -243,9 +246,32 @@ signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats,
   MomUnit* d_units = reinterpret_cast<MomUnit*>(ws + kWsHeaderBytes);
   float* partials = reinterpret_cast<float*>(ws + kWsHeaderBytes + align_up((size_t)units * sizeof(MomUnit), 256));
   cudaError_t e = upload_bytes(d_units, mu.data(), mu.size() * sizeof(MomUnit), s);
-  if (e == cudaSuccess) e = launch_momentum(d_units, units, blocks, grad_dtype == SIGNMUON_BF16, beta, partials, s);
-  if (e == cudaSuccess) e = launch_momentum_finalize(d_units, units, partials, inv_norm, s);
+  if (e == cudaSuccess)
+    e = launch_momentum(d_units, units, blocks, grad_dtype == SIGNMUON_BF16, beta, partials, out_mode, s);
+  if (e == cudaSuccess) e = launch_momentum_finalize(d_units, units, partials, inv_norm, out_mode, s);
   return cuda_status(e);
+}
+
+signmuon_status signmuon_momentum_norm(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                       signmuon_dtype grad_dtype, const void* const* grad, float* const* mom,
+                                       float beta, void* const* x_bf16, float* inv_norm, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+  return momentum_run(shapes, n_mats, n_workers, grad_dtype, grad, mom, beta, x_bf16, 0, inv_norm, workspace,
+                      ws_bytes, stream);
+}
+
+signmuon_status signmuon_momentum_sign(const signmuon_shape* shapes, int n_mats, int n_workers,
+                                       signmuon_dtype grad_dtype, const void* const* grad, float* const* mom,
+                                       float beta, int int8_out, void* const* signs, float* inv_norm,
+                                       void* workspace, size_t ws_bytes, void* stream) {
+  signmuon_status st = validate_shapes(shapes, n_mats);
+  if (st) return st;
+  // Packed words are written 32 consecutive elements at a time: whole words per row.
+  if (!int8_out)
+    for (int i = 0; i < n_mats; ++i)
+      if (shapes[i].cols % 32) return SIGNMUON_ERR_UNSUPPORTED;
+  return momentum_run(shapes, n_mats, n_workers, grad_dtype, grad, mom, beta, signs, int8_out ? 2 : 1, inv_norm,
+                      workspace, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------ spectral scaling

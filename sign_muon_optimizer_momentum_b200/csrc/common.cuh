@@ -120,7 +120,7 @@ struct NsLaunch {
 struct MomUnit {
   const void* grad;
   float* mom;
-  __nv_bfloat16* x;
+  __nv_bfloat16* x;   // the bf16 copy of M; in the sign modes the packed / int8 sign buffer
   int64_t n;          // rows * cols
   int32_t rows, cols, ld_x;
   int32_t block_begin;  // first block of this unit in the flattened grid
@@ -163,9 +163,9 @@ constexpr int kSpecSmemCols = 8192;  // v is staged in shared memory up to this 
 // ---------------------------------------------------------------------------
 cudaError_t upload_bytes(void* dst_device, const void* src_host, size_t bytes, cudaStream_t stream);
 cudaError_t launch_momentum(const MomUnit* units, int n_units, int total_blocks, int grad_bf16,
-                            float beta, float* partials, cudaStream_t stream);
+                            float beta, float* partials, int out_mode, cudaStream_t stream);
 cudaError_t launch_momentum_finalize(const MomUnit* units, int n_units, const float* partials,
-                                     float* inv_norm, cudaStream_t stream);
+                                     float* inv_norm, int out_mode, cudaStream_t stream);
 cudaError_t launch_sign_pack(signmuon_shape shape, int u_bf16, const void* u, int64_t ld_u,
                              int int8_out, void* out, int64_t out_words, cudaStream_t stream);
 cudaError_t launch_vote(const VoteMat* mats, int n_mats, int total_blocks, const void* const* sign_table,

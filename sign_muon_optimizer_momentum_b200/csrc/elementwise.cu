@@ -91,6 +91,11 @@ __device__ __forceinline__ float momentum_one(float m, float g, double beta, dou
   return (float)fma(beta, (double)m, omb * (double)g);
 }
 
+// What the momentum kernel writes besides the momentum: the bf16 copy X of
+// the Newton-Schulz input, or (k = 0) the signs of X0 = M / norm directly.
+enum MomOut { kMomX = 0, kMomPack = 1, kMomInt8 = 2 };
+
+template <int kOut>
 __global__ void __launch_bounds__(kMomThreads)
 momentum_kernel(const MomUnit* __restrict__ units, int n_units, int grad_bf16, float beta_f,
                 float* __restrict__ partials) {
@@ -106,9 +111,14 @@ momentum_kernel(const MomUnit* __restrict__ units, int n_units, int grad_bf16, f
 #pragma unroll
   for (int it = 0; it < kMomElemsPerThread / 8; ++it) {
     const int64_t e0 = base + (int64_t)it * (kMomThreads * 8) + threadIdx.x * 8;
-    if (e0 >= u.n) break;
+    // The packed mode combines four threads' bits by shuffles, so its warps
+    // stay together: no early exit (units are whole 32-column words there).
+    if constexpr (kOut != kMomPack) {
+      if (e0 >= u.n) break;
+    }
     float g[8], m[8];
-    if (e0 + 8 <= u.n) {
+    const bool full = e0 + 8 <= u.n;
+    if (full) {
       if (grad_bf16) {
         const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(u.grad) + e0);
         const __nv_bfloat162* gp = reinterpret_cast<const __nv_bfloat162*>(&gv);
@@ -135,7 +145,30 @@ momentum_kernel(const MomUnit* __restrict__ units, int n_units, int grad_bf16, f
       }
       *reinterpret_cast<float4*>(u.mom + e0) = make_float4(m[0], m[1], m[2], m[3]);
       *reinterpret_cast<float4*>(u.mom + e0 + 4) = make_float4(m[4], m[5], m[6], m[7]);
-      if (dense) {
+    }
+    if constexpr (kOut == kMomPack) {
+      // sign(X0) = sign(M) for a finite norm (the finalize kernel handles
+      // the others): bit j = !(m_j < 0); lanes 4q..4q+3 hold one word.
+      uint32_t bits = 0;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) bits |= (m[j] < 0.f) ? 0u : (1u << j);
+      }
+      uint32_t word = bits;
+      word |= __shfl_down_sync(0xffffffffu, bits, 1) << 8;
+      word |= __shfl_down_sync(0xffffffffu, bits, 2) << 16;
+      word |= __shfl_down_sync(0xffffffffu, bits, 3) << 24;
+      if (full && (threadIdx.x & 3) == 0) static_cast<uint32_t*>(static_cast<void*>(u.x))[e0 >> 5] = word;
+    } else if (full) {
+      if constexpr (kOut == kMomInt8) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          lo |= (uint32_t)(m[j] < 0.f ? 0xFFu : 0x01u) << (8 * j);
+          hi |= (uint32_t)(m[4 + j] < 0.f ? 0xFFu : 0x01u) << (8 * j);
+        }
+        *reinterpret_cast<uint2*>(reinterpret_cast<int8_t*>(u.x) + e0) = make_uint2(lo, hi);
+      } else if (dense) {
         __nv_bfloat162 xb[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) xb[j] = __floats2bfloat162_rn(m[2 * j], m[2 * j + 1]);
@@ -148,15 +181,19 @@ momentum_kernel(const MomUnit* __restrict__ units, int n_units, int grad_bf16, f
           u.x[r * u.ld_x + c] = __float2bfloat16_rn(m[j]);
         }
       }
-    } else {
+    } else if (e0 < u.n) {
       for (int j = 0; j < 8; ++j) {
         const int64_t e = e0 + j;
         if (e >= u.n) break;
         const float mj = momentum_one(u.mom[e], load_grad(u.grad, e, grad_bf16), beta, omb);
         u.mom[e] = mj;
         ssq = fmaf(mj, mj, ssq);
-        const int64_t r = e / u.cols, c = e - r * u.cols;
-        u.x[r * u.ld_x + c] = __float2bfloat16_rn(mj);
+        if constexpr (kOut == kMomInt8) {
+          reinterpret_cast<int8_t*>(u.x)[e] = mj < 0.f ? int8_t(-1) : int8_t(1);
+        } else {
+          const int64_t r = e / u.cols, c = e - r * u.cols;
+          u.x[r * u.ld_x + c] = __float2bfloat16_rn(mj);
+        }
       }
     }
   }
@@ -175,10 +212,12 @@ momentum_kernel(const MomUnit* __restrict__ units, int n_units, int grad_bf16, f
 }
 
 // inv_norm[u] = 1 / (sqrt(sum of the unit's partials) + 1e-7), partials summed
-// in fp64 in a fixed order.
+// in fp64 in a fixed order.  In the sign modes a unit whose norm is not
+// finite (a NaN or an overflow in M) has X0 = M / norm NaN or zero in every
+// entry, so all its signs are +1: the block overwrites them.
 __global__ void __launch_bounds__(256)
 momentum_finalize_kernel(const MomUnit* __restrict__ units, const float* __restrict__ partials,
-                         float* __restrict__ inv_norm) {
+                         float* __restrict__ inv_norm, int sign_mode) {
   const MomUnit u = units[blockIdx.x];
   double s = 0.0;
   for (int i = threadIdx.x; i < u.block_count; i += blockDim.x) s += (double)partials[u.block_begin + i];
@@ -189,19 +228,34 @@ momentum_finalize_kernel(const MomUnit* __restrict__ units, const float* __restr
     if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
     __syncthreads();
   }
-  if (threadIdx.x == 0) inv_norm[blockIdx.x] = (float)(1.0 / (sqrt(red[0]) + 1e-7));
+  const double norm = sqrt(red[0]);
+  if (threadIdx.x == 0) inv_norm[blockIdx.x] = (float)(1.0 / (norm + 1e-7));
+  if (sign_mode != kMomX && !isfinite((float)norm)) {
+    if (sign_mode == kMomPack) {
+      uint32_t* w = reinterpret_cast<uint32_t*>(u.x);
+      for (int64_t i = threadIdx.x; i < u.n / 32; i += blockDim.x) w[i] = 0xFFFFFFFFu;
+    } else {
+      int8_t* o = reinterpret_cast<int8_t*>(u.x);
+      for (int64_t i = threadIdx.x; i < u.n; i += blockDim.x) o[i] = 1;
+    }
+  }
 }
 
 cudaError_t launch_momentum(const MomUnit* units, int n_units, int total_blocks, int grad_bf16,
-                            float beta, float* partials, cudaStream_t stream) {
+                            float beta, float* partials, int out_mode, cudaStream_t stream) {
   if (total_blocks <= 0) return cudaSuccess;
-  momentum_kernel<<<total_blocks, kMomThreads, 0, stream>>>(units, n_units, grad_bf16, beta, partials);
+  if (out_mode == kMomPack)
+    momentum_kernel<kMomPack><<<total_blocks, kMomThreads, 0, stream>>>(units, n_units, grad_bf16, beta, partials);
+  else if (out_mode == kMomInt8)
+    momentum_kernel<kMomInt8><<<total_blocks, kMomThreads, 0, stream>>>(units, n_units, grad_bf16, beta, partials);
+  else
+    momentum_kernel<kMomX><<<total_blocks, kMomThreads, 0, stream>>>(units, n_units, grad_bf16, beta, partials);
   return cudaGetLastError();
 }
 
 cudaError_t launch_momentum_finalize(const MomUnit* units, int n_units, const float* partials,
-                                     float* inv_norm, cudaStream_t stream) {
-  momentum_finalize_kernel<<<n_units, 256, 0, stream>>>(units, partials, inv_norm);
+                                     float* inv_norm, int out_mode, cudaStream_t stream) {
+  momentum_finalize_kernel<<<n_units, 256, 0, stream>>>(units, partials, inv_norm, out_mode);
   return cudaGetLastError();
 }
 

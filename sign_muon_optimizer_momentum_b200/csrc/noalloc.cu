@@ -108,7 +108,7 @@ extern "C" signmuon_status signmuon_momentum_norm_noalloc(const signmuon_shape* 
   MomUnit* d_units = static_cast<MomUnit*>(scratch);
   float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocTableBytes);
   cudaError_t e = upload_bytes(d_units, mu.data(), mu.size() * sizeof(MomUnit), s);
-  if (e == cudaSuccess) e = launch_momentum(d_units, (int)units, b, grad_dtype == SIGNMUON_BF16, beta, partials, s);
-  if (e == cudaSuccess) e = launch_momentum_finalize(d_units, (int)units, partials, inv_norm, s);
+  if (e == cudaSuccess) e = launch_momentum(d_units, (int)units, b, grad_dtype == SIGNMUON_BF16, beta, partials, 0, s);
+  if (e == cudaSuccess) e = launch_momentum_finalize(d_units, (int)units, partials, inv_norm, 0, s);
   return e == cudaSuccess ? SIGNMUON_OK : SIGNMUON_ERR_CUDA;
 }

@@ -83,13 +83,20 @@ class SignMuonStep:
         dev = self.device
         M = self.n_workers
         self.units = len(self.shapes) * M
+        # k = 0 with the Frobenius scale: sign(X0) = sign(M) (all +1 for a
+        # non-finite norm), so the momentum kernel writes the signs directly
+        # (no bf16 copy of M, no Newton-Schulz call).  Packed signs need whole
+        # 32-column words per row.
+        self.fused_sign = (self.k == 0 and norm == "frobenius" and
+                           (variant == "int8" or all(c % 32 == 0 for _, c in self.shapes)))
         self.mom: List[torch.Tensor] = []
         self.x: List[torch.Tensor] = []
         self.signs: List[torch.Tensor] = []
         for (r, c) in self.shapes:
             for _ in range(M):
                 self.mom.append(torch.zeros((r, c), dtype=torch.float32, device=dev))
-                self.x.append(torch.empty((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device=dev))
+                if not self.fused_sign:
+                    self.x.append(torch.empty((r, L.signmuon_x_ld(c)), dtype=torch.bfloat16, device=dev))
                 if variant == "pack1":
                     self.signs.append(torch.empty(L.signmuon_packed_words((r, c)), dtype=torch.int32,
                                                   device=dev))
@@ -102,7 +109,9 @@ class SignMuonStep:
         self._ns_plan_key = self._polar_plan_key = None
         full = L.signmuon_newton_schulz_workspace_bytes(self.shapes, M)
         minimal = L.signmuon_newton_schulz_workspace_bytes(self.shapes, M, minimal=True)
-        self.ws_ns = torch.empty(max(minimal, min(full, ns_workspace_cap)), dtype=torch.uint8, device=dev)
+        # (No Newton-Schulz workspace when k = 0 runs fused.)
+        self.ws_ns = torch.empty(0 if self.fused_sign else max(minimal, min(full, ns_workspace_cap)),
+                                 dtype=torch.uint8, device=dev)
         self.ws_vote = torch.empty(L.signmuon_vote_workspace_bytes(self.shapes, M), dtype=torch.uint8,
                                    device=dev)
         if self.norm == "spectral":
@@ -134,6 +143,12 @@ class SignMuonStep:
         for u, g in enumerate(grads):
             r, c = self.shapes[u // self.n_workers]
             gptr.append(_check_buf(g, (r, c), gdt, f"grad[{u}]"))
+        if self.fused_sign:
+            L.signmuon_momentum_sign(self.shapes, self.n_workers, _dtype_code(gdt), gptr,
+                                     [m.data_ptr() for m in self.mom], self.beta, self.variant == "int8",
+                                     [x.data_ptr() for x in self.signs], self.inv_norm.data_ptr(),
+                                     self.ws_mom.data_ptr(), self.ws_mom.numel(), stream)
+            return
         L.signmuon_momentum_norm(self.shapes, self.n_workers, _dtype_code(gdt), gptr,
                                  [m.data_ptr() for m in self.mom], self.beta,
                                  [x.data_ptr() for x in self.x], self.inv_norm.data_ptr(),
@@ -144,11 +159,17 @@ class SignMuonStep:
                                      self.ws_spec.numel(), stream)
 
     def newton_schulz(self, stream: int, out_mode: Optional[int] = None, outs=None) -> None:
+        if self.fused_sign:
+            if out_mode is not None or outs is not None:
+                raise RuntimeError("k = 0 runs fused into the momentum call: there is no separate output")
+            return                      # the signs were written by momentum_norm
         self._ns_plan_for(stream, out_mode, outs)
         a, b, c = self.coeffs
         L.signmuon_newton_schulz_run(self._ns_plan, self.k, a, b, c, 0.0, stream)
 
     def _ns_plan_for(self, stream: int, out_mode: Optional[int], outs) -> None:
+        if self.fused_sign:
+            return
         # The unit table (tensor maps, buffer addresses) is built once per set
         # of output buffers; every later call only launches the iterations.
         if out_mode is None:
@@ -238,8 +259,8 @@ class SignMuonStep:
         mom = uploads(self.units * 56) + 2
         if self.norm == "spectral":
             mom += uploads(self.units * 48) + 1 + 2 * self.spectral_iters
-        ns_waves = self._waves(self.shapes, M, self.ws_ns.numel())
-        ns = (3 * self.k if self.k > 0 else 1) * ns_waves
+        ns_waves = 0 if self.fused_sign else self._waves(self.shapes, M, self.ws_ns.numel())
+        ns = 0 if self.fused_sign else (3 * self.k if self.k > 0 else 1) * ns_waves
         vote = uploads(-(-n_mats * 64 // 256) * 256 + self.units * 8) + 1
         total = mom + ns + vote
         if self.polar:

@@ -88,6 +88,12 @@ def test_argument_validation_returns_status(lib):
     assert _err(L.signmuon_momentum_norm, [(0, 8)], 1, 0, [fake], [fake], 0.9, [fake], fake, fake, 1 << 20) == 1
     assert _err(L.signmuon_momentum_norm, shp, 128, 0, [fake] * 128, [fake] * 128, 0.9, [fake] * 128, fake,
                 fake, 1 << 30) == 1
+    # Fused momentum + sign (k = 0): packed output needs cols % 32 == 0.
+    ms_ = L.signmuon_momentum_sign
+    assert _err(ms_, [(4, 40)], 1, 0, [fake], [fake], 0.9, False, [fake], fake, fake, 1 << 20) == 3
+    assert _err(ms_, [(4, 64)], 1, 0, [fake], [fake], 0.9, False, [odd], fake, fake, 1 << 20) == 2
+    assert _err(ms_, [(4, 40)], 1, 0, [fake], [fake], 0.9, True, [0], fake, fake, 1 << 20) == 1
+    assert _err(ms_, [(4, 40)], 1, 0, [fake], [fake], 0.9, True, [fake], fake, fake, 16) == 4
     # Newton-Schulz.
     a, b, c = 3.4445, -4.7750, 2.0315
     ns = L.signmuon_newton_schulz_batched

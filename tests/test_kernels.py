@@ -230,6 +230,45 @@ def test_momentum_norm_exact(shapes, M, grad_dtype):
         assert math.isclose(inv[u].item(), ref_inv, rel_tol=1e-5)
 
 
+@pytest.mark.parametrize("int8_out", [False, True])
+@pytest.mark.parametrize("grad_dtype", [torch.float32, torch.bfloat16])
+def test_momentum_sign_fused_matches_oracle(int8_out, grad_dtype):
+    """k = 0 fused: momentum bit-exact and the signs of X0 = M / (||M|| + eps)
+    exactly as the oracle's (a NaN unit gives all +1, a zero unit all +1)."""
+    shapes = [(64, 96), (96, 64), (32, 2048)] + ([(33, 147), (5, 40)] if int8_out else [])
+    M = 3
+    grads, moms = seeded_state(shapes, M, 29, grad_dtype=grad_dtype)
+    grads[1][3, 5] = float("nan")                       # unit 1: NaN norm
+    grads[2].zero_()
+    moms[2].zero_()                                     # unit 2: zero momentum
+    moms[4][0, :] = -0.0                                # signed zeros stay +1
+    gd = [g.cuda() for g in grads]
+    md = [m.cuda() for m in moms]
+    if int8_out:
+        signs = [torch.zeros(shapes[u // M], dtype=torch.int8, device="cuda") for u in range(len(gd))]
+    else:
+        signs = [torch.zeros(L.signmuon_packed_words(shapes[u // M]), dtype=torch.int32, device="cuda")
+                 for u in range(len(gd))]
+    inv = torch.empty(len(gd), dtype=torch.float32, device="cuda")
+    w = ws(L.signmuon_momentum_workspace_bytes(shapes, M))
+    code = L.SIGNMUON_BF16 if grad_dtype == torch.bfloat16 else L.SIGNMUON_F32
+    L.signmuon_momentum_sign(shapes, M, code, [g.data_ptr() for g in gd], [m.data_ptr() for m in md], 0.9,
+                             int8_out, [x.data_ptr() for x in signs], inv.data_ptr(), w.data_ptr(), w.numel(),
+                             stream())
+    torch.cuda.synchronize()
+    for u in range(len(gd)):
+        r, c = shapes[u // M]
+        m_ref = O.momentum_update(f64(moms[u]), f64(grads[u]), float(np.float32(0.9)))
+        assert np.array_equal(f64(md[u]), m_ref, equal_nan=True)
+        ref = O.sign_entries(O.frobenius_normalize(m_ref))
+        if int8_out:
+            got = signs[u].cpu().numpy()
+        else:
+            got = unpack_words(signs[u].cpu().numpy().view(np.uint32), r, c)
+        assert np.array_equal(got, ref), (u, shapes[u // M])
+    assert (unpack_words(signs[1].cpu().numpy().view(np.uint32), *shapes[0]) == 1).all() if not int8_out else True
+
+
 def test_momentum_zero_gradient_gives_zero_x():
     shapes, M = [(32, 64)], 2
     g = [torch.zeros(32, 64, device="cuda") for _ in range(M)]
