@@ -62,7 +62,7 @@ typedef enum signmuon_status {
   SIGNMUON_OK = 0,
   SIGNMUON_ERR_INVALID_ARG = 1,  /* null pointer, size <= 0, count out of range */
   SIGNMUON_ERR_ALIGNMENT = 2,    /* a buffer is not 16-byte aligned             */
-  SIGNMUON_ERR_UNSUPPORTED = 3,  /* valid request this build cannot run        */
+  SIGNMUON_ERR_UNSUPPORTED = 3,  /* valid request this library cannot run      */
   SIGNMUON_ERR_WORKSPACE = 4,    /* workspace null or smaller than required     */
   SIGNMUON_ERR_CUDA = 5          /* a CUDA call or kernel launch failed        */
 } signmuon_status;
