@@ -323,8 +323,12 @@ def run_gpu(args, wl):
     else:
         opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
                            polar=wl.polar, device=dev, norm=args.norm)
-    weights = [w.to(dev) for w in syn.initial_weights(wl, rank)]
-    signal = [g.to(dev) for g in syn.gradient_signal(wl, rank)]
+    # Replicas draw their own problem; with --exchange all ranks share W and
+    # the gradient signal G* (one model, data-parallel), and their workers
+    # differ through the per-rank noise drawn below.
+    problem_seed = 0 if args.exchange else rank
+    weights = [w.to(dev) for w in syn.initial_weights(wl, problem_seed)]
+    signal = [g.to(dev) for g in syn.gradient_signal(wl, problem_seed)]
     n_sets = 2
     grad_sets = []
     for t in range(n_sets):
