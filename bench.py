@@ -27,9 +27,32 @@ import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
-# stdout carries exactly one JSON line: NCCL's own messages (its version banner
-# at communicator setup among them) go to stderr unless the caller chose a file.
+# stdout carries exactly one JSON line (see emit()): NCCL's own messages go to
+# stderr unless the caller chose a file.
 os.environ.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
+_RESULT_FD = None
+
+
+def _claim_stdout():
+    """Keeps the real stdout for the result line and points file descriptor 1
+    at stderr, so that whatever else writes to it (library banners printed
+    from C, e.g. NCCL's version line at communicator setup) cannot add lines
+    to stdout."""
+    global _RESULT_FD
+    if _RESULT_FD is None:
+        sys.stdout.flush()
+        _RESULT_FD = os.dup(1)
+        os.dup2(2, 1)
+
+
+def emit(obj):
+    """Writes the one JSON result line to the real stdout."""
+    data = (json.dumps(obj) + "\n").encode()
+    if _RESULT_FD is None:
+        sys.stdout.write(data.decode())
+        sys.stdout.flush()
+    else:
+        os.write(_RESULT_FD, data)
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
@@ -261,7 +284,7 @@ def run_reference(args, wl):
             "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
                              "cores": blas_threads() or host_cores(), "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
+    emit(line)
     return 0
 
 
@@ -508,7 +531,7 @@ def run_gpu(args, wl):
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
-        print(json.dumps(result), flush=True)
+        emit(result)
     return 0
 
 
@@ -596,11 +619,12 @@ def run_vote_sweep(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     if rank == 0:
-        print(json.dumps(res), flush=True)
+        emit(res)
     return 0
 
 
 def main():
+    _claim_stdout()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
