@@ -158,8 +158,11 @@ def _packed_device(s_list, shape):
     return outs
 
 
+# M = 126 and 127: the largest worker counts (even: ties; the byte sums and
+# the seven counter planes at their range).
 VOTE_CASES = [((4, 32), 1), ((64, 64), 2), ((37, 96), 3), ((256, 256), 8), ((100, 1024), 16),
-              ((64, 4096), 64), ((33, 147), 5), ((31, 33), 4), ((2, 1000), 7), ((512, 1024), 64)]
+              ((64, 4096), 64), ((33, 147), 5), ((31, 33), 4), ((2, 1000), 7), ((512, 1024), 64),
+              ((16, 512), 126), ((9, 160), 127)]
 
 
 @pytest.mark.parametrize("shape,M", VOTE_CASES)
