@@ -155,6 +155,26 @@ def _brute_pack(s):
     return out
 
 
+def test_k0_signs_are_the_momentum_signs_unless_the_norm_is_not_finite():
+    """With k = 0 the Newton-Schulz output is X0 = M / (||M||_F + 1e-7): its
+    sign equals sign(M) entry by entry (0 and -0 -> +1) whenever the norm is
+    finite, and is +1 everywhere when M holds a NaN or an infinity (X0 is
+    then NaN, or +-0 beside a NaN).  Checked on values spanning fp32's range,
+    subnormals included, so that no entry of X0 underflows in fp64."""
+    rng = np.random.default_rng(3)
+    m = rng.standard_normal((40, 64)) * np.float64(10.0) ** rng.integers(-44, 30, (40, 64))
+    m = m.astype(np.float32).astype(np.float64)
+    m[0, :5] = [0.0, -0.0, 1e-45, -1e-45, -3e38]
+    x0 = O.newton_schulz(O.frobenius_normalize(m), 0)
+    assert np.array_equal(O.sign_entries(x0), O.sign_entries(m))
+    for bad in (np.nan, np.inf, -np.inf):
+        mb = m.copy()
+        mb[7, 9] = bad
+        with np.errstate(invalid="ignore", over="ignore"):
+            s = O.sign_entries(O.newton_schulz(O.frobenius_normalize(mb), 0))
+        assert (s == 1).all(), bad
+
+
 @pytest.mark.parametrize("shape", [(1, 1), (3, 31), (2, 32), (4, 33), (5, 147), (2, 96)])
 def test_pack_against_brute_force_and_roundtrip(shape):
     s = np.where(_rng(sum(shape)).random(shape) < 0.5, -1, 1).astype(np.int8)
