@@ -137,7 +137,7 @@ class SignMuonDistStep:
     def __init__(self, shapes: Sequence[Tuple[int, int]], local_workers: int, k: int, variant: str,
                  beta: float, eta: float, w_dtype: torch.dtype, polar: bool = False,
                  coeffs=NS_QUINTIC, device: Optional[torch.device] = None, group=None,
-                 world_size: Optional[int] = None, rank: Optional[int] = None, n_groups: int = 4,
+                 world_size: Optional[int] = None, rank: Optional[int] = None, n_groups: Optional[int] = None,
                  ns_workspace_cap: int = 16 << 30):
         if world_size is None or rank is None:
             import torch.distributed as dist
@@ -154,6 +154,10 @@ class SignMuonDistStep:
         self.beta, self.eta, self.w_dtype = float(beta), float(eta), w_dtype
         self.polar, self.coeffs = bool(polar), tuple(float(x) for x in coeffs)
         self.device = dev = torch.device(device or "cuda")
+        # Several groups let the exchange of one overlap the Newton-Schulz
+        # iterations of the next; a single rank has nothing to overlap.
+        if n_groups is None:
+            n_groups = 1 if self.world_size == 1 else 4
         self.layout = lay = exchange_layout(self.shapes, Ml, n_groups, variant)
         n_mats = len(self.shapes)
         self.units = n_mats * Ml
