@@ -400,35 +400,6 @@ __device__ __forceinline__ void operand_maps(const NsLaunch& L, const NsUnit* u,
 }
 
 // ---------------------------------------------------------------------------
-// Epilogue helpers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void unpack_bf16x8(const uint4& raw, float* v) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 f = __bfloat1622float2(h[j]);
-    v[2 * j] = f.x;
-    v[2 * j + 1] = f.y;
-  }
-}
-
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, bool vec, int nvalid, const float (&v)[32]) {
-  if (vec) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      __nv_bfloat162 h[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) h[j] = __floats2bfloat162_rn(v[q * 8 + 2 * j], v[q * 8 + 2 * j + 1]);
-      *reinterpret_cast<uint4*>(p + q * 8) = *reinterpret_cast<const uint4*>(h);
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < nvalid) p[j] = __float2bfloat16_rn(v[j]);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
 template <bool kPair>
