@@ -12,6 +12,9 @@
 // with, in the last iteration, the entrywise sign fused into the epilogue and
 // written as packed bits or int8 (steps 2-3 of the summary's flow), or the
 // update W <- W - eta U (the optional local polar step, step 5).
+// Of the symmetric A, P and B' only the 256x256 blocks on and above the
+// diagonal are computed and stored; the stages that consume them read a
+// k-block below the diagonal as the transpose of the stored block.
 //
 // Two tile modes (chosen per launch by the host from the padding cost):
 //   single: one CTA per SM computes a 128x256 tile with
@@ -146,11 +149,8 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sm
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until this thread's bulk stores have read their shared-memory sources.
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Same, but the most recent group may still be reading.
+// Wait until all but the most recent of this thread's bulk store groups
+// have read their shared-memory sources.
 __device__ __forceinline__ void bulk_wait_read_all_but_one() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
@@ -338,7 +338,21 @@ struct Tile {
   int M, N, K;
   int m0, n0;
   int a_mn, b_mn, sym;
+  int a_up, b_up;  // operand is a symmetric matrix of which only the upper 256-blocks are stored
 };
+
+// Symmetric products (A, P, B') are stored as their 256x256 blocks (I, J)
+// with J >= I only.  An operand that is one of them reads k-block
+// [k0, k0 + 64) of its rows [r0, r0 + 128) -- all in 256-block r0 / 256 --
+// directly when k0 / 256 >= r0 / 256, and otherwise as the transpose of the
+// stored block (k0 / 256, r0 / 256): an MN-major box at (x = r0, y = k0).
+// Both CTAs of a pair share the decision (their rows lie in one 256-block).
+__device__ __forceinline__ int a_major(const Tile& T, int k0) {
+  return T.a_mn | (T.a_up & (int)((k0 >> 8) < (T.m0 >> 8)));
+}
+__device__ __forceinline__ int b_major(const Tile& T, int k0) {
+  return T.b_mn | (T.b_up & (int)((k0 >> 8) < (T.n0 >> 8)));
+}
 
 // Problem dimensions, operand majors and tile origin of local tile li of a
 // unit with the given shape.
@@ -346,20 +360,21 @@ __device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, i
   const bool tall = rows > cols;
   const int s = tall ? cols : rows, l = tall ? rows : cols;
   Tile T;
+  T.a_up = 0; T.b_up = 0;
   if (stage == kStageGram) {
     T.M = s; T.N = s; T.K = l; T.sym = 1; T.a_mn = tall; T.b_mn = tall;
-  } else if (stage == kStageSquare) {
-    T.M = s; T.N = s; T.K = s; T.sym = 1; T.a_mn = 0; T.b_mn = 0;
-  } else if (!tall) {  // X' = B' X: A-op = B' (K-major), B-op = X (MN-major)
-    T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 1;
+  } else if (stage == kStageSquare) {  // A P: both operands symmetric
+    T.M = s; T.N = s; T.K = s; T.sym = 1; T.a_mn = 0; T.b_mn = 0; T.a_up = 1; T.b_up = 1;
+  } else if (!tall) {  // X' = B' X: A-op = B' (symmetric, K-major), B-op = X (MN-major)
+    T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 1; T.a_up = 1;
   } else {             // X' = X B': A-op = X (K-major), B-op = B' (symmetric, K-major)
-    T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 0;
+    T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 0; T.b_up = 1;
   }
   const int tiles_n = (T.N + kBN - 1) / kBN;
   int tm = 0, tn = 0;
   if (T.sym) {
-    // Tiles entirely below the diagonal are skipped: row tile tm starts at
-    // column tile tm * tile_m / 256.
+    // Only the upper 256-blocks of a symmetric output are computed (and
+    // stored): row tile tm starts at column tile tm * tile_m / 256.
     const int sh = tile_m == 256 ? 0 : 1;
     while (true) {
       const int cnt = tiles_n - (tm >> sh);
@@ -490,22 +505,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
           const uint32_t sb = sa + C::kStageA;
           const int k0 = kb * kBK;
+          const int amn = a_major(T, k0), bmn = b_major(T, k0);
 #pragma unroll
           for (int j = 0; j < C::kRowsA / kBoxRows; ++j) {
             const int mn = a_row0 + j * kBoxRows;
             if constexpr (kPair)
-              tma_load_2d_pair(sa + j * kBoxBytes, ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
+              tma_load_2d_pair(sa + j * kBoxBytes, ma, fb, amn ? mn : k0, amn ? k0 : mn);
             else
-              tma_load_2d(sa + j * kBoxBytes, ma, fb, T.a_mn ? mn : k0, T.a_mn ? k0 : mn);
+              tma_load_2d(sa + j * kBoxBytes, ma, fb, amn ? mn : k0, amn ? k0 : mn);
           }
 #pragma unroll
           for (int j = 0; j < C::kRowsB / kBoxRows; ++j) {
             if (b_from_a) break;
             const int mn = b_row0 + j * kBoxRows;
             if constexpr (kPair)
-              tma_load_2d_pair(sb + j * kBoxBytes, mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
+              tma_load_2d_pair(sb + j * kBoxBytes, mb, fb, bmn ? mn : k0, bmn ? k0 : mn);
             else
-              tma_load_2d(sb + j * kBoxBytes, mb, fb, T.b_mn ? mn : k0, T.b_mn ? k0 : mn);
+              tma_load_2d(sb + j * kBoxBytes, mb, fb, bmn ? mn : k0, bmn ? k0 : mn);
           }
           ++issued_kb;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -526,7 +542,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         const NsTileRec rec = rs.advance(L, t, tile_stride);
         const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
         // The square stage multiplies the fp16 A and P; all others are bf16.
-        const uint32_t idesc = instr_desc(T.a_mn, T.b_mn, C::kTileM, L.stage == kStageSquare);
+        const bool fp16_ops = L.stage == kStageSquare;
         const bool b_from_a = diag_b_from_a<kPair>(L, T);
         const int nkb = (T.K + kBK - 1) / kBK;
         if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag)) {
@@ -546,11 +562,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           tc_fence_after();
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
           const uint32_t sb = b_from_a ? sa : sa + C::kStageA;
+          const int amn = a_major(T, kb * kBK), bmn = b_major(T, kb * kBK);
+          const uint32_t idesc = instr_desc(amn, bmn, C::kTileM, fp16_ops);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-            const uint32_t aoff = T.a_mn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
-            const uint32_t boff = T.b_mn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
-            tc_mma<kPair>(tmem_d, smem_desc(sa + aoff, T.a_mn), smem_desc(sb + boff, T.b_mn), idesc,
+            const uint32_t aoff = amn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
+            const uint32_t boff = bmn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
+            tc_mma<kPair>(tmem_d, smem_desc(sa + aoff, amn), smem_desc(sb + boff, bmn), idesc,
                           (kb | kk) != 0);
           }
           // The stage is free (in both CTAs of a pair) once these MMAs finish.
@@ -661,62 +679,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           for (int j = 0; j < 32; ++j) v[j] = s * __uint_as_float(raw[j]);
         }
         if (bf16_out) {
-          // Blocks to write (warp-uniform): a symmetric output stores the
-          // blocks above the diagonal together with their transposes, and
-          // each diagonal block once (made symmetric); the iterate stores
-          // every block.  The Gram stage writes two outputs: A, then
-          // P = b I + c A (from the fp32 value of A).
-          const bool diag = T.sym && gc0 == grow0;
-          const bool mirror = T.sym && gc0 > grow0;
+          // Each 32x32 block is staged in shared memory and written by a TMA
+          // store.  The tiles of a symmetric output cover its upper
+          // 256-blocks only, which is all that is stored of it (its
+          // consumers read the other blocks transposed).  The Gram stage
+          // writes two outputs: A, then P = b I + c A (from the fp32 value
+          // of A).
           const int n_out = (L.stage == kStageGram) ? 2 : 1;
-          for (int o = 0; o < n_out && (!T.sym || diag || mirror); ++o) {
+          // The Gram stage's A and P are fp16, everything else bf16.
+          const bool half_out = L.stage == kStageGram;
+          for (int o = 0; o < n_out; ++o) {
             if (o == 1) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = fmaf(L.c, v[j], (gc0 + j == grow) ? L.b : 0.f);
             }
             const CUtensorMap* map = o == 0 ? uf.st_out : uf.st_p;
-            // The iterate alternates its two staging blocks, so only the
-            // store before last must have finished reading; symmetric
-            // outputs use both blocks per output.
+            // Stores alternate between the two staging blocks, so only the
+            // store before last must have finished reading.
             uint8_t* dst = stg0;
             uint32_t dst_s = stg0_s;
-            if (!T.sym && (stage_flip ^= 1)) { dst = stg1; dst_s = stg1_s; }
+            if (stage_flip ^= 1) { dst = stg1; dst_s = stg1_s; }
             if (stores_pending) {
-              if (lane == 0) {
-                if (T.sym) bulk_wait_read_all(); else bulk_wait_read_all_but_one();
-              }
+              if (lane == 0) bulk_wait_read_all_but_one();
               __syncwarp();
             }
-            // The Gram stage's A and P are fp16, everything else bf16.
-            const bool half_out = L.stage == kStageGram;
-            if (!diag) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                uint32_t w[4];
+            for (int k = 0; k < 4; ++k) {
+              uint32_t w[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
-                *reinterpret_cast<uint4*>(dst + stage_off(lane, 8 * k)) = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-              if (mirror) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  *reinterpret_cast<uint16_t*>(stg1 + stage_off(j, lane)) = to16(v[j], half_out);
-              }
-            } else {
-              // Diagonal block: row `lane` supplies (lane, j >= lane) and, by
-              // symmetry, (j > lane, lane); together the whole block.
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const uint16_t h = to16(v[j], half_out);
-                if (j >= lane) *reinterpret_cast<uint16_t*>(stg0 + stage_off(lane, j)) = h;
-                if (j > lane) *reinterpret_cast<uint16_t*>(stg0 + stage_off(j, lane)) = h;
-              }
+              for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
+              *reinterpret_cast<uint4*>(dst + stage_off(lane, 8 * k)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
             fence_smem_to_async();
             __syncwarp();
             if (lane == 0) {
               tma_store_2d(map, dst_s, gc0, grow0);
-              if (mirror) tma_store_2d(map, stg1_s, grow0, gc0);
               bulk_commit();
             }
             stores_pending = true;
