@@ -197,7 +197,9 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
  * on the tensor cores (bf16 operands, fp32 accumulation, bf16 between
  * iterations).  The kernels store A and P = b I + c A in fp16, form
  * B' = a I + A P (= a I + b A + c A^2, bf16) and compute X <- B' X (X B'):
- * the same map with the a X term folded into the product.
+ * the same map with the a X term folded into the product.  Of the
+ * symmetric A, P and B' only the 256x256 blocks on and above the diagonal
+ * are computed and stored in the workspace.
  * The last iteration's epilogue writes, per out_mode:
  *   PACK1:    out[u] = packed sign(U)   (uint32, signmuon_packed_words words)
  *   INT8:     out[u] = int8 sign(U)     ([rows, cols])
@@ -207,8 +209,8 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
  * k = 0 writes the same outputs from U = X0.
  *
  * x_bf16 buffers are CLOBBERED (used as one of the two iterate buffers).
- * Coefficients a, b, c are the caller's (the build uses 3.4445, -4.7750,
- * 2.0315).  k must be in [0, 64].
+ * Coefficients a, b, c are the caller's (the Python step class passes
+ * 3.4445, -4.7750, 2.0315).  k must be in [0, 64].
  * workspace: device; signmuon_newton_schulz_workspace_bytes(..., 0) bytes
  * run all units at once, any size >= the value for minimal=1 runs them in
  * successive waves.
