@@ -317,7 +317,10 @@ signmuon_status signmuon_vote_update(const signmuon_shape* shapes, int n_mats, i
  * The array (1 MiB) is held on every GPU that loads the library until the
  * process exits.  The first call on each device looks up the array's device
  * address (once per device, with that device current); make that first call
- * before any stream capture.  All calls share the array and each call
+ * before any stream capture.  The address is cached for the life of the
+ * process and belongs to the device's primary context: after
+ * cudaDeviceReset it is stale, so do not call this entry point again in
+ * that process.  All calls share the array and each call
  * rewrites what it reads, so nothing needs clearing, but calls whose kernels
  * can overlap on the GPU (different streams with no ordering) race on it.
  * ---------------------------------------------------------------------- */

@@ -18,7 +18,6 @@ constexpr int kAbiVersion = 1;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inline int32_t x_ld_of(int32_t cols) { return (cols + 7) / 8 * 8; }
 inline int64_t wpr_of(int32_t cols) { return (cols + 31) / 32; }
 inline int64_t packed_words_of(signmuon_shape s) { return ((int64_t)s.rows * wpr_of(s.cols) + 3) / 4 * 4; }
 
@@ -49,12 +48,6 @@ signmuon_status check_workspace(void* ws, size_t have, size_t need) {
 }
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
-
-inline signmuon_status cuda_status(cudaError_t e) {
-  if (e == cudaSuccess) return SIGNMUON_OK;
-  g_last_cuda_error = e;
-  return SIGNMUON_ERR_CUDA;
-}
 
 // ----------------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -149,6 +142,12 @@ size_t ns_rec_bytes(const signmuon_shape* shapes, int n_mats, int n_workers) {
 }
 
 }  // namespace
+
+signmuon_status signmuon::cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SIGNMUON_OK;
+  g_last_cuda_error = e;
+  return SIGNMUON_ERR_CUDA;
+}
 
 extern "C" {
 

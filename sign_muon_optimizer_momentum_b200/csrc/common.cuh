@@ -46,6 +46,14 @@ constexpr int kBarrierBytes = 256;
 constexpr int kStageBlockBytes = 32 * 32 * 2;
 constexpr int kStagingBytes = (kEpilogueThreads / 32) * 2 * kStageBlockBytes;  // 32 KB
 
+// Row stride, in elements, of a bf16 Newton-Schulz buffer: cols rounded up
+// to 8 (16 bytes, the TMA stride granule).  The public signmuon_x_ld.
+inline int32_t x_ld_of(int32_t cols) { return (cols + 7) / 8 * 8; }
+
+// Maps a CUDA error to a status; a failure is also recorded as the calling
+// thread's last error (read back by signmuon_last_error_string).
+signmuon_status cuda_status(cudaError_t e);
+
 // Output rows per tile: 128 for one CTA, 256 for a CTA pair.
 inline int ns_tile_m(int pair) { return pair ? 256 : 128; }
 

@@ -17,6 +17,12 @@
 // rewrites the parts it reads, so nothing needs to start at zero.  All calls
 // share the array: two calls whose kernels overlap on the GPU (different
 // streams without ordering between them) race on it and must not be issued.
+//
+// The device address of the array is looked up once per device and cached
+// for the life of the process.  It belongs to the device's primary context:
+// after cudaDeviceReset (which destroys that context and the module's
+// copy of the array) the cached address is stale, and this entry point must
+// not be called again in that process.
 #include <mutex>
 #include <vector>
 
@@ -83,7 +89,8 @@ extern "C" signmuon_status signmuon_momentum_norm_noalloc(const signmuon_shape* 
   if (!aligned16(inv_norm)) return SIGNMUON_ERR_ALIGNMENT;
 
   void* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return SIGNMUON_ERR_CUDA;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   std::vector<MomUnit> mu((size_t)units);
@@ -98,7 +105,7 @@ extern "C" signmuon_status signmuon_momentum_norm_noalloc(const signmuon_shape* 
       u.rows = shapes[i].rows;
       u.cols = shapes[i].cols;
       u.n = (int64_t)u.rows * u.cols;
-      u.ld_x = (u.cols + 7) / 8 * 8;
+      u.ld_x = x_ld_of(u.cols);
       u.block_begin = b;
       u.block_count = cnt;
       u.pad_ = 0;
@@ -107,8 +114,8 @@ extern "C" signmuon_status signmuon_momentum_norm_noalloc(const signmuon_shape* 
   }
   MomUnit* d_units = static_cast<MomUnit*>(scratch);
   float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocTableBytes);
-  cudaError_t e = upload_bytes(d_units, mu.data(), mu.size() * sizeof(MomUnit), s);
+  e = upload_bytes(d_units, mu.data(), mu.size() * sizeof(MomUnit), s);
   if (e == cudaSuccess) e = launch_momentum(d_units, (int)units, b, grad_dtype == SIGNMUON_BF16, beta, partials, 0, s);
   if (e == cudaSuccess) e = launch_momentum_finalize(d_units, (int)units, partials, inv_norm, 0, s);
-  return e == cudaSuccess ? SIGNMUON_OK : SIGNMUON_ERR_CUDA;
+  return cuda_status(e);
 }

@@ -99,6 +99,23 @@ def test_normalisation_bounds_spectral_norm_by_one():
     assert np.all(O.frobenius_normalize(np.zeros((3, 4))) == 0)
 
 
+def test_ns_coefficients_are_the_stated_quintic():
+    """The pages print no Newton-Schulz polynomial; the specification fixes
+    the quintic (a, b, c) = (3.4445, -4.7750, 2.0315).  The oracle and the
+    step class each carry that literal (they share no code), so both are
+    pinned to it here: a typo in either would otherwise reach both sides of
+    every GPU parity test that takes its coefficients from one of them."""
+    from sign_muon_optimizer_momentum_b200 import step as S
+    assert O.NS_QUINTIC == (3.4445, -4.7750, 2.0315)
+    assert S.NS_QUINTIC == (3.4445, -4.7750, 2.0315)
+    # The scalar map of these coefficients: phi(1) = a + b + c = 0.701 and a
+    # maximum of 1.2024 on [0, 1] (the orbit band used below).
+    s = np.linspace(0.0, 1.0, 200001)
+    phi = 3.4445 * s - 4.7750 * s ** 3 + 2.0315 * s ** 5
+    assert abs(phi[-1] - 0.701) < 1e-12
+    assert abs(phi.max() - 1.2024) < 1e-4
+
+
 def test_quintic_iterates_land_in_band():
     """Singular values in [1e-3, 1] are driven into [0.6818, 1.2024] after six
     quintic steps (the band of the scalar map's orbit), not onto 1."""

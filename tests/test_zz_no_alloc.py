@@ -69,7 +69,7 @@ def test_noalloc_refuses_requests_beyond_its_scratch(cuda_lib):
         L.signmuon_momentum_norm_noalloc(too_many_units, 1, 0, [fake] * 1171, [fake] * 1171, 0.9,
                                          [fake] * 1171, fake)
     assert e.value.status == L.SIGNMUON_ERR_WORKSPACE
-    too_many_elems = [(65536, 16385)]     # 245761 blocks of 4096 elements
+    too_many_elems = [(65536, 16385)]     # 262160 blocks of 4096 elements; the limit is 245760
     with pytest.raises(L.SignMuonError) as e:
         L.signmuon_momentum_norm_noalloc(too_many_elems, 1, 0, [fake], [fake], 0.9, [fake], fake)
     assert e.value.status == L.SIGNMUON_ERR_WORKSPACE
