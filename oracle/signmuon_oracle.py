@@ -264,17 +264,36 @@ def majority_vote_packed(words_list, cols):
 # Parameter update (SignMuon summary, §2 "Algorithmic flow", step 4)
 # ---------------------------------------------------------------------------
 def apply_update(w, eta, direction, w_dtype):
-    """W_{t+1} = W_t - eta * D, computed in fp64 and rounded once to W's dtype.
+    """W_{t+1} = W_t - eta * D, rounded once (to nearest, ties to even) from
+    the exact difference to W's dtype.
 
     ``w`` holds the stored weights (fp32 or bf16 values, as fp64 or fp32);
-    ``eta`` is the fp32 learning rate the device receives.  With D the voted
-    signs in {-1,0,+1} and |W|, eta within a few binades of each other the
-    fp64 difference is exact, so the result is the correctly rounded value.
+    ``eta`` is the fp32 learning rate the device receives.  The summary gives
+    the update but not its rounding; the reading here is "exact, then one
+    rounding".  The product p = eta * D is exact in fp64 whenever D has at
+    most 29 significant bits (the voted signs in {-1, 0, +1}, or the fp32
+    values of a polar direction computed on the device).  The difference
+    w - p is then split exactly into hi + lo (hi = the fp64 difference, lo
+    its rounding error, by the two-sum rule).  Rounding hi gives the correctly
+    rounded result unless hi lies exactly on a rounding midpoint of the
+    target grid while lo is non-zero: then the exact value lies on lo's side
+    of that midpoint (no double and so no midpoint lies strictly between hi
+    and the exact value), and the neighbour on that side is taken.
     """
     w = np.asarray(w, dtype=np.float64)
     d = np.asarray(direction, dtype=np.float64)
     eta = float(np.float32(eta))
-    return round_to_dtype(w - eta * d, w_dtype)
+    p = eta * d
+    hi = w - p
+    z = hi - w
+    lo = (w - (hi - z)) + (-p - z)                    # hi + lo == w - p exactly
+    r = round_to_dtype(hi, w_dtype)
+    up = round_to_dtype(np.nextafter(hi, np.inf), w_dtype)
+    down = round_to_dtype(np.nextafter(hi, -np.inf), w_dtype)
+    midpoint = (up != down) & (r != hi)               # hi halfway between two grid values
+    r = np.where(midpoint & (lo > 0), up, r)
+    r = np.where(midpoint & (lo < 0), down, r)
+    return r
 
 
 # ---------------------------------------------------------------------------

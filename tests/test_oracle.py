@@ -334,6 +334,58 @@ def test_update_moves_each_weight_by_eta_or_not_at_all(w_dtype):
     assert np.array_equal(w_new, O.round_to_dtype(w_new, w_dtype))
 
 
+def _exact_round_brute(x, w_dtype):
+    """Correct rounding of the exact rational x to fp32 or bf16 by brute
+    force: the nearest of the representable values around it, compared with
+    exact rational distances; a tie goes to the even significand."""
+    from fractions import Fraction
+    f = np.float32(float(x))
+    bits = int(np.array([f], np.float32).view(np.uint32)[0])
+    step, cands = (1, []) if w_dtype == "f32" else (0x10000, [])
+    base = bits if w_dtype == "f32" else bits & 0xFFFF0000
+    for k in range(-3, 4):
+        b = (base + k * step) & 0xFFFFFFFF
+        c = float(np.array([b], np.uint32).view(np.float32)[0])
+        if np.isfinite(c):
+            cands.append((abs(Fraction(c) - x), (b // step) % 2, c))
+    best = min(d for d, _, _ in cands)
+    winners = sorted({(odd, c) for d, odd, c in cands if d == best})
+    return winners[0][1]
+
+
+def test_update_rounds_the_exact_difference_once():
+    """W - eta * D is rounded once from its exact value.  Two constructed
+    cases put the fp64 difference exactly on a rounding midpoint of the
+    target while the exact value lies 2^-54 (bf16) or 2^-70 (fp32) above it:
+    rounding the fp64 value would tie to the even neighbour, the correct
+    result is the odd one above.  Random fp32 directions (as the device's
+    polar step produces) are checked against exact rational arithmetic."""
+    from fractions import Fraction
+    # bf16: W = 1 + 2^-7, eta = 2^-8 (1 + 2^-23), D = 1 - 2^-23:
+    # W - eta D = 1 + 2^-8 + 2^-54, just above the midpoint 1 + 2^-8.
+    w, eta, dd = 1.0 + 2.0 ** -7, 2.0 ** -8 * (1 + 2.0 ** -23), 1.0 - 2.0 ** -23
+    assert np.float32(eta) == eta and np.float32(dd) == dd
+    got = O.apply_update(np.array([w]), eta, np.array([dd]), "bf16")[0]
+    assert got == 1.0 + 2.0 ** -7 == _exact_round_brute(Fraction(w) - Fraction(eta) * Fraction(dd), "bf16")
+    # fp32: W = 1 + 2^-23, eta = 2^-24 (1 + 2^-23), D = 1 - 2^-23:
+    # W - eta D = 1 + 2^-24 + 2^-70.
+    w, eta = 1.0 + 2.0 ** -23, 2.0 ** -24 * (1 + 2.0 ** -23)
+    got = O.apply_update(np.array([w]), eta, np.array([dd]), "f32")[0]
+    assert got == 1.0 + 2.0 ** -23 == _exact_round_brute(Fraction(w) - Fraction(eta) * Fraction(dd), "f32")
+    # Mirror images (negative weights, negative direction) round away too.
+    got = O.apply_update(np.array([-(1.0 + 2.0 ** -7)]), 2.0 ** -8 * (1 + 2.0 ** -23), np.array([-dd]), "bf16")
+    assert got[0] == -(1.0 + 2.0 ** -7)
+    rng = _rng(13)
+    for w_dtype in ("f32", "bf16"):
+        w = O.round_to_dtype(0.02 * rng.standard_normal(400), w_dtype)
+        w[:40] = O.round_to_dtype(rng.standard_normal(40) * 10.0 ** rng.integers(-8, 3, 40), w_dtype)
+        d = O.round_to_f32(rng.standard_normal(400) * 10.0 ** rng.integers(-4, 1, 400))
+        eta = float(np.float32(0.02))
+        got = O.apply_update(w, eta, d, w_dtype)
+        for wi, di, gi in zip(w, d, got):
+            assert gi == _exact_round_brute(Fraction(wi) - Fraction(eta) * Fraction(di), w_dtype), (wi, di)
+
+
 # --------------------------------------------------------------------------
 # Optional local polar step
 # --------------------------------------------------------------------------
