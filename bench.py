@@ -7,7 +7,12 @@ workload: momentum + Frobenius norm, k Newton-Schulz iterations with the sign
 fused into the last one, and the majority vote fused with the update (plus
 the local polar step when the workload has it).  The metric is
 params * workers / s (whole job); inputs are resident in HBM and larger than
-L2.  With N > 1 (torchrun) every rank runs an independent replica by default:
+L2.  The default workload is the batch of 32 square 4096 x 4096 matrices
+(M = 16 workers, k = 5, 1-bit vote, local polar step); its line also carries
+three more rows measured in the same run, each with its roofline: the vote +
+update sweep point (2^30 parameters, M = 16, fp32 W), the majority-vote Signum
+step (k = 0) and the step with spectral scaling, both on the nanoGPT-small
+matrices (`--no-extras` skips them).  With N > 1 (torchrun) every rank runs an independent replica by default:
 the M workers are buffers on one GPU, so the step has no exchange; with
 --exchange every rank runs the workload's workers and the signs of all ranks
 are exchanged (NCCL) before one vote over all of them.
@@ -58,9 +63,9 @@ if ROOT not in sys.path:
 
 METRIC = "params·workers/s per Sign-Muon step"
 UNIT = "params*workers/s"
-DEFAULT_CONFIG = "nanogpt_small"
+DEFAULT_CONFIG = "square4096x32"
 # Timed steps per workload when --steps is not given (about a second of GPU time).
-DEFAULT_STEPS = {"single256": 200, "nanogpt_small": 60, "resnet50": 100, "square4096x32": 3,
+DEFAULT_STEPS = {"single256": 200, "nanogpt_small": 60, "resnet50": 100, "square4096x32": 10,
                  "signum_nanogpt_small": 100}
 
 
@@ -80,6 +85,7 @@ KERNEL_SOURCES = {
     "ns_gemm_kernel": (_CSRC + "ns_gemm.cu", _CSRC + "common.cuh"),
     "momentum_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
     "vote_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
+    "spectral_rowpass_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
 }
 
 
@@ -210,21 +216,25 @@ def oracle_sample_step(wl, units, seed=0):
 
 
 def oracle_sample(wl, budget_s):
-    """(matrix, worker) units, one matrix of each shape first and all of its
-    workers, whose oracle step fits in about budget_s."""
+    """(matrix, worker) units whose oracle step fits in about budget_s: one
+    unit of every distinct shape first (so that every shape, and both the
+    wide and the tall Newton-Schulz branch, is in the sample), then further
+    workers of those matrices, shape by shape in turn."""
     order, seen = [], set()
     for i, s in enumerate(wl.shapes):
         if s not in seen:
             seen.add(s)
             order.append(i)
     t0 = time.perf_counter()
-    chosen = []
-    for i in order:
-        for m in range(wl.n_workers):
-            chosen.append((i, m))
-            oracle_sample_step(wl, [(i, m)])
+    chosen = [(i, 0) for i in order]
+    for u in chosen:
+        oracle_sample_step(wl, [u])
+    for m in range(1, wl.n_workers):
+        for i in order:
             if time.perf_counter() - t0 > budget_s:
                 return chosen
+            chosen.append((i, m))
+            oracle_sample_step(wl, [(i, m)])
     return chosen
 
 
@@ -280,7 +290,7 @@ def run_reference(args, wl):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(wl),
+            "data": "synthetic", "config": line_config(wl, args, int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
                              "cores": blas_threads() or host_cores(), "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -294,13 +304,278 @@ def workload_config(wl):
             "beta": wl.beta, "eta": wl.eta}
 
 
+def resident_bytes(wl):
+    """Gradients (W's dtype) and fp32 momentum of every (matrix, worker) unit."""
+    return wl.params * wl.n_workers * ((2 if wl.w_dtype == "bf16" else 4) + 4)
+
+
+def line_config(wl, args, world):
+    """The `config` of the result line; both arms print the same one."""
+    cfg = dict(workload_config(wl), norm=args.norm)
+    cfg["parallelism"] = (f"dp{world}-{'allgather' if wl.variant == 'pack1' else 'allreduce'}"
+                          if args.exchange else f"replicas{world}")
+    cfg["l2"] = f"inputs larger than L2 ({resident_bytes(wl) / 2**30:.1f} GiB gradients+momentum resident)"
+    cfg["launch"] = "cuda_graph" if args.graph else "eager"
+    return cfg
+
+
 # --------------------------------------------------------------------------- GPU arm
+class Ctx:
+    """Process-group and device facts of this rank, shared by the timed runs."""
+
+    def __init__(self, world, rank, local, dev):
+        self.world, self.rank, self.local, self.dev = world, rank, local, dev
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        import torch
+        torch.cuda.synchronize()
+
+    def max_over_ranks(self, x):
+        return max_over_ranks_value(x, self.world, self.dev)
+
+
+def ns_roofline(wl, ns_ms, ms_total, pk, steps):
+    """Newton-Schulz roofline: algorithmic FLOPs of the step's NS call over
+    its mean duration, against the sustained bf16 peak when the timed region
+    lasts 0.5 s or more (the GPU then sits at its power cap, the condition of
+    the sustained figure), else the burst peak."""
+    flops = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters)
+    note = ("Newton-Schulz call of the step (the local polar step is timed with the vote)" if wl.polar
+            else "Newton-Schulz call of the step")
+    achieved = flops / (ns_ms / 1e3) / 1e12
+    dense = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters, True) / (ns_ms / 1e3) / 1e12
+    sustained = ms_total >= 500.0
+    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    return {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": captured_traffic("ns_gemm_kernel", wl.name),
+            "note": f"{note}: {flops / 1e12:.3f} TFLOP algorithmic (symmetric-aware: 3s^2l + s^3 per iteration "
+                    f"and unit) per step over {ns_ms:.3f} ms (CUDA events, mean of {steps} timed steps, "
+                    f"{ms_total / 1e3:.2f} s of timed work); dense-equivalent {dense:.1f} TFLOP/s; peak = "
+                    f"{pk['source']} {'sustained' if sustained else 'burst'} bf16 cuBLAS (burst "
+                    f"{pk['bf16_tflops']}, sustained {pk['bf16_tflops_sustained']}); frac of burst "
+                    f"{achieved / pk['bf16_tflops']:.3f}, of sustained {achieved / pk['bf16_tflops_sustained']:.3f}"}
+
+
+def momentum_roofline(wl, opt, mom_ms, pk):
+    """k = 0 (majority-vote Signum): the momentum pass dominates.  Fused (the
+    momentum kernel writes the signs) or momentum + bf16 copy."""
+    fused = getattr(opt, "fused_sign", False)
+    out_b = (1 / 8 if wl.variant == "pack1" else 1) if fused else 2
+    gbytes = wl.params * wl.n_workers * ((2 if wl.w_dtype == "bf16" else 4) + 8 + out_b)
+    achieved = gbytes / (mom_ms / 1e3) / 1e9
+    out_what = ("packed sign" if wl.variant == "pack1" else "int8 sign") if fused else "bf16 copy"
+    return {"bound": "hbm", "kernel": "momentum_kernel", "achieved": achieved, "peak": pk["hbm_gbs"],
+            "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": captured_traffic("momentum_kernel", wl.name),
+            "note": f"momentum call: {gbytes / 1e9:.3f} GB algorithmic (gradient read, fp32 momentum read+write, "
+                    f"{out_what} write) per step over {mom_ms:.3f} ms"}
+
+
+def time_workload(ctx, wl, args, *, norm, steps, warmup, graph=False, exchange=False, e2e=False, clocks=False):
+    """Builds the workload's optimizer and inputs on this rank and times
+    `steps` whole steps after `warmup` (CUDA events on the step's stream,
+    max over ranks).  Returns the measured figures."""
+    import torch
+    from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
+    dev, rank, world = ctx.dev, ctx.rank, ctx.world
+    dt = syn.torch_dtype(wl.w_dtype)
+    if exchange:
+        # One group of n_workers workers per GPU; the signs of all GPUs are
+        # exchanged (1-bit all-gather for packed workloads, int8 SUM
+        # all-reduce for int8 ones) and every GPU votes over all of them.
+        from sign_muon_optimizer_momentum_b200.distributed import SignMuonDistStep
+        if norm != "frobenius" or graph:
+            raise SystemExit("--exchange runs eagerly with the Frobenius scaling only")
+        opt = SignMuonDistStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
+                               polar=wl.polar, device=dev)
+    else:
+        opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
+                           polar=wl.polar, device=dev, norm=norm)
+    # Replicas draw their own problem; with --exchange all ranks share W and
+    # the gradient signal G* (one model, data-parallel), and their workers
+    # differ through the per-rank noise drawn below.
+    problem_seed = 0 if exchange else rank
+    weights = [w.to(dev) for w in syn.initial_weights(wl, problem_seed)]
+    signal = [g.to(dev) for g in syn.gradient_signal(wl, problem_seed)]
+    n_sets = 2
+    grad_sets = []
+    for t in range(n_sets):
+        gs = []
+        for i in range(len(wl.shapes)):
+            for m in range(wl.n_workers):
+                gs.append(syn.worker_gradient(wl, signal[i], i, m, t, rank))
+        grad_sets.append(gs)
+    del signal
+    stream = torch.cuda.current_stream(dev)
+    s_ptr = stream.cuda_stream
+
+    def one_step(t, ev=None):
+        gs = grad_sets[t % n_sets]
+        if ev is not None:
+            ev[0].record(stream)
+        opt.momentum_norm(gs, s_ptr)
+        if ev is not None:
+            ev[1].record(stream)
+        opt.newton_schulz(s_ptr)
+        if ev is not None:
+            ev[2].record(stream)
+        opt.vote_update(weights, s_ptr)
+        if ev is not None:
+            ev[3].record(stream)
+
+    graphs = None
+    if graph:
+        # One CUDA graph per gradient set: each replay is a whole step.
+        graphs = [opt.capture(weights, grad_sets[t]) for t in range(n_sets)]
+    for t in range(warmup):
+        if graphs:
+            graphs[t % n_sets].replay()
+        else:
+            one_step(t)
+    ctx.barrier()
+    if graphs:
+        # Phases from the captured kernels cannot be told apart on the host:
+        # they are taken from eager steps (same kernels), the step time from
+        # the replays.
+        ph_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(steps)]
+        for t in range(steps):
+            one_step(t, ph_ev[t])
+        ctx.barrier()
+    sampler = ClockSampler(ctx.local) if (clocks and rank == 0) else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx.barrier()
+    start.record(stream)
+    for t in range(steps):
+        if graphs:
+            graphs[t % n_sets].replay()
+        else:
+            one_step(t, ev[t])
+    stop.record(stream)
+    ctx.barrier()
+    ms = ctx.max_over_ranks(start.elapsed_time(stop))
+    if graphs:
+        ev = ph_ev
+    phases = {"momentum": sum(e[0].elapsed_time(e[1]) for e in ev) / steps,
+              "newton_schulz": sum(e[1].elapsed_time(e[2]) for e in ev) / steps,
+              "vote_update": sum(e[2].elapsed_time(e[3]) for e in ev) / steps}
+    clk = sampler.stop() if sampler else None
+    units_per_step = wl.params * wl.n_workers
+    out = {"ms_total": ms, "ms_per_step": ms / steps, "value": job_throughput(units_per_step, steps, world, ms),
+           "phases_ms": phases, "gpu_launches": opt.kernel_launches_per_step() * steps, "clocks": clk, "opt": opt}
+    if exchange:
+        out["exchange_bytes_per_step"] = opt.exchange_bytes_per_step()
+    if norm == "spectral":
+        # The power iterations alone, timed on the step's own bf16 copies of
+        # the momentum (they hold the last step's values).
+        from sign_muon_optimizer_momentum_b200 import _lib as L
+        xp = [x.data_ptr() for x in opt.x]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        for r in range(reps + 3):
+            if r == 3:
+                a.record(stream)
+            L.signmuon_spectral_norm(opt.shapes, opt.n_workers, xp, opt.spectral_iters, opt.inv_norm.data_ptr(),
+                                     opt.ws_spec.data_ptr(), opt.ws_spec.numel(), s_ptr)
+        b.record(stream)
+        ctx.barrier()
+        out["spectral_ms"] = ctx.max_over_ranks(a.elapsed_time(b)) / reps
+    if e2e:
+        # End to end through the public step with HOST buffers: each step's
+        # gradients come from pinned host memory and the updated weights go
+        # back to host memory.  The next step's gradients are copied on a
+        # second stream while the current step computes (copy engines overlap
+        # the kernels).
+        host_g = [g.cpu().pin_memory() for g in grad_sets[0]]
+        host_w = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in weights]
+        h2d = sum(g.numel() * g.element_size() for g in host_g)
+        d2h = sum(w.numel() * w.element_size() for w in weights)
+        copy_stream = torch.cuda.Stream(dev)
+        copied = [torch.cuda.Event(), torch.cuda.Event()]
+        consumed = [torch.cuda.Event(), torch.cuda.Event()]
+
+        def h2d_into(buf):
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(consumed[buf])
+                for hg, dg in zip(host_g, grad_sets[buf]):
+                    dg.copy_(hg, non_blocking=True)
+                copied[buf].record(copy_stream)
+
+        def e2e_steps(n):
+            h2d_into(0)
+            for t in range(n):
+                buf = t % 2
+                if t + 1 < n:
+                    h2d_into(1 - buf)
+                stream.wait_event(copied[buf])
+                opt.step(weights, grad_sets[buf])
+                consumed[buf].record(stream)
+                for hw, w in zip(host_w, weights):
+                    hw.copy_(w, non_blocking=True)
+
+        e2e_steps(2)
+        ctx.barrier()
+        e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(steps, 10))
+        e_start.record(stream)
+        e2e_steps(n_e2e)
+        e_stop.record(stream)
+        ctx.barrier()
+        e_ms = ctx.max_over_ranks(e_start.elapsed_time(e_stop))
+        out["e2e"] = {"value": units_per_step * n_e2e * world / (e_ms / 1e3), "unit": UNIT,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+                      "ms_per_step": e_ms / n_e2e,
+                      "note": "gradients H2D from pinned host memory (overlapped with the previous step on a copy "
+                              "stream) + step + weights D2H, every step"}
+        del host_g, host_w
+    if graphs:
+        del graphs
+    return out
+
+
+def extra_signum(ctx, args, pk):
+    """Majority-vote Signum (k = 0) on the nanoGPT-small matrices: the fused
+    momentum + sign pass, then the vote + update."""
+    from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    wl = syn.WORKLOADS["signum_nanogpt_small"]
+    r = time_workload(ctx, wl, args, norm="frobenius", steps=50, warmup=5)
+    return {"workload": wl.name, "config": workload_config(wl), "metric": METRIC, "value": r["value"], "unit": UNIT,
+            "ms_per_step": r["ms_per_step"], "steps": 50, "warmup": 5, "phases_ms": r["phases_ms"],
+            "roofline": momentum_roofline(wl, r["opt"], r["phases_ms"]["momentum"], pk)}
+
+
+def extra_spectral(ctx, args, pk):
+    """The nanoGPT-small step with spectral scaling of the Newton-Schulz input
+    (5 power iterations per unit); roofline of the power-iteration kernels:
+    per iteration each unit's bf16 copy of M is read once (2 B/param), its
+    row-block partial sums written and read back (1/8 + 1/8 B/param)."""
+    from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    wl = syn.WORKLOADS["nanogpt_small"]
+    r = time_workload(ctx, wl, args, norm="spectral", steps=20, warmup=3)
+    iters = r["opt"].spectral_iters
+    gbytes = iters * wl.params * wl.n_workers * 2.25
+    achieved = gbytes / (r["spectral_ms"] / 1e3) / 1e9
+    return {"workload": wl.name, "config": dict(workload_config(wl), norm="spectral", spectral_iters=iters),
+            "metric": METRIC, "value": r["value"], "unit": UNIT, "ms_per_step": r["ms_per_step"], "steps": 20,
+            "warmup": 3, "phases_ms": dict(r["phases_ms"], spectral_alone=r["spectral_ms"]),
+            "roofline": {"bound": "hbm", "kernel": "spectral_rowpass_kernel", "achieved": achieved,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                         "traffic": captured_traffic("spectral_rowpass_kernel", wl.name)
+                         if "spectral_rowpass_kernel" in KERNEL_SOURCES else None,
+                         "note": f"{iters} power iterations: {gbytes / 1e9:.3f} GB algorithmic (2.25 B per "
+                                 f"param*worker and iteration) over {r['spectral_ms']:.3f} ms, timed alone"}}
+
+
 def run_gpu(args, wl):
     import torch
     import torch.distributed as dist
     from sign_muon_optimizer_momentum_b200 import build as _build
-    from sign_muon_optimizer_momentum_b200 import synthetic as syn
-    from sign_muon_optimizer_momentum_b200.step import SignMuonStep
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -323,210 +598,34 @@ def run_gpu(args, wl):
             dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
                                     timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", 0))
     _build.build()
-    dev = torch.device("cuda", torch.cuda.current_device())
-    dt = syn.torch_dtype(wl.w_dtype)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x):
-        return max_over_ranks_value(x, world, dev)
-
-    if args.exchange:
-        # One group of n_workers workers per GPU; the signs of all GPUs are
-        # exchanged (1-bit all-gather for packed workloads, int8 SUM
-        # all-reduce for int8 ones) and every GPU votes over all of them.
-        from sign_muon_optimizer_momentum_b200.distributed import SignMuonDistStep
-        if args.norm != "frobenius" or args.graph:
-            raise SystemExit("--exchange runs eagerly with the Frobenius scaling only")
-        opt = SignMuonDistStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
-                               polar=wl.polar, device=dev)
-    else:
-        opt = SignMuonStep(wl.shapes, wl.n_workers, wl.ns_iters, wl.variant, wl.beta, wl.eta, dt,
-                           polar=wl.polar, device=dev, norm=args.norm)
-    # Replicas draw their own problem; with --exchange all ranks share W and
-    # the gradient signal G* (one model, data-parallel), and their workers
-    # differ through the per-rank noise drawn below.
-    problem_seed = 0 if args.exchange else rank
-    weights = [w.to(dev) for w in syn.initial_weights(wl, problem_seed)]
-    signal = [g.to(dev) for g in syn.gradient_signal(wl, problem_seed)]
-    n_sets = 2
-    grad_sets = []
-    for t in range(n_sets):
-        gs = []
-        for i in range(len(wl.shapes)):
-            for m in range(wl.n_workers):
-                gs.append(syn.worker_gradient(wl, signal[i], i, m, t, rank))
-        grad_sets.append(gs)
-    del signal
-    stream = torch.cuda.current_stream(dev)
-    s_ptr = stream.cuda_stream
-    resident = sum(g.numel() * g.element_size() for g in grad_sets[0]) + sum(m.numel() * 4 for m in opt.mom)
-
-    def one_step(t, ev=None):
-        gs = grad_sets[t % n_sets]
-        if ev is not None:
-            ev[0].record(stream)
-        opt.momentum_norm(gs, s_ptr)
-        if ev is not None:
-            ev[1].record(stream)
-        opt.newton_schulz(s_ptr)
-        if ev is not None:
-            ev[2].record(stream)
-        opt.vote_update(weights, s_ptr)
-        if ev is not None:
-            ev[3].record(stream)
-
-    graphs = None
-    if args.graph:
-        # One CUDA graph per gradient set: each replay is a whole step.
-        graphs = [opt.capture(weights, grad_sets[t]) for t in range(n_sets)]
-
-    for t in range(args.warmup):
-        if graphs:
-            graphs[t % n_sets].replay()
-        else:
-            one_step(t)
-    barrier()
-
-    if graphs:
-        # Phases from the captured kernels cannot be told apart on the host:
-        # they are taken from eager steps (same kernels), the step time from
-        # the replays.
-        ph_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(args.steps)]
-        for t in range(args.steps):
-            one_step(t, ph_ev[t])
-        barrier()
-
-    clocks = ClockSampler(local) if rank == 0 else None
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    ns_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    start.record(stream)
-    for t in range(args.steps):
-        if graphs:
-            graphs[t % n_sets].replay()
-        else:
-            one_step(t, ns_ev[t])
-    stop.record(stream)
-    barrier()
-    ms = max_over_ranks(start.elapsed_time(stop))
-    if graphs:
-        ns_ev = ph_ev
-    mom_ms = sum(e[0].elapsed_time(e[1]) for e in ns_ev) / args.steps
-    ns_ms = sum(e[1].elapsed_time(e[2]) for e in ns_ev) / args.steps
-    vote_ms = sum(e[2].elapsed_time(e[3]) for e in ns_ev) / args.steps
-    clk = clocks.stop() if clocks else None
-
-    units_per_step = wl.params * wl.n_workers
-    value = job_throughput(units_per_step, args.steps, world, ms)
-
-    # End to end through the public step with HOST buffers: each step's
-    # gradients come from pinned host memory and the updated weights go back
-    # to host memory.  The next step's gradients are copied on a second stream
-    # while the current step computes (copy engines overlap the kernels).
-    host_g = [g.cpu().pin_memory() for g in grad_sets[0]]
-    host_w = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in weights]
-    h2d = sum(g.numel() * g.element_size() for g in host_g)
-    d2h = sum(w.numel() * w.element_size() for w in weights)
-    copy_stream = torch.cuda.Stream(dev)
-    copied = [torch.cuda.Event(), torch.cuda.Event()]
-    consumed = [torch.cuda.Event(), torch.cuda.Event()]
-
-    def h2d_into(buf):
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(consumed[buf])
-            for hg, dg in zip(host_g, grad_sets[buf]):
-                dg.copy_(hg, non_blocking=True)
-            copied[buf].record(copy_stream)
-
-    def e2e_steps(n):
-        h2d_into(0)
-        for t in range(n):
-            buf = t % 2
-            if t + 1 < n:
-                h2d_into(1 - buf)
-            stream.wait_event(copied[buf])
-            opt.step(weights, grad_sets[buf])
-            consumed[buf].record(stream)
-            for hw, w in zip(host_w, weights):
-                hw.copy_(w, non_blocking=True)
-
-    e2e_steps(2)
-    barrier()
-    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(3, min(args.steps, 10))
-    e_start.record(stream)
-    e2e_steps(n_e2e)
-    e_stop.record(stream)
-    barrier()
-    e_ms = max_over_ranks(e_start.elapsed_time(e_stop))
-    e2e = {"value": units_per_step * n_e2e * world / (e_ms / 1e3), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-           "ms_per_step": e_ms / n_e2e,
-           "note": "gradients H2D from pinned host memory (overlapped with the previous step on a copy "
-                   "stream) + step + weights D2H, every step"}
-
+    ctx = Ctx(world, rank, local, torch.device("cuda", torch.cuda.current_device()))
     pk = peaks()
+    r = time_workload(ctx, wl, args, norm=args.norm, steps=args.steps, warmup=args.warmup, graph=args.graph,
+                      exchange=args.exchange, e2e=True, clocks=True)
     if wl.ns_iters > 0:
-        flops = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters)
-        if wl.polar:
-            flops_note = "Newton-Schulz call of the step (the local polar step is timed with the vote)"
-        else:
-            flops_note = "Newton-Schulz call of the step"
-        achieved = flops / (ns_ms / 1e3) / 1e12
-        dense = ns_flops(wl.shapes, wl.n_workers, wl.ns_iters, True) / (ns_ms / 1e3) / 1e12
-        # The kernel runs inside the timed steps back to back: over a timed
-        # region of half a second or more the GPU sits at its power cap, the
-        # condition of the sustained bf16 peak; shorter regions compare with
-        # the burst peak.
-        sustained = ms >= 500.0
-        peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-        roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved,
-                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                    "traffic": captured_traffic("ns_gemm_kernel", wl.name),
-                    "note": f"{flops_note}: {flops / 1e12:.3f} TFLOP algorithmic (symmetric-aware: 3s^2l + s^3 "
-                            f"per iteration and unit) per step over {ns_ms:.3f} ms (CUDA events, mean of "
-                            f"{args.steps} timed steps, {ms / 1e3:.2f} s of timed work); dense-equivalent "
-                            f"{dense:.1f} TFLOP/s; peak = {pk['source']} "
-                            f"{'sustained' if sustained else 'burst'} bf16 cuBLAS (burst {pk['bf16_tflops']}, "
-                            f"sustained {pk['bf16_tflops_sustained']}); frac of burst "
-                            f"{achieved / pk['bf16_tflops']:.3f}"}
+        roofline = ns_roofline(wl, r["phases_ms"]["newton_schulz"], r["ms_total"], pk, args.steps)
     else:
-        # k = 0 (majority-vote Signum): the momentum pass dominates.  Fused
-        # (the momentum kernel writes the signs) or momentum + bf16 copy.
-        fused = getattr(opt, "fused_sign", False)
-        out_b = (1 / 8 if wl.variant == "pack1" else 1) if fused else 2
-        gbytes = wl.params * wl.n_workers * ((2 if wl.w_dtype == "bf16" else 4) + 8 + out_b)
-        achieved = gbytes / (mom_ms / 1e3) / 1e9
-        out_what = ("packed sign" if wl.variant == "pack1" else "int8 sign") if fused else "bf16 copy"
-        roofline = {"bound": "hbm", "kernel": "momentum_kernel", "achieved": achieved, "peak": pk["hbm_gbs"],
-                    "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                    "traffic": captured_traffic("momentum_kernel", wl.name),
-                    "note": f"momentum call: {gbytes / 1e9:.3f} GB algorithmic (gradient read, fp32 momentum "
-                            f"read+write, {out_what} write) per step over {mom_ms:.3f} ms"}
-    result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-              "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        roofline = momentum_roofline(wl, r["opt"], r["phases_ms"]["momentum"], pk)
+    result = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+              "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-              "config": dict(workload_config(wl), norm=args.norm,
-                             parallelism=(f"dp{world}-{'allgather' if wl.variant == 'pack1' else 'allreduce'}"
-                                          if args.exchange else f"replicas{world}"),
-                             l2=f"inputs larger than L2 ({resident / 2**30:.1f} GiB gradients+momentum resident)"),
-              "roofline": roofline, "e2e": e2e,
-              "phases_ms": {"momentum": mom_ms, "newton_schulz": ns_ms, "vote_update": vote_ms},
-              "gpu_launches": opt.kernel_launches_per_step() * args.steps,
-              "clocks": clk}
-    result["config"]["launch"] = "cuda_graph" if graphs else "eager"
+              "config": line_config(wl, args, world), "roofline": roofline, "e2e": r["e2e"],
+              "phases_ms": r["phases_ms"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"]}
     if args.exchange:
         result["config"]["vote_workers"] = world * wl.n_workers
-        result["config"]["exchange_bytes_per_step"] = opt.exchange_bytes_per_step()
+        result["config"]["exchange_bytes_per_step"] = r["exchange_bytes_per_step"]
+    del r
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl)
+    if wl.name == DEFAULT_CONFIG and not args.no_extras and not args.exchange:
+        # Rows measured beside the headline workload, each with its roofline.
+        result["vote_sweep"] = time_vote_sweep(ctx, 1 << 30, 16, "f32", steps=20, warmup=5)
+        torch.cuda.empty_cache()
+        result["signum"] = extra_signum(ctx, args, pk)
+        torch.cuda.empty_cache()
+        result["spectral"] = extra_spectral(ctx, args, pk)
+        torch.cuda.empty_cache()
     if pg:
         dist.barrier()
         dist.destroy_process_group()
@@ -535,14 +634,71 @@ def run_gpu(args, wl):
     return 0
 
 
-def run_vote_sweep(args):
+def time_vote_sweep(ctx, P, M, w_dtype, steps, warmup, clocks=False):
     """Vote + update alone (the bandwidth-bound row): P params as (P/1024, 1024)
-    W (fp32 by default, or bf16), M packed sign buffers with P(+1) ~ U(0,1)
-    per entry."""
+    W (fp32 or bf16), M packed sign buffers with P(+1) ~ U(0,1) per entry."""
     import torch
     from sign_muon_optimizer_momentum_b200 import _lib as L
-    from sign_muon_optimizer_momentum_b200 import build as _build
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    dev, rank, world = ctx.dev, ctx.rank, ctx.world
+    shape = (P // 1024, 1024)
+    stream = torch.cuda.current_stream(dev)
+    words = L.signmuon_packed_words(shape)
+    signs = []
+    for m, s8 in syn.vote_sweep_signs(P, M, seed=rank, device=dev):
+        buf = torch.empty(words, dtype=torch.int32, device=dev)
+        L.signmuon_sign_pack(shape, L.SIGNMUON_F32, s8.float().data_ptr(), 1024, 0, buf.data_ptr(),
+                             stream.cuda_stream)
+        torch.cuda.synchronize()
+        signs.append(buf)
+        del s8
+    w_bf16 = w_dtype == "bf16"
+    w = syn.gaussian(shape, 0.02, dev, "W", rank, 0, dtype=torch.bfloat16 if w_bf16 else torch.float32)
+    w_code = L.SIGNMUON_BF16 if w_bf16 else L.SIGNMUON_F32
+    w_bytes = 2 if w_bf16 else 4
+    wsz = L.signmuon_vote_workspace_bytes([shape], M)
+    wsb = torch.zeros(wsz, dtype=torch.uint8, device=dev)
+    sp = [t.data_ptr() for t in signs]
+
+    def step():
+        L.signmuon_vote_update([shape], M, False, sp, w_code, [w.data_ptr()], 0.01, None, 0, 0,
+                               wsb.data_ptr(), wsz, stream.cuda_stream)
+
+    for _ in range(warmup):
+        step()
+    ctx.barrier()
+    sampler = ClockSampler(ctx.local) if (clocks and rank == 0) else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    ctx.barrier()
+    ms = ctx.max_over_ranks(a.elapsed_time(b))
+    clk = sampler.stop() if sampler else None
+    per = ms / steps
+    bytes_per = P * (M / 8 + 2 * w_bytes)
+    pk = peaks()
+    gbs = bytes_per / (per / 1e3) / 1e9
+    return {"metric": METRIC, "value": P * M * world / (per / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": per, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+            "config": {"workload": "vote_sweep", "params": P, "workers": M, "w_dtype": w_dtype, "eta": 0.01,
+                       "l2": f"inputs larger than L2 ({bytes_per / 2**30:.2f} GiB per step)"},
+            "roofline": {"bound": "hbm", "kernel": "vote_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                         "traffic": captured_traffic("vote_kernel", f"vote_sweep_P{P}_M{M}_{w_dtype}"),
+                         "note": f"algorithmic {M}/8 + {2 * w_bytes} B/param (packed signs read, "
+                                 f"{w_dtype} W read+write); peak = {pk['source']} copy bandwidth"},
+            "gpu_launches": 2 * steps, "clocks": clk}
+
+
+def run_vote_sweep(args):
+    import torch
+    from sign_muon_optimizer_momentum_b200 import build as _build
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -555,66 +711,9 @@ def run_vote_sweep(args):
     else:
         torch.cuda.set_device(0)
     _build.build()
-    dev = torch.device("cuda", torch.cuda.current_device())
-    P, M = args.sweep_params, args.sweep_workers
-    shape = (P // 1024, 1024)
-    stream = torch.cuda.current_stream(dev)
-    words = L.signmuon_packed_words(shape)
-    signs = []
-    for m, s8 in syn.vote_sweep_signs(P, M, seed=rank, device=dev):
-        buf = torch.empty(words, dtype=torch.int32, device=dev)
-        L.signmuon_sign_pack(shape, L.SIGNMUON_F32, s8.float().data_ptr(), 1024, 0, buf.data_ptr(),
-                             stream.cuda_stream)
-        torch.cuda.synchronize()
-        signs.append(buf)
-        del s8
-    w_bf16 = args.sweep_w_dtype == "bf16"
-    w = syn.gaussian(shape, 0.02, dev, "W", rank, 0, dtype=torch.bfloat16 if w_bf16 else torch.float32)
-    w_code = L.SIGNMUON_BF16 if w_bf16 else L.SIGNMUON_F32
-    w_bytes = 2 if w_bf16 else 4
-    wsz = L.signmuon_vote_workspace_bytes([shape], M)
-    wsb = torch.zeros(wsz, dtype=torch.uint8, device=dev)
-    sp = [t.data_ptr() for t in signs]
-
-    def step():
-        L.signmuon_vote_update([shape], M, False, sp, w_code, [w.data_ptr()], 0.01, None, 0, 0,
-                               wsb.data_ptr(), wsz, stream.cuda_stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local) if rank == 0 else None
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(args.steps):
-        step()
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-    clk = clocks.stop() if clocks else None
-    per = ms / args.steps
-    bytes_per = P * (M / 8 + 2 * w_bytes)
-    pk = peaks()
-    gbs = bytes_per / (per / 1e3) / 1e9
-    res = {"metric": METRIC, "value": P * M * world / (per / 1e3), "unit": UNIT, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": per, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
-           "config": {"workload": "vote_sweep", "params": P, "workers": M, "w_dtype": args.sweep_w_dtype, "eta": 0.01,
-                      "l2": f"inputs larger than L2 ({bytes_per / 2**30:.2f} GiB per step)"},
-           "roofline": {"bound": "hbm", "kernel": "vote_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
-                        "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
-                        "traffic": captured_traffic("vote_kernel", f"vote_sweep_P{P}_M{M}_{args.sweep_w_dtype}"),
-                        "note": f"algorithmic {M}/8 + {2 * w_bytes} B/param (packed signs read, "
-                                f"{args.sweep_w_dtype} W read+write)"},
-           "gpu_launches": 2 * args.steps, "clocks": clk}
+    ctx = Ctx(world, rank, local, torch.device("cuda", torch.cuda.current_device()))
+    res = time_vote_sweep(ctx, args.sweep_params, args.sweep_workers, args.sweep_w_dtype, args.steps, args.warmup,
+                          clocks=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -631,6 +730,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--mats", type=int, default=None,
                     help="keep only the first N matrices of the workload (small profiling cases)")
+    ap.add_argument("--workers", type=int, default=None,
+                    help="override the workload's number of workers (small profiling cases)")
     ap.add_argument("--sweep-params", type=int, default=1 << 30)
     ap.add_argument("--sweep-workers", type=int, default=16)
     ap.add_argument("--sweep-w-dtype", default="f32", choices=["f32", "bf16"],
@@ -638,6 +739,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the vote-sweep, Signum and spectral rows measured beside the default workload")
     ap.add_argument("--norm", default="frobenius", choices=["frobenius", "spectral"],
                     help="scaling of the Newton-Schulz input (spectral: 5 power iterations)")
     ap.add_argument("--graph", action="store_true",
@@ -653,9 +756,11 @@ def main():
             args.steps = 50
         return run_vote_sweep(args)
     wl = syn.WORKLOADS[args.config]
-    if args.mats:
+    if args.mats or args.workers:
         import dataclasses
-        wl = dataclasses.replace(wl, name=f"{wl.name}[:{args.mats}]", shapes=wl.shapes[: args.mats])
+        name = wl.name + (f"[:{args.mats}]" if args.mats else "") + (f"[M={args.workers}]" if args.workers else "")
+        wl = dataclasses.replace(wl, name=name, shapes=wl.shapes[: args.mats] if args.mats else wl.shapes,
+                                 n_workers=args.workers or wl.n_workers)
     if args.steps is None:
         args.steps = 10 if args.impl == "reference" else DEFAULT_STEPS.get(wl.name, 20)
     if args.warmup < 3 and args.impl == "ours":

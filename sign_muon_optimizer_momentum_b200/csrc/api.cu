@@ -543,6 +543,21 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
   NsUnit* d_units = reinterpret_cast<NsUnit*>(hdr->workspace + kWsHeaderBytes);
   const NsTileRec* d_recs =
       reinterpret_cast<const NsTileRec*>(hdr->workspace + kWsHeaderBytes + ns_desc_bytes(hdr->n_units));
+  // SIGNMUON_NS_INJECT_WAIT_TIMEOUT_US=<n> (1 <= n <= 2000000): fault
+  // injection for testing the bounded waits.  Every Newton-Schulz GEMM
+  // launch withholds its operand loads and gives up waiting after n
+  // microseconds, recording a wait-timeout code in the workspace; its
+  // outputs are left unwritten.  Unset (the default): full 2 s limit, normal
+  // operation.
+  uint64_t wait_limit_ns = kWaitTimeoutNs;
+  int withhold = 0;
+  if (const char* inj = getenv("SIGNMUON_NS_INJECT_WAIT_TIMEOUT_US")) {
+    const long us = strtol(inj, nullptr, 10);
+    if (us >= 1 && us <= 2000000) {
+      wait_limit_ns = (uint64_t)us * 1000ull;
+      withhold = 1;
+    }
+  }
   cudaError_t e = cudaSuccess;
   for (int wv = 0; wv < hdr->n_waves; ++wv) {
     const NsPlanWave& W = waves[wv];
@@ -565,6 +580,8 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
       L.eta = eta;
       L.w_dtype = hdr->w_dtype;
       L.err = reinterpret_cast<uint32_t*>(hdr->workspace);
+      L.wait_limit_ns = wait_limit_ns;
+      L.withhold_loads = withhold;
       for (int stg = 0; stg < 3; ++stg) {
         L.stage = stg;
         L.recs = d_recs + W.rec0[stg];

@@ -122,6 +122,11 @@ struct NsLaunch {
   int pair;         // 1: CTA-pair (cta_group::2) 256x256 tiles; 0: one CTA, 128x256
   float a, b, c, eta;
   uint32_t* err;
+  uint64_t wait_limit_ns;  // every bounded wait gives up after this long
+  // Fault injection for testing the bounded waits: the producer arms no
+  // barrier and issues no copy, so the consumers' waits run out.
+  int withhold_loads;
+  int pad_;
 };
 
 // Momentum units.

@@ -75,9 +75,10 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Returns
-// false if it did not within kWaitTimeoutNs, or if another role has already
-// given up (abort flag set).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// false if it did not within limit_ns, or if another role has already given
+// up (abort flag set).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t n = 0;
@@ -85,7 +86,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_test(bar, parity)) return true;
     if ((++n & 63) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
     }
   }
 }
@@ -167,6 +168,37 @@ __device__ __forceinline__ uint16_t to16(float x, bool half) {
 }
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool half) {
   return (uint32_t)to16(lo, half) | ((uint32_t)to16(hi, half) << 16);
+}
+
+// W - eta * u rounded once, to nearest (ties to even), to bf16: the rare
+// case of update_bf16 below.  The fp32 value s = fmaf(-eta, u, w) is a bf16
+// midpoint; the exact difference lies on one side of it or on it.  In fp64
+// p = eta * u is exact, the two-sum rule splits w - p exactly into hi + lo,
+// and hi - s is exact (hi and s both lie within an fp32 ulp of the exact
+// value), so the side is the sign of hi - s, or of lo when hi == s.
+__device__ __noinline__ uint32_t update_bf16_midpoint(float w, float eta, float u, float s) {
+  const double wd = (double)w;
+  const double p = (double)eta * (double)u;
+  const double hi = wd - p;
+  const double z = hi - wd;
+  const double lo = (wd - (hi - z)) + (-p - z);
+  const double diff = hi - (double)s;
+  const int side = diff > 0.0 ? 1 : diff < 0.0 ? -1 : (lo > 0.0 ? 1 : (lo < 0.0 ? -1 : 0));
+  const uint32_t bits = __float_as_uint(s);
+  const uint32_t t = bits >> 16;  // s truncated toward zero: the bf16 neighbour nearer 0
+  const bool neg = (bits >> 31) != 0;
+  const bool away = side == 0 ? (t & 1u) != 0 : (neg ? side < 0 : side > 0);
+  return t + (away ? 1u : 0u);
+}
+
+// bf16 W - eta * u with a single rounding of the exact difference.  fmaf
+// rounds the exact value to fp32; a bf16 rounding boundary is an fp32 value,
+// so that fp32 value rounds to the same bf16 as the exact one unless it is
+// itself a bf16 midpoint (low 16 bits 0x8000).
+__device__ __forceinline__ __nv_bfloat16 update_bf16(float w, float eta, float u) {
+  const float s = fmaf(-eta, u, w);
+  if ((__float_as_uint(s) & 0xFFFFu) != 0x8000u || !isfinite(s)) return __float2bfloat16_rn(s);
+  return __ushort_as_bfloat16((unsigned short)update_bf16_midpoint(w, eta, u, s));
 }
 
 // Byte offset of element (r, c) in a 32x32 16-bit staging block laid out as the
@@ -488,11 +520,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         const int b_row0 = T.n0 + (int)rank * C::kRowsB;
         const bool b_from_a = diag_b_from_a<kPair>(L, T);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(smem_addr(&empty_bar[stage]), phase ^ 1, abort_flag)) {
+          if (!mbar_wait(smem_addr(&empty_bar[stage]), phase ^ 1, abort_flag, L.wait_limit_ns)) {
             atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutProducer);
             *abort_flag = 1;
             ok = false;
             break;
+          }
+          if (L.withhold_loads) {
+            // Fault injection: nothing is armed or copied, so this stage's
+            // full barrier never completes and the MMA issuer's wait runs
+            // out (no copy is in flight at exit).
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            continue;
           }
           const uint32_t own_full = smem_addr(&full_bar[stage]);
           // Pair mode: both CTAs' copies complete on the even CTA's barrier,
@@ -545,7 +584,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         const bool fp16_ops = L.stage == kStageSquare;
         const bool b_from_a = diag_b_from_a<kPair>(L, T);
         const int nkb = (T.K + kBK - 1) / kBK;
-        if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag)) {
+        if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag, L.wait_limit_ns)) {
           atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
           *abort_flag = 1;
           break;
@@ -553,7 +592,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         tc_fence_after();
         const uint32_t tmem_d = tmem_base + (uint32_t)(acc * kAccCols);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(smem_addr(&full_bar[stage]), phase, abort_flag)) {
+          if (!mbar_wait(smem_addr(&full_bar[stage]), phase, abort_flag, L.wait_limit_ns)) {
             atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
             *abort_flag = 1;
             ok = false;
@@ -584,11 +623,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       }
       // Drain: wait until every MMA this thread issued has completed.
       tc_commit<kPair>(smem_addr(drain_bar));
-      if (!mbar_wait(smem_addr(drain_bar), 0, abort_flag)) {
+      if (!mbar_wait(smem_addr(drain_bar), 0, abort_flag, L.wait_limit_ns)) {
         // Ignore the abort flag for the drain itself: wait out the full limit.
         const uint64_t t0 = global_timer_ns();
         while (!mbar_test(smem_addr(drain_bar), 0)) {
-          if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+          if (global_timer_ns() - t0 > L.wait_limit_ns) {
             atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutDrain);
             break;
           }
@@ -639,7 +678,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         s = L.first ? __ldg(L.scales + rec.unit) : 1.f;
       }
       const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
-      if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag)) {
+      if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag, L.wait_limit_ns)) {
         atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutEpilogue);
         *abort_flag = 1;
         break;
@@ -778,13 +817,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                   __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&raw[q4]);
 #pragma unroll
                   for (int j = 0; j < 8; ++j)
-                    e[j] = __float2bfloat16_rn(fmaf(-L.eta, v[8 * q4 + j], __bfloat162float(e[j])));
+                    e[j] = update_bf16(__bfloat162float(e[j]), L.eta, v[8 * q4 + j]);
                   reinterpret_cast<uint4*>(w)[q4] = raw[q4];
                 }
               } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                  if (j < nvalid) w[j] = __float2bfloat16_rn(fmaf(-L.eta, v[j], __bfloat162float(w[j])));
+                  if (j < nvalid) w[j] = update_bf16(__bfloat162float(w[j]), L.eta, v[j]);
               }
             } else {
               float* w = static_cast<float*>(uf.out) + off;
@@ -840,7 +879,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       const uint32_t bar = rank == 0 ? smem_addr(&full_bar[s]) : smem_addr(&empty_bar[s]);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_test(bar, last_round & 1)) {
-        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        if (global_timer_ns() - t0 > L.wait_limit_ns) {
           atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutDrain);
           break;
         }

@@ -23,6 +23,12 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    # The same config dict as the GPU arm prints for this workload and launch.
+    sys.path.insert(0, ROOT)
+    import bench
+    from sign_muon_optimizer_momentum_b200 import synthetic as syn
+    args = type("A", (), {"norm": "frobenius", "exchange": False, "graph": False})()
+    assert d["config"] == bench.line_config(syn.WORKLOADS["single256"], args, 1)
 
 
 def test_reference_arm_runs_on_rank_zero_only():

@@ -5,8 +5,10 @@ CPU: the exchange layout and the collectives on two gloo ranks — every slot
 the vote reads holds the right rank's signs for the right (matrix, worker).
 GPU: two ranks emulated in one process (the exchange done by concatenation /
 addition on the device, no collective) give bit for bit the weights of the
-single-process step over all their workers; one NCCL rank runs the
-pipelined step() and matches it too."""
+single-process step over all their workers, and -- fed every rank's own
+signs -- the oracle's majority vote and update give bit for bit the same
+weights (the vote matrix, for the local polar step); one NCCL rank runs the
+pipelined step() and matches both too."""
 import os
 import socket
 
@@ -169,6 +171,41 @@ def _grads(shapes, M, step, dtype):
             for i in range(len(shapes)) for m in range(M)]
 
 
+def _unit_signs(buf, off, shape, variant):
+    """The {-1,+1} signs of one unit from an exchange buffer (packed words or
+    int8 at element offset `off`)."""
+    from oracle import signmuon_oracle as O
+    r, c = shape
+    if variant == "pack1":
+        wpr = (c + 31) // 32
+        words = buf[off:off + r * wpr].cpu().numpy().view(np.uint32).reshape(r, wpr)
+        return O.unpack_signs(words, c)
+    return buf[off:off + r * c].cpu().numpy().reshape(r, c)
+
+
+def _oracle_votes(shapes, layout, local_bufs, variant):
+    """The oracle's majority vote of every matrix over all world x local
+    workers, from each rank's own (pre-exchange) sign buffers; global worker
+    r * local_workers + m."""
+    from oracle import signmuon_oracle as O
+    Ml = layout.local_workers
+    votes = []
+    for i, shape in enumerate(shapes):
+        g = layout.group_of[i]
+        signs = [_unit_signs(bufs[g], layout.offsets[i * Ml + m], shape, variant)
+                 for bufs in local_bufs for m in range(Ml)]
+        votes.append(O.majority_vote(signs))
+    return votes
+
+
+def _check_against_oracle(shapes, votes, w_prev, w_new, dtype, eta):
+    from oracle import signmuon_oracle as O
+    wd = "bf16" if dtype == torch.bfloat16 else "f32"
+    for i, shape in enumerate(shapes):
+        ref = O.apply_update(w_prev[i].double().cpu().numpy(), eta, votes[i], wd)
+        assert np.array_equal(w_new[i].double().cpu().numpy(), ref), shape
+
+
 def _single_process_reference(shapes, M, k, variant, dtype, steps, polar):
     from sign_muon_optimizer_momentum_b200.step import SignMuonStep
     opt = SignMuonStep(shapes, M, k, variant, 0.9, 0.02, dtype, polar=polar)
@@ -196,6 +233,10 @@ def test_two_emulated_ranks_match_single_process(cuda_lib, monkeypatch, variant,
         for r, rk in enumerate(ranks):
             mine = [g_all[i * M + r * Ml + m].cuda() for i in range(len(shapes)) for m in range(Ml)]
             rk.local_phase(mine)
+        torch.cuda.synchronize()
+        # Oracle: the majority vote of every rank's own signs, then the update.
+        votes = _oracle_votes(shapes, ranks[0].layout, [[b.clone() for b in rk.local] for rk in ranks], variant)
+        w_prev = [[x.clone() for x in w] for w in ws]
         for g in range(len(ranks[0].layout.groups)):     # the exchange, done on the device
             if variant == "pack1":
                 cat = torch.cat([rk.local[g] for rk in ranks])
@@ -207,7 +248,13 @@ def test_two_emulated_ranks_match_single_process(cuda_lib, monkeypatch, variant,
                     rk.local[g].copy_(tot)
         for rk, w in zip(ranks, ws):
             rk.vote_phase(w)
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        for rk, w, wp in zip(ranks, ws, w_prev):
+            if polar:      # the vote matrix the local polar step starts from
+                for i, (r_, c_) in enumerate(shapes):
+                    assert np.array_equal(rk.vote[i][:, :c_].double().cpu().numpy(), votes[i])
+            else:          # vote + update bit-exact against the oracle
+                _check_against_oracle(shapes, votes, wp, w, dtype, 0.02)
     for w in ws:
         for a, b in zip(w, ref):
             assert torch.equal(a.cpu(), b)
@@ -227,8 +274,13 @@ def test_nccl_single_rank_step_matches_single_process(cuda_lib, monkeypatch, var
         opt = D.SignMuonDistStep(shapes, Ml, k, variant, 0.9, 0.02, dtype, n_groups=3)
         w = [syn.gaussian(s, 0.02, "cpu", "Wd", i, dtype=dtype).cuda() for i, s in enumerate(shapes)]
         for t in range(steps):
+            w_prev = [x.clone() for x in w]
             opt.step(w, [g.cuda() for g in _grads(shapes, Ml, t, dtype)])
-        torch.cuda.synchronize()
+            torch.cuda.synchronize()
+            # After the collective (one rank) the local buffers still hold this
+            # rank's signs: the oracle's vote + update of them is bit-exact.
+            votes = _oracle_votes(shapes, opt.layout, [opt.local], variant)
+            _check_against_oracle(shapes, votes, w_prev, w, dtype, 0.02)
         for a, b in zip(w, ref):
             assert torch.equal(a.cpu(), b)
         assert opt.exchange_bytes_per_step() == sum(opt.layout.group_len) * (4 if variant == "pack1" else 1)
