@@ -601,7 +601,7 @@ def run_gpu(args, wl):
     ctx = Ctx(world, rank, local, torch.device("cuda", torch.cuda.current_device()))
     pk = peaks()
     r = time_workload(ctx, wl, args, norm=args.norm, steps=args.steps, warmup=args.warmup, graph=args.graph,
-                      exchange=args.exchange, e2e=True, clocks=True)
+                      exchange=args.exchange, e2e=not args.no_e2e, clocks=True)
     if wl.ns_iters > 0:
         roofline = ns_roofline(wl, r["phases_ms"]["newton_schulz"], r["ms_total"], pk, args.steps)
     else:
@@ -609,7 +609,7 @@ def run_gpu(args, wl):
     result = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-              "config": line_config(wl, args, world), "roofline": roofline, "e2e": r["e2e"],
+              "config": line_config(wl, args, world), "roofline": roofline, "e2e": r.get("e2e"),
               "phases_ms": r["phases_ms"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"]}
     if args.exchange:
         result["config"]["vote_workers"] = world * wl.n_workers
@@ -739,6 +739,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg with host buffers (profiling runs only: the line then has no e2e)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the vote-sweep, Signum and spectral rows measured beside the default workload")
     ap.add_argument("--norm", default="frobenius", choices=["frobenius", "spectral"],
