@@ -288,7 +288,8 @@ def test_momentum_zero_gradient_gives_zero_x():
 # ---------------------------------------------------------------------------
 NS_CASES = [([(256, 256)], 4, 1), ([(128, 384), (384, 128)], 2, 2), ([(100, 300), (300, 100)], 2, 5),
             ([(64, 147), (147, 64)], 3, 1), ([(768, 2304)], 1, 5), ([(3072, 768)], 1, 5),
-            ([(1, 1), (1, 40), (40, 1)], 2, 3), ([(513, 513)], 1, 2), ([(2048, 1000)], 1, 1)]
+            ([(1, 1), (1, 40), (40, 1)], 2, 3), ([(513, 513)], 1, 2), ([(2048, 1000)], 1, 1),
+            ([(768, 768), (768, 3072)], 1, 5), ([(512, 4608), (2048, 512), (256, 2304)], 1, 1)]
 
 
 @pytest.mark.parametrize("shapes,M,k", NS_CASES)
