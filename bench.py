@@ -611,6 +611,8 @@ def run_gpu(args, wl):
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
               "config": line_config(wl, args, world), "roofline": roofline, "e2e": r.get("e2e"),
               "phases_ms": r["phases_ms"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"]}
+    if "spectral_ms" in r:
+        result["phases_ms"]["spectral_alone"] = r["spectral_ms"]
     if args.exchange:
         result["config"]["vote_workers"] = world * wl.n_workers
         result["config"]["exchange_bytes_per_step"] = r["exchange_bytes_per_step"]
