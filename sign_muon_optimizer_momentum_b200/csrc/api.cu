@@ -2,6 +2,7 @@
 // planning (tensor maps, unit tables) and kernel launches.  The declarations
 // and their contracts are in include/signmuon.h.
 #include <algorithm>
+#include <climits>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -371,7 +372,9 @@ struct NsPlanHeader {
 struct NsPlanWave {
   int32_t u0, nu;
   int32_t total[3], pair[3];
-  int64_t rec0[3];  // first tile record of each stage (index into the record table)
+  int64_t rec0[3];   // first tile record of each stage (index into the record table)
+  int32_t long_k[3];  // CTA-pair stage whose every tile has K >= kLongK
+  int32_t pad_;
 };
 constexpr uint64_t kNsPlanMagic = 0x314e4c50534e4d53ull;  // "SMNSPLN1"
 constexpr size_t kNsPlanHeaderBytes = (sizeof(NsPlanHeader) + 63) / 64 * 64;
@@ -495,6 +498,14 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
       int pair = pair_area <= 1.15 * single_area ? 1 : 0;
       if (forced_mode >= 0) pair = forced_mode;
       W.pair[stg] = pair;
+      // The reduction length of a unit's tiles: the long side for the Gram
+      // product, the short side for the other two.
+      int min_k = INT32_MAX;
+      for (int ui = W.u0; ui < W.u0 + W.nu; ++ui) {
+        const int kr = stg == kStageGram ? std::max(hu[ui].rows, hu[ui].cols) : std::min(hu[ui].rows, hu[ui].cols);
+        min_k = std::min(min_k, kr);
+      }
+      W.long_k[stg] = pair && min_k >= kLongK ? 1 : 0;
       int pre = 0;
       W.rec0[stg] = (int64_t)recs.size();
       for (int ui = W.u0; ui < W.u0 + W.nu; ++ui) {
@@ -587,6 +598,7 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
         L.recs = d_recs + W.rec0[stg];
         L.total_tiles = W.total[stg];
         L.pair = W.pair[stg];
+        L.long_k = W.long_k[stg];
         L.out_kind = (stg == kStageApply && it == k - 1) ? hdr->out_mode : (int)kOutIterate;
         e = launch_ns_gemm(L, s);
         if (e != cudaSuccess) return cuda_status(e);

@@ -126,8 +126,11 @@ struct NsLaunch {
   // Fault injection for testing the bounded waits: the producer arms no
   // barrier and issues no copy, so the consumers' waits run out.
   int withhold_loads;
-  int pad_;
+  int long_k;       // CTA pairs, every tile K >= kLongK: 7-stage layout, direct stores
 };
+
+// Reduction length from which a CTA-pair launch uses the long layout.
+constexpr int kLongK = 2048;
 
 // Momentum units.
 struct MomUnit {

@@ -221,6 +221,15 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Pair mode: one commit arrives on the barrier at the same shared-memory
+// offset in both CTAs of the cluster (CTA mask 0b11).
+__device__ __forceinline__ void tc_commit_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
 template <bool kPair>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   if constexpr (kPair)
@@ -326,17 +335,24 @@ __device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn, int tile_m, b
          ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(tile_m >> 4) << 24);
 }
 
-// Per-mode tile and pipeline shape.
-template <bool kPair>
+// Per-mode tile and pipeline shape.  kLong (CTA pairs only): launches whose
+// every tile has a long reduction (K >= kLongK) store their 16-bit outputs
+// straight from registers and give the epilogue's staging memory to a
+// seventh pipeline stage.  The mainloop of such tiles is long enough to hide
+// the slower stores, and the extra stage covers more of the refill latency
+// (the MMA issuer's wait for a stage that has to come back from L2).
+template <bool kPair, bool kLong = false>
 struct GemmCfg {
+  static_assert(kPair || !kLong, "the long-reduction layout is a CTA-pair layout");
   static constexpr int kTileM = kPair ? 256 : 128;  // output rows per tile
   static constexpr int kRowsA = 128;                // A-operand rows held by one CTA
   static constexpr int kRowsB = kPair ? 128 : 256;  // B-operand rows held by one CTA
   static constexpr int kStageA = kRowsA * kBK * 2;
   static constexpr int kStageB = kRowsB * kBK * 2;
   static constexpr int kStageBytes = kStageA + kStageB;  // 32 KB or 48 KB
-  static constexpr int kStages = kPair ? 6 : 4;
-  static constexpr int kSmem = kStages * kStageBytes + kStagingBytes + kBarrierBytes + 1024 /*align*/;
+  static constexpr int kStages = kPair ? (kLong ? 7 : 6) : 4;
+  static constexpr int kStaging = kLong ? 0 : kStagingBytes;
+  static constexpr int kSmem = kStages * kStageBytes + kStaging + kBarrierBytes + 1024 /*align*/;
   static_assert(kSmem <= 232448, "shared memory per CTA");
   static_assert((2 * kStages + 5) * 8 + 8 <= kBarrierBytes, "barrier area");
 };
@@ -449,14 +465,14 @@ __device__ __forceinline__ void operand_maps(const NsLaunch& L, const NsUnit* u,
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <bool kPair>
+template <bool kPair, bool kLong>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ NsLaunch L) {
-  using C = GemmCfg<kPair>;
+  using C = GemmCfg<kPair, kLong>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Stage buffers must be 1 KB aligned for the 128-byte swizzle atoms.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // Layout: stage ring | epilogue staging (1 KB aligned) | barriers.
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + kStagingBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kStaging);
   uint64_t* full_bar = bars;                          // [kStages]
   uint64_t* empty_bar = bars + C::kStages;            // [kStages]
   uint64_t* tfull_bar = bars + 2 * C::kStages;        // [2]
@@ -611,14 +627,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                           (kb | kk) != 0);
           }
           // The stage is free (in both CTAs of a pair) once these MMAs finish.
-          tc_commit<kPair>(smem_addr(&empty_bar[stage]));
-          if constexpr (kPair) tc_commit<kPair>(map_to_rank(smem_addr(&empty_bar[stage]), 1));
+          if constexpr (kPair) tc_commit_both(smem_addr(&empty_bar[stage]));
+          else tc_commit<kPair>(smem_addr(&empty_bar[stage]));
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         // Accumulator ready for the epilogue (of both CTAs of a pair).
-        tc_commit<kPair>(smem_addr(&tfull_bar[acc]));
-        if constexpr (kPair) tc_commit<kPair>(map_to_rank(smem_addr(&tfull_bar[acc]), 1));
+        if constexpr (kPair) tc_commit_both(smem_addr(&tfull_bar[acc]));
+        else tc_commit<kPair>(smem_addr(&tfull_bar[acc]));
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
       // Drain: wait until every MMA this thread issued has completed.
@@ -662,7 +678,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       const CUtensorMap* st_p;    // Gram stage: store map of P = bI + cA
       void* out;
       int cols;
-    } uf = {nullptr, nullptr, nullptr, 0};
+      uint8_t* o16;               // long layout: this stage's 16-bit output
+      uint8_t* p16;               //   the Gram stage's P
+      int ld;                     //   and their row stride (elements)
+    } uf = {nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0};
     float s = 1.f;
     for (int t = first_tile; t < L.total_tiles; t += tile_stride) {
       const NsTileRec rec = rs.advance(L, t, tile_stride);
@@ -674,6 +693,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                   : (L.parity ? &un->st_x : &un->st_xalt);
         uf.st_p = &un->st_p;
         uf.out = un->out;
+        if constexpr (kLong) {
+          uf.o16 = static_cast<uint8_t*>(L.stage == kStageGram     ? un->a
+                                         : L.stage == kStageSquare ? static_cast<void*>(un->b)
+                                         : static_cast<void*>(L.parity ? un->x : un->xalt));
+          uf.p16 = static_cast<uint8_t*>(un->p);
+          uf.ld = L.stage == kStageApply ? un->ld_x : un->ld_s;
+        }
         uf.cols = rec.cols;
         s = L.first ? __ldg(L.scales + rec.unit) : 1.f;
       }
@@ -731,6 +757,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             if (o == 1) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = fmaf(L.c, v[j], (gc0 + j == grow) ? L.b : 0.f);
+            }
+            if constexpr (kLong) {
+              // Straight from registers: each lane writes its row's 32
+              // columns (64 bytes) as four 16-byte stores, those starting
+              // inside the matrix (the row stride is a multiple of 8, so a
+              // store never crosses into the next row).
+              if (row_ok) {
+                uint4* dst = reinterpret_cast<uint4*>((o == 0 ? uf.o16 : uf.p16) +
+                                                      ((int64_t)grow * uf.ld + gc0) * 2);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  uint32_t w[4];
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
+                  if (8 * k < nvalid) dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+              }
+              continue;
             }
             const CUtensorMap* map = o == 0 ? uf.st_out : uf.st_p;
             // Stores alternate between the two staging blocks, so only the
@@ -907,18 +951,21 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
     int n = 0;
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ns_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<false>::kSmem);
+    e = cudaFuncSetAttribute(ns_gemm_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<false, false>::kSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ns_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<true>::kSmem);
+    e = cudaFuncSetAttribute(ns_gemm_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<true, false>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(ns_gemm_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<true, true>::kSmem);
     if (e != cudaSuccess) return e;
     g_num_sms[dev] = n;
   }
   const int sms = g_num_sms[dev];
   if (!p.pair) {
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-    ns_gemm_kernel<false><<<grid, kGemmThreads, GemmCfg<false>::kSmem, stream>>>(p);
+    ns_gemm_kernel<false, false><<<grid, kGemmThreads, GemmCfg<false, false>::kSmem, stream>>>(p);
     return cudaGetLastError();
   }
   // One cluster of two CTAs per pair tile worker.
@@ -926,7 +973,7 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = GemmCfg<true>::kSmem;
+  cfg.dynamicSmemBytes = p.long_k ? GemmCfg<true, true>::kSmem : GemmCfg<true, false>::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -935,7 +982,8 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true>, p);
+  if (p.long_k) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true, true>, p);
+  return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true, false>, p);
 }
 
 }  // namespace signmuon
