@@ -78,11 +78,12 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-# The sources of each kernel; a captured traffic figure is used only while
+# The sources of each kernel (for the Newton-Schulz kernel also the plan,
+# which fixes its tile order); a captured traffic figure is used only while
 # they are unchanged.
 _CSRC = "sign_muon_optimizer_momentum_b200/csrc/"
 KERNEL_SOURCES = {
-    "ns_gemm_kernel": (_CSRC + "ns_gemm.cu", _CSRC + "common.cuh"),
+    "ns_gemm_kernel": (_CSRC + "ns_gemm.cu", _CSRC + "common.cuh", _CSRC + "api.cu"),
     "momentum_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
     "vote_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
     "spectral_rowpass_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),

@@ -512,8 +512,22 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
         hu[ui].tile_begin[stg] = pre;
         hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg, pair);
         pre += hu[ui].tile_count[stg];
-        for (int li = 0; li < hu[ui].tile_count[stg]; ++li)
-          recs.push_back(NsTileRec{ui - W.u0, li, hu[ui].rows, hu[ui].cols});
+        if (stg == kStageApply && hu[ui].rows <= hu[ui].cols) {
+          // Apply of a wide unit (X' = B'X): X is the B operand, so the tiles
+          // go column by column -- consecutive tiles (running at the same
+          // time on neighbouring CTA pairs) share one column block of X,
+          // which is read from DRAM once instead of once per row of tiles.
+          // (A tall unit's X is the A operand: row by row, the tile_of
+          // numbering, already keeps its row blocks together.)
+          const int bm = ns_tile_m(pair);
+          const int tiles_m = (hu[ui].rows + bm - 1) / bm, tiles_n = (hu[ui].cols + kBN - 1) / kBN;
+          for (int tn = 0; tn < tiles_n; ++tn)
+            for (int tm = 0; tm < tiles_m; ++tm)
+              recs.push_back(NsTileRec{ui - W.u0, tm * tiles_n + tn, hu[ui].rows, hu[ui].cols});
+        } else {
+          for (int li = 0; li < hu[ui].tile_count[stg]; ++li)
+            recs.push_back(NsTileRec{ui - W.u0, li, hu[ui].rows, hu[ui].cols});
+        }
       }
       W.total[stg] = pre;
       // Launch order.  With few tiles per CTA (pair) the round-robin

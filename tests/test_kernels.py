@@ -923,6 +923,35 @@ def test_square4096_batch_full_size_sampled():
     assert np.array_equal(f64(weights[3]), O.apply_update(f64(w_before), wl.eta, u_gpu, "bf16"))
 
 
+@pytest.mark.parametrize("shapes,M,k", [([(2056, 2100)], 1, 2), ([(300, 2100), (2100, 300)], 2, 1)])
+def test_long_reduction_layout_ragged_edges(shapes, M, k, monkeypatch):
+    """Launches whose every tile has a reduction of 2048 or more use the
+    seven-stage layout that stores its 16-bit outputs from registers.  Ragged
+    sizes (2056 x 2100: all three products long; 300 x 2100 and its
+    transpose: the Gram product long) put row and column edges inside tiles
+    and inside 32-column chunks: U within the Newton-Schulz tolerance of the
+    oracle, and packed signs equal to the signs of that U."""
+    monkeypatch.setenv("SIGNMUON_NS_TILE_MODE", "pair")
+    grads, moms = seeded_state(shapes, M, 23)
+    us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(grads))]
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], 0.9,
+                           torch.float32)
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, us)
+    packed = [torch.zeros(L.signmuon_packed_words(shapes[u // M]), dtype=torch.int32, device="cuda")
+              for u in range(len(grads))]
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], 0.9,
+                           torch.float32)
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_PACK1, packed)
+    for u in range(len(grads)):
+        r, c = shapes[u // M]
+        _, ref = oracle_u(moms[u], grads[u], 0.9, k)
+        got = f64(us[u])
+        assert rel_fro(got, ref) <= NS_TOL, shapes[u // M]
+        big = np.abs(ref) > 1e-3
+        assert np.mean((got[big] < 0) == (ref[big] < 0)) >= SIGN_AGREE
+        assert np.array_equal(unpack_words(packed[u].cpu().numpy().view(np.uint32), r, c), O.sign_entries(got))
+
+
 @pytest.mark.slow
 def test_square4096_two_units_ns_over_waves(monkeypatch):
     """Newton-Schulz at s = 4096 (K = 4096 mainloops, 16 x 16 upper-block
