@@ -26,7 +26,10 @@
 //           SM streams a third less operand data per FLOP and keeps more
 //           k-blocks in flight.  Each CTA loads its own halves (no TMA
 //           multicast); the odd CTA's copies complete on the even CTA's
-//           barrier.
+//           barrier, and one multicast commit frees a stage in both CTAs.
+//           Launches whose every reduction is at least kLongK long use a
+//           seventh stage instead of the epilogue's staging memory and store
+//           their 16-bit outputs from registers (the long-reduction layout).
 // Roles (320 threads per CTA):
 //   warp 0     TMA producer: 64x64 bf16 boxes, 128-byte swizzle
 //   warp 1     MMA issuer (even CTA of a pair): kind::f16, N=256, K=16,
@@ -656,7 +659,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     // column half (w-2)/4 of the accumulator.  bf16 outputs (A, B', the next
     // X) are staged per 32x32 block in shared memory and written by TMA
     // stores (whole lines; rows/columns outside the matrix are dropped by the
-    // TMA); the other outputs are stored directly.
+    // TMA) -- in the long-reduction layout they are stored from registers;
+    // the other outputs are stored directly.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     constexpr int kChunks = kBN / 32 / 2;  // 32-column chunks per warp
