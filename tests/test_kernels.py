@@ -469,6 +469,42 @@ def test_polar_step_update(w_dtype):
         assert np.array_equal(f64(w[i]), O.apply_update(f64(w0[i]), eta, f64(u_gpu[i]), wd)), shapes[i]
 
 
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
+def test_polar_step_all_ties_leaves_weights_bit_identical(w_dtype):
+    """Two workers with opposite signs everywhere: every vote ties, nnz = 0,
+    1/sqrt(nnz) is taken as 0, the polar step's U is 0 and W stays bit for
+    bit (signed zeros included), as the oracle's zero vote does."""
+    shapes, eta = [(256, 384), (72, 300)], 0.02
+    flat, w0 = [], []
+    for i, (r, c) in enumerate(shapes):
+        pos = torch.ones((r, c), dtype=torch.int8)
+        flat += _packed_device([pos, -pos], (r, c))
+        w = syn.gaussian((r, c), 0.02, "cpu", "tiew", i, dtype=w_dtype)
+        w[0, :8] = 0.0
+        w[0, 8:16] = -0.0
+        w0.append(w)
+    votes = [torch.full((r, L.signmuon_x_ld(c)), 3.0, dtype=torch.bfloat16, device="cuda") for r, c in shapes]
+    nnz = torch.full((len(shapes),), -1, dtype=torch.int64, device="cuda")
+    inv = torch.full((len(shapes),), 5.0, dtype=torch.float32, device="cuda")
+    wk = ws(L.signmuon_vote_workspace_bytes(shapes, 2))
+    L.signmuon_vote_update(shapes, 2, False, [x.data_ptr() for x in flat], L.SIGNMUON_F32, None, eta,
+                           [v.data_ptr() for v in votes], nnz.data_ptr(), inv.data_ptr(), wk.data_ptr(), wk.numel(),
+                           stream())
+    torch.cuda.synchronize()
+    assert nnz.tolist() == [0, 0] and inv.tolist() == [0.0, 0.0]
+    for v, (r, c) in zip(votes, shapes):
+        assert bool((v[:, :c] == 0).all())
+    w = [t.cuda() for t in w0]
+    code = L.SIGNMUON_BF16 if w_dtype == torch.bfloat16 else L.SIGNMUON_F32
+    gpu_ns(shapes, 1, votes, inv, 1, L.SIGNMUON_OUT_UPDATE_W, None, code, w, eta)
+    ibits = torch.int16 if w_dtype == torch.bfloat16 else torch.int32
+    wd = "bf16" if w_dtype == torch.bfloat16 else "f32"
+    for a, b in zip(w, w0):
+        assert torch.equal(a.cpu().view(ibits), b.view(ibits))
+        ref = O.apply_update(f64(b), eta, O.polar_direction(np.zeros(b.shape), 1), wd)
+        assert np.array_equal(f64(a), ref)
+
+
 def gpu_polar_u(shapes, votes, inv):
     """U of the local polar step (one iteration on the voted matrices), as
     fp32, through the same Newton-Schulz call with the U output."""
