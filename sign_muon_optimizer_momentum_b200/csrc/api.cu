@@ -104,19 +104,20 @@ UnitBytes ns_unit_bytes(signmuon_shape sh) {
   return u;
 }
 
-// Tiles of one unit in one stage; pair = 1 for 256x256 CTA-pair tiles.
-int ns_tiles(int rows, int cols, int stage, int pair) {
+// Tiles of one unit in one stage; pair = 1 for 256x256 CTA-pair tiles,
+// wide = 1 (pairs only) for 256x512 ones.
+int ns_tiles(int rows, int cols, int stage, int pair, int wide = 0) {
   const bool tall = rows > cols;
   const int s = tall ? cols : rows;
   const int bm = ns_tile_m(pair);
+  const int bn = wide ? 2 * kBN : kBN;
   if (stage == kStageApply) {
-    return ((rows + bm - 1) / bm) * ((cols + kBN - 1) / kBN);
+    return ((rows + bm - 1) / bm) * ((cols + bn - 1) / bn);
   }
-  // Symmetric outputs: row tile tm starts at column tile tm * bm / 256.
-  const int tm = (s + bm - 1) / bm, tn = (s + kBN - 1) / kBN;
-  const int sh = pair ? 0 : 1;
+  // Symmetric outputs: row tile i starts at the column tile holding column i * bm.
+  const int tm = (s + bm - 1) / bm, tn = (s + bn - 1) / bn;
   int n = 0;
-  for (int i = 0; i < tm; ++i) n += tn - (i >> sh);
+  for (int i = 0; i < tm; ++i) n += tn - i * bm / bn;
   return n;
 }
 
@@ -374,7 +375,7 @@ struct NsPlanWave {
   int32_t total[3], pair[3];
   int64_t rec0[3];   // first tile record of each stage (index into the record table)
   int32_t long_k[3];  // CTA-pair stage whose every tile has K >= kLongK
-  int32_t pad_;
+  int32_t wide[3];    //   and which runs 256x512 tiles
 };
 constexpr uint64_t kNsPlanMagic = 0x314e4c50534e4d53ull;  // "SMNSPLN1"
 constexpr size_t kNsPlanHeaderBytes = (sizeof(NsPlanHeader) + 63) / 64 * 64;
@@ -477,6 +478,10 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
     if (!strcmp(m, "single")) forced_mode = 0;
     else if (!strcmp(m, "pair")) forced_mode = 1;
   }
+  // SIGNMUON_NS_WIDE=0 keeps the long-reduction launches on 256x256 tiles
+  // (the tests compare both layouts on the same inputs).
+  bool wide_ok = true;
+  if (const char* m = getenv("SIGNMUON_NS_WIDE")) wide_ok = strcmp(m, "0") != 0;
   // Per wave and stage, pick the tile mode with the least padded work (the
   // CTA-pair mode is preferred unless it pads more than 15 % extra), then
   // number the tiles; prefixes restart at each wave (a launch covers one
@@ -506,11 +511,13 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
         min_k = std::min(min_k, kr);
       }
       W.long_k[stg] = pair && min_k >= kLongK ? 1 : 0;
+      W.wide[stg] = W.long_k[stg] && wide_ok ? 1 : 0;
+      const int wide = W.wide[stg];
       int pre = 0;
       W.rec0[stg] = (int64_t)recs.size();
       for (int ui = W.u0; ui < W.u0 + W.nu; ++ui) {
         hu[ui].tile_begin[stg] = pre;
-        hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg, pair);
+        hu[ui].tile_count[stg] = ns_tiles(hu[ui].rows, hu[ui].cols, stg, pair, wide);
         pre += hu[ui].tile_count[stg];
         if (stg == kStageApply && hu[ui].rows <= hu[ui].cols) {
           // Apply of a wide unit (X' = B'X): X is the B operand, so the tiles
@@ -519,8 +526,8 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
           // which is read from DRAM once instead of once per row of tiles.
           // (A tall unit's X is the A operand: row by row, the tile_of
           // numbering, already keeps its row blocks together.)
-          const int bm = ns_tile_m(pair);
-          const int tiles_m = (hu[ui].rows + bm - 1) / bm, tiles_n = (hu[ui].cols + kBN - 1) / kBN;
+          const int bm = ns_tile_m(pair), bn = wide ? 2 * kBN : kBN;
+          const int tiles_m = (hu[ui].rows + bm - 1) / bm, tiles_n = (hu[ui].cols + bn - 1) / bn;
           for (int tn = 0; tn < tiles_n; ++tn)
             for (int tm = 0; tm < tiles_m; ++tm)
               recs.push_back(NsTileRec{ui - W.u0, tm * tiles_n + tn, hu[ui].rows, hu[ui].cols});
@@ -613,6 +620,7 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
         L.total_tiles = W.total[stg];
         L.pair = W.pair[stg];
         L.long_k = W.long_k[stg];
+        L.wide = W.wide[stg];
         L.out_kind = (stg == kStageApply && it == k - 1) ? hdr->out_mode : (int)kOutIterate;
         e = launch_ns_gemm(L, s);
         if (e != cudaSuccess) return cuda_status(e);

@@ -126,7 +126,8 @@ struct NsLaunch {
   // Fault injection for testing the bounded waits: the producer arms no
   // barrier and issues no copy, so the consumers' waits run out.
   int withhold_loads;
-  int long_k;       // CTA pairs, every tile K >= kLongK: 7-stage layout, direct stores
+  int long_k;       // CTA pairs, every tile K >= kLongK: direct stores, no staging
+  int wide;         // with long_k: 256x512 tiles, two N = 256 halves of one accumulator
 };
 
 // Reduction length from which a CTA-pair launch uses the long layout.

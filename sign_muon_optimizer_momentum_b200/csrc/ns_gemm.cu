@@ -344,16 +344,27 @@ __device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn, int tile_m, b
 // seventh pipeline stage.  The mainloop of such tiles is long enough to hide
 // the slower stores, and the extra stage covers more of the refill latency
 // (the MMA issuer's wait for a stage that has to come back from L2).
-template <bool kPair, bool kLong = false>
+//
+// kWide (long layout only): a pair tile is 256 x 512, two N = 256 MMAs per
+// K step into the two 256-column halves of TMEM, so the accumulator is no
+// longer double-buffered: the halves take the place of the two buffers.  Each
+// SM then streams 48 KB per 1024 MMA cycles instead of 32 KB per 512 (a
+// quarter less operand traffic per FLOP), in four 48 KB stages.
+template <bool kPair, bool kLong = false, bool kWide = false>
 struct GemmCfg {
   static_assert(kPair || !kLong, "the long-reduction layout is a CTA-pair layout");
+  static_assert(kLong || !kWide, "the 256x512 tile is a long-reduction layout");
   static constexpr int kTileM = kPair ? 256 : 128;  // output rows per tile
+  static constexpr int kHalves = kWide ? 2 : 1;     // N = 256 accumulators per tile
+  static constexpr int kTileN = kHalves * kBN;      // output columns per tile
   static constexpr int kRowsA = 128;                // A-operand rows held by one CTA
-  static constexpr int kRowsB = kPair ? 128 : 256;  // B-operand rows held by one CTA
+  static constexpr int kRowsBH = kPair ? 128 : 256; // B-operand rows per half held by one CTA
+  static constexpr int kRowsB = kHalves * kRowsBH;
   static constexpr int kStageA = kRowsA * kBK * 2;
+  static constexpr int kStageBH = kRowsBH * kBK * 2;
   static constexpr int kStageB = kRowsB * kBK * 2;
   static constexpr int kStageBytes = kStageA + kStageB;  // 32 KB or 48 KB
-  static constexpr int kStages = kPair ? (kLong ? 7 : 6) : 4;
+  static constexpr int kStages = kPair ? (kWide ? 4 : kLong ? 7 : 6) : 4;
   static constexpr int kStaging = kLong ? 0 : kStagingBytes;
   static constexpr int kSmem = kStages * kStageBytes + kStaging + kBarrierBytes + 1024 /*align*/;
   static_assert(kSmem <= 232448, "shared memory per CTA");
@@ -401,13 +412,13 @@ struct Tile {
 __device__ __forceinline__ int a_major(const Tile& T, int k0) {
   return T.a_mn | (T.a_up & (int)((k0 >> 8) < (T.m0 >> 8)));
 }
-__device__ __forceinline__ int b_major(const Tile& T, int k0) {
-  return T.b_mn | (T.b_up & (int)((k0 >> 8) < (T.n0 >> 8)));
+__device__ __forceinline__ int b_major(const Tile& T, int k0, int n0) {
+  return T.b_mn | (T.b_up & (int)((k0 >> 8) < (n0 >> 8)));
 }
 
 // Problem dimensions, operand majors and tile origin of local tile li of a
 // unit with the given shape.
-__device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, int tile_m) {
+__device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, int tile_m, int tile_n) {
   const bool tall = rows > cols;
   const int s = tall ? cols : rows, l = tall ? rows : cols;
   Tile T;
@@ -421,15 +432,16 @@ __device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, i
   } else {             // X' = X B': A-op = X (K-major), B-op = B' (symmetric, K-major)
     T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 0; T.b_up = 1;
   }
-  const int tiles_n = (T.N + kBN - 1) / kBN;
+  const int tiles_n = (T.N + tile_n - 1) / tile_n;
   int tm = 0, tn = 0;
   if (T.sym) {
     // Only the upper 256-blocks of a symmetric output are computed (and
-    // stored): row tile tm starts at column tile tm * tile_m / 256.
-    const int sh = tile_m == 256 ? 0 : 1;
+    // stored): row tile tm starts at the column tile holding column
+    // tm * tile_m.
     while (true) {
-      const int cnt = tiles_n - (tm >> sh);
-      if (li < cnt) { tn = (tm >> sh) + li; break; }
+      const int first = tm * tile_m / tile_n;
+      const int cnt = tiles_n - first;
+      if (li < cnt) { tn = first + li; break; }
       li -= cnt;
       ++tm;
     }
@@ -438,16 +450,26 @@ __device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, i
     tn = li - tm * tiles_n;
   }
   T.m0 = tm * tile_m;
-  T.n0 = tn * kBN;
+  T.n0 = tn * tile_n;
   return T;
 }
 
-// Pair mode, Gram stage, diagonal tile: each CTA's B rows (n0 + 128 rank ..)
-// are its A rows (m0 + 128 rank ..) of the same operand, so B is read from
-// the A buffer and not loaded.
+// Whether the N = 256 half h of a tile (columns n0 + 256 h ..) is computed:
+// it starts inside the matrix and, for a symmetric output, on or above the
+// diagonal block (the tile's rows lie in one 256-block).  Half 0 of every
+// 256-column tile is.
+__device__ __forceinline__ bool half_ok(const Tile& T, int h) {
+  const int n0 = T.n0 + h * kBN;
+  return n0 < T.N && (!T.sym || n0 >= (T.m0 & ~255));
+}
+
+// Pair mode, Gram stage, diagonal block: each CTA's B rows of the half
+// starting at column n0 (n0 + 128 rank ..) are its A rows (m0 + 128 rank ..)
+// of the same operand, so that half of B is read from the A buffer and not
+// loaded.
 template <bool kPair>
-__device__ __forceinline__ bool diag_b_from_a(const NsLaunch& L, const Tile& T) {
-  return kPair && L.stage == kStageGram && T.m0 == T.n0;
+__device__ __forceinline__ bool diag_b_from_a(const NsLaunch& L, const Tile& T, int n0) {
+  return kPair && L.stage == kStageGram && T.m0 == n0;
 }
 
 // Tensor maps of the two operands of a unit's tile.
@@ -468,9 +490,9 @@ __device__ __forceinline__ void operand_maps(const NsLaunch& L, const NsUnit* u,
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <bool kPair, bool kLong>
+template <bool kPair, bool kLong, bool kWide>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ NsLaunch L) {
-  using C = GemmCfg<kPair, kLong>;
+  using C = GemmCfg<kPair, kLong, kWide>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Stage buffers must be 1 KB aligned for the 128-byte swizzle atoms.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -533,11 +555,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           tensormap_acquire(ma);
           tensormap_acquire(mb);
         }
-        const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
+        const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM, C::kTileN);
         const int nkb = (T.K + kBK - 1) / kBK;
         const int a_row0 = T.m0 + (int)rank * C::kRowsA;
-        const int b_row0 = T.n0 + (int)rank * C::kRowsB;
-        const bool b_from_a = diag_b_from_a<kPair>(L, T);
+        // B halves to load: computed, and not read from the A buffer.
+        bool load_b[C::kHalves];
+        int stage_bytes = C::kStageA;
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h) {
+          load_b[h] = half_ok(T, h) && !diag_b_from_a<kPair>(L, T, T.n0 + h * kBN);
+          if (load_b[h]) stage_bytes += C::kStageBH;
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(smem_addr(&empty_bar[stage]), phase ^ 1, abort_flag, L.wait_limit_ns)) {
             atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutProducer);
@@ -554,16 +582,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           }
           const uint32_t own_full = smem_addr(&full_bar[stage]);
           // Pair mode: both CTAs' copies complete on the even CTA's barrier,
-          // which the even CTA arms for both.  On a diagonal tile of a
+          // which the even CTA arms for both.  On a diagonal block of a
           // symmetric product each CTA's B half is its A half (the same rows
-          // of the same matrix), so only A is loaded.
-          const int stage_bytes = b_from_a ? C::kStageA : C::kStageBytes;
+          // of the same matrix), so that B half is not loaded; nor is a half
+          // that is not computed.
           if (rank == 0) mbar_arrive_expect_tx(own_full, (kPair ? 2 : 1) * stage_bytes);
           const uint32_t fb = kPair ? map_to_rank(own_full, 0) : own_full;
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
-          const uint32_t sb = sa + C::kStageA;
           const int k0 = kb * kBK;
-          const int amn = a_major(T, k0), bmn = b_major(T, k0);
+          const int amn = a_major(T, k0);
 #pragma unroll
           for (int j = 0; j < C::kRowsA / kBoxRows; ++j) {
             const int mn = a_row0 + j * kBoxRows;
@@ -573,13 +600,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
               tma_load_2d(sa + j * kBoxBytes, ma, fb, amn ? mn : k0, amn ? k0 : mn);
           }
 #pragma unroll
-          for (int j = 0; j < C::kRowsB / kBoxRows; ++j) {
-            if (b_from_a) break;
-            const int mn = b_row0 + j * kBoxRows;
-            if constexpr (kPair)
-              tma_load_2d_pair(sb + j * kBoxBytes, mb, fb, bmn ? mn : k0, bmn ? k0 : mn);
-            else
-              tma_load_2d(sb + j * kBoxBytes, mb, fb, bmn ? mn : k0, bmn ? k0 : mn);
+          for (int h = 0; h < C::kHalves; ++h) {
+            if (!load_b[h]) continue;
+            const int n0 = T.n0 + h * kBN;
+            const int b_row0 = n0 + (int)rank * C::kRowsBH;
+            const int bmn = b_major(T, k0, n0);
+            const uint32_t sb = sa + C::kStageA + h * C::kStageBH;
+#pragma unroll
+            for (int j = 0; j < C::kRowsBH / kBoxRows; ++j) {
+              const int mn = b_row0 + j * kBoxRows;
+              if constexpr (kPair)
+                tma_load_2d_pair(sb + j * kBoxBytes, mb, fb, bmn ? mn : k0, bmn ? k0 : mn);
+              else
+                tma_load_2d(sb + j * kBoxBytes, mb, fb, bmn ? mn : k0, bmn ? k0 : mn);
+            }
           }
           ++issued_kb;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -598,11 +632,95 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       rs.start(L, first_tile);
       for (int t = first_tile; t < L.total_tiles && ok; t += tile_stride) {
         const NsTileRec rec = rs.advance(L, t, tile_stride);
-        const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
+        const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM, C::kTileN);
         // The square stage multiplies the fp16 A and P; all others are bf16.
         const bool fp16_ops = L.stage == kStageSquare;
-        const bool b_from_a = diag_b_from_a<kPair>(L, T);
         const int nkb = (T.K + kBK - 1) / kBK;
+        if constexpr (kWide) {
+          // 256x512 tile: accumulator half h (TMEM columns 256 h ..) takes
+          // the barriers of buffer h.  So that draining one half overlaps
+          // MMAs into the other, the first (and last) kStages k-blocks issue
+          // their half-0 MMAs ahead of their half-1 MMAs: the tile starts as
+          // soon as half 0 of the previous tile has been read out, and half 0
+          // of this tile is handed to the epilogue while the half-1 MMAs of
+          // its last k-blocks still run.  A stage is released once both of
+          // its halves' MMAs are issued.
+          bool hok[2], bfa[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            hok[h] = half_ok(T, h);
+            bfa[h] = diag_b_from_a<kPair>(L, T, T.n0 + h * kBN);
+          }
+          const int s0 = stage;
+          const uint32_t ph0 = phase;
+          auto slot = [&](int i) { return (s0 + i) % C::kStages; };
+          auto wait_full = [&](int i) {
+            const int pos = s0 + i;
+            if (!mbar_wait(smem_addr(&full_bar[pos % C::kStages]), ph0 ^ (uint32_t)((pos / C::kStages) & 1),
+                           abort_flag, L.wait_limit_ns)) {
+              atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
+              *abort_flag = 1;
+              return false;
+            }
+            tc_fence_after();
+            return true;
+          };
+          auto wait_acc = [&](int h) {
+            if (!mbar_wait(smem_addr(&tempty_bar[h]), acc_phase ^ 1, abort_flag, L.wait_limit_ns)) {
+              atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
+              *abort_flag = 1;
+              return false;
+            }
+            tc_fence_after();
+            return true;
+          };
+          auto issue = [&](int i, int h) {
+            if (!hok[h]) return;
+            const uint32_t sa = smem_addr(smem + slot(i) * C::kStageBytes);
+            const uint32_t sb = bfa[h] ? sa : sa + C::kStageA + h * C::kStageBH;
+            const int amn = a_major(T, i * kBK), bmn = b_major(T, i * kBK, T.n0 + h * kBN);
+            const uint32_t idesc = instr_desc(amn, bmn, C::kTileM, fp16_ops);
+            const uint32_t tmem_d = tmem_base + (uint32_t)(h * kAccCols);
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+              const uint32_t aoff = amn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
+              const uint32_t boff = bmn ? kk * (kUmmaK * 128) : kk * (kUmmaK * 2);
+              tc_mma<kPair>(tmem_d, smem_desc(sa + aoff, amn), smem_desc(sb + boff, bmn), idesc, (i | kk) != 0);
+            }
+          };
+          auto release = [&](int i) { tc_commit_both(smem_addr(&empty_bar[slot(i)])); };
+          const int P = min(C::kStages, nkb);
+          const int E = min(C::kStages, nkb - P);
+          ok = wait_acc(0);
+          for (int i = 0; ok && i < P; ++i)
+            if ((ok = wait_full(i))) issue(i, 0);
+          if (ok) ok = wait_acc(1);
+          for (int i = 0; ok && i < P; ++i) {
+            issue(i, 1);
+            release(i);
+          }
+          for (int i = P; ok && i < nkb - E; ++i) {
+            if (!(ok = wait_full(i))) break;
+            issue(i, 0);
+            issue(i, 1);
+            release(i);
+          }
+          for (int i = nkb - E; ok && i < nkb; ++i)
+            if ((ok = wait_full(i))) issue(i, 0);
+          if (!ok) break;
+          tc_commit_both(smem_addr(&tfull_bar[0]));
+          for (int i = nkb - E; i < nkb; ++i) {
+            issue(i, 1);
+            release(i);
+          }
+          tc_commit_both(smem_addr(&tfull_bar[1]));
+          const int pos = s0 + nkb;
+          stage = pos % C::kStages;
+          phase = ph0 ^ (uint32_t)((pos / C::kStages) & 1);
+          acc_phase ^= 1;
+          continue;
+        }
+        const bool b_from_a = diag_b_from_a<kPair>(L, T, T.n0);
         if (!mbar_wait(smem_addr(&tempty_bar[acc]), acc_phase ^ 1, abort_flag, L.wait_limit_ns)) {
           atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutMma);
           *abort_flag = 1;
@@ -620,7 +738,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           tc_fence_after();
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
           const uint32_t sb = b_from_a ? sa : sa + C::kStageA;
-          const int amn = a_major(T, kb * kBK), bmn = b_major(T, kb * kBK);
+          const int amn = a_major(T, kb * kBK), bmn = b_major(T, kb * kBK, T.n0);
           const uint32_t idesc = instr_desc(amn, bmn, C::kTileM, fp16_ops);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
@@ -707,205 +825,214 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         uf.cols = rec.cols;
         s = L.first ? __ldg(L.scales + rec.unit) : 1.f;
       }
-      const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM);
-      if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag, L.wait_limit_ns)) {
-        atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutEpilogue);
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const int grow0 = T.m0 + (int)rank * 128 + q * 32;  // first row of this warp's 32-row block
-      const int grow = grow0 + lane;
-      const bool row_ok = grow < T.M;
-      const bool bf16_out = T.sym || L.out_kind == kOutIterate;
-      // Chunks of this warp's column half that hold valid columns (warp-uniform).
-      const int n_ch = max(0, min(kChunks, (T.N - T.n0 - half * kChunks * 32 + 31) / 32));
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
-      uint32_t nxt[32];
-      if (n_ch > 0) tmem_ld32_async(tbase + (uint32_t)(half * kChunks * 32), nxt);
+      const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM, C::kTileN);
+      // A 256x512 tile is drained as its two 256-column halves, each with the
+      // barriers of accumulator buffer h (as two consecutive 256-column tiles).
+      bool ep_ok = true;
 #pragma unroll 1
-      for (int cc = 0; cc < n_ch; ++cc) {
-        const int ch = half * kChunks + cc;
-        const int gc0 = T.n0 + ch * 32;
-        tmem_wait_ld(nxt);
-        uint32_t raw[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) raw[j] = nxt[j];
-        // The next chunk's TMEM load overlaps this chunk's math and stores.
-        if (cc + 1 < n_ch) tmem_ld32_async(tbase + (uint32_t)((ch + 1) * 32), nxt);
-        const int nvalid = min(32, T.N - gc0);
-        float v[32];
-        if (L.stage == kStageGram) {
-          const float s2 = s * s;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) * s2;
-        } else if (L.stage == kStageSquare) {
-          // B' = a I + A P with P = b I + c A, i.e. a I + b A + c A^2.
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) + ((gc0 + j == grow) ? L.a : 0.f);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = s * __uint_as_float(raw[j]);
+      for (int h = 0; h < C::kHalves; ++h) {
+        const int n0 = T.n0 + h * kBN;
+        if (!mbar_wait(smem_addr(&tfull_bar[acc]), acc_phase, abort_flag, L.wait_limit_ns)) {
+          atomicCAS(L.err, 0u, (uint32_t)kErrWaitTimeoutEpilogue);
+          *abort_flag = 1;
+          ep_ok = false;
+          break;
         }
-        if (bf16_out) {
-          // Each 32x32 block is staged in shared memory and written by a TMA
-          // store.  The tiles of a symmetric output cover its upper
-          // 256-blocks only, which is all that is stored of it (its
-          // consumers read the other blocks transposed).  The Gram stage
-          // writes two outputs: A, then P = b I + c A (from the fp32 value
-          // of A).
-          const int n_out = (L.stage == kStageGram) ? 2 : 1;
-          // The Gram stage's A and P are fp16, everything else bf16.
-          const bool half_out = L.stage == kStageGram;
-          for (int o = 0; o < n_out; ++o) {
-            if (o == 1) {
+        tc_fence_after();
+        const int grow0 = T.m0 + (int)rank * 128 + q * 32;  // first row of this warp's 32-row block
+        const int grow = grow0 + lane;
+        const bool row_ok = grow < T.M;
+        const bool bf16_out = T.sym || L.out_kind == kOutIterate;
+        // Chunks of this warp's column half that hold valid columns (warp-uniform).
+        const int n_ch = half_ok(T, h) ? max(0, min(kChunks, (T.N - n0 - half * kChunks * 32 + 31) / 32)) : 0;
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
+        uint32_t nxt[32];
+        if (n_ch > 0) tmem_ld32_async(tbase + (uint32_t)(half * kChunks * 32), nxt);
+#pragma unroll 1
+        for (int cc = 0; cc < n_ch; ++cc) {
+          const int ch = half * kChunks + cc;
+          const int gc0 = n0 + ch * 32;
+          tmem_wait_ld(nxt);
+          uint32_t raw[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = fmaf(L.c, v[j], (gc0 + j == grow) ? L.b : 0.f);
-            }
-            if constexpr (kLong) {
-              // Straight from registers: each lane writes its row's 32
-              // columns (64 bytes) as four 16-byte stores, those starting
-              // inside the matrix (the row stride is a multiple of 8, so a
-              // store never crosses into the next row).
-              if (row_ok) {
-                uint4* dst = reinterpret_cast<uint4*>((o == 0 ? uf.o16 : uf.p16) +
-                                                      ((int64_t)grow * uf.ld + gc0) * 2);
+          for (int j = 0; j < 32; ++j) raw[j] = nxt[j];
+          // The next chunk's TMEM load overlaps this chunk's math and stores.
+          if (cc + 1 < n_ch) tmem_ld32_async(tbase + (uint32_t)((ch + 1) * 32), nxt);
+          const int nvalid = min(32, T.N - gc0);
+          float v[32];
+          if (L.stage == kStageGram) {
+            const float s2 = s * s;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  uint32_t w[4];
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) * s2;
+          } else if (L.stage == kStageSquare) {
+            // B' = a I + A P with P = b I + c A, i.e. a I + b A + c A^2.
 #pragma unroll
-                  for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
-                  if (8 * k < nvalid) dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-              }
-              continue;
-            }
-            const CUtensorMap* map = o == 0 ? uf.st_out : uf.st_p;
-            // Stores alternate between the two staging blocks, so only the
-            // store before last must have finished reading.
-            uint8_t* dst = stg0;
-            uint32_t dst_s = stg0_s;
-            if (stage_flip ^= 1) { dst = stg1; dst_s = stg1_s; }
-            if (stores_pending) {
-              if (lane == 0) bulk_wait_read_all_but_one();
-              __syncwarp();
-            }
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) + ((gc0 + j == grow) ? L.a : 0.f);
+          } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint32_t w[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
-              *reinterpret_cast<uint4*>(dst + stage_off(lane, 8 * k)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            fence_smem_to_async();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(map, dst_s, gc0, grow0);
-              bulk_commit();
-            }
-            stores_pending = true;
+            for (int j = 0; j < 32; ++j) v[j] = s * __uint_as_float(raw[j]);
           }
-        } else if (row_ok) {
-          if (L.out_kind == kOutPack1) {
-            uint32_t word = 0;
+          if (bf16_out) {
+            // Each 32x32 block is staged in shared memory and written by a TMA
+            // store.  The tiles of a symmetric output cover its upper
+            // 256-blocks only, which is all that is stored of it (its
+            // consumers read the other blocks transposed).  The Gram stage
+            // writes two outputs: A, then P = b I + c A (from the fp32 value
+            // of A).
+            const int n_out = (L.stage == kStageGram) ? 2 : 1;
+            // The Gram stage's A and P are fp16, everything else bf16.
+            const bool half_out = L.stage == kStageGram;
+            for (int o = 0; o < n_out; ++o) {
+              if (o == 1) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) word |= (j < nvalid && !(v[j] < 0.f)) ? (1u << j) : 0u;
-            const int wpr = (uf.cols + 31) >> 5;
-            static_cast<uint32_t*>(uf.out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
-          } else if (L.out_kind == kOutInt8) {
-            // A lane writes 32 bytes of its row, in the widest stores the
-            // row's alignment allows (the row starts at grow * cols bytes;
-            // gc0 is a multiple of 32).
-            int8_t* o = static_cast<int8_t*>(uf.out) + (int64_t)grow * uf.cols + gc0;
-            uint32_t pk[8];
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-              uint32_t x = 0;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) x |= (uint32_t)((v[4 * w + j] < 0.f) ? 0xFFu : 0x01u) << (8 * j);
-              pk[w] = x;
-            }
-            if (nvalid == 32 && (uf.cols & 15) == 0) {
-              reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            } else if (nvalid == 32 && (uf.cols & 7) == 0) {
-#pragma unroll
-              for (int w = 0; w < 4; ++w) reinterpret_cast<uint2*>(o)[w] = make_uint2(pk[2 * w], pk[2 * w + 1]);
-            } else if (nvalid == 32 && (uf.cols & 3) == 0) {
-#pragma unroll
-              for (int w = 0; w < 8; ++w) reinterpret_cast<uint32_t*>(o)[w] = pk[w];
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nvalid) o[j] = v[j] < 0.f ? int8_t(-1) : int8_t(1);
-            }
-          } else if (L.out_kind == kOutUF32) {
-            float* o = static_cast<float*>(uf.out) + (int64_t)grow * uf.cols + gc0;
-            if (nvalid == 32 && (uf.cols & 3) == 0) {
-#pragma unroll
-              for (int w = 0; w < 8; ++w)
-                reinterpret_cast<float4*>(o)[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nvalid) o[j] = v[j];
-            }
-          } else {  // kOutUpdateW: W <- W - eta * U
-            // 16-byte vectors when the row is aligned for them; the loads
-            // are all issued before the stores.
-            const int64_t off = (int64_t)grow * uf.cols + gc0;
-            if (L.w_dtype == SIGNMUON_BF16) {
-              __nv_bfloat16* w = static_cast<__nv_bfloat16*>(uf.out) + off;
-              if (nvalid == 32 && (uf.cols & 7) == 0) {
-                uint4 raw[4];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) raw[q4] = reinterpret_cast<const uint4*>(w)[q4];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                  __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&raw[q4]);
-#pragma unroll
-                  for (int j = 0; j < 8; ++j)
-                    e[j] = update_bf16(__bfloat162float(e[j]), L.eta, v[8 * q4 + j]);
-                  reinterpret_cast<uint4*>(w)[q4] = raw[q4];
-                }
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < nvalid) w[j] = update_bf16(__bfloat162float(w[j]), L.eta, v[j]);
+                for (int j = 0; j < 32; ++j) v[j] = fmaf(L.c, v[j], (gc0 + j == grow) ? L.b : 0.f);
               }
-            } else {
-              float* w = static_cast<float*>(uf.out) + off;
-              if (nvalid == 32 && (uf.cols & 3) == 0) {
+              if constexpr (kLong) {
+                // Straight from registers: each lane writes its row's 32
+                // columns (64 bytes) as four 16-byte stores, those starting
+                // inside the matrix (the row stride is a multiple of 8, so a
+                // store never crosses into the next row).
+                if (row_ok) {
+                  uint4* dst = reinterpret_cast<uint4*>((o == 0 ? uf.o16 : uf.p16) +
+                                                        ((int64_t)grow * uf.ld + gc0) * 2);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {  // two halves of 16 weights (register pressure)
-                  float4 x[4];
+                  for (int k = 0; k < 4; ++k) {
+                    uint32_t w[4];
 #pragma unroll
-                  for (int q4 = 0; q4 < 4; ++q4) x[q4] = reinterpret_cast<const float4*>(w)[4 * h + q4];
-#pragma unroll
-                  for (int q4 = 0; q4 < 4; ++q4) {
-                    const int j = 16 * h + 4 * q4;
-                    x[q4].x = fmaf(-L.eta, v[j + 0], x[q4].x);
-                    x[q4].y = fmaf(-L.eta, v[j + 1], x[q4].y);
-                    x[q4].z = fmaf(-L.eta, v[j + 2], x[q4].z);
-                    x[q4].w = fmaf(-L.eta, v[j + 3], x[q4].w);
-                    reinterpret_cast<float4*>(w)[4 * h + q4] = x[q4];
+                    for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
+                    if (8 * k < nvalid) dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
                   }
                 }
+                continue;
+              }
+              const CUtensorMap* map = o == 0 ? uf.st_out : uf.st_p;
+              // Stores alternate between the two staging blocks, so only the
+              // store before last must have finished reading.
+              uint8_t* dst = stg0;
+              uint32_t dst_s = stg0_s;
+              if (stage_flip ^= 1) { dst = stg1; dst_s = stg1_s; }
+              if (stores_pending) {
+                if (lane == 0) bulk_wait_read_all_but_one();
+                __syncwarp();
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                uint32_t w[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) w[j] = pack2(v[8 * k + 2 * j], v[8 * k + 2 * j + 1], half_out);
+                *reinterpret_cast<uint4*>(dst + stage_off(lane, 8 * k)) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+              fence_smem_to_async();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(map, dst_s, gc0, grow0);
+                bulk_commit();
+              }
+              stores_pending = true;
+            }
+          } else if (row_ok) {
+            if (L.out_kind == kOutPack1) {
+              uint32_t word = 0;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) word |= (j < nvalid && !(v[j] < 0.f)) ? (1u << j) : 0u;
+              const int wpr = (uf.cols + 31) >> 5;
+              static_cast<uint32_t*>(uf.out)[(int64_t)grow * wpr + (gc0 >> 5)] = word;
+            } else if (L.out_kind == kOutInt8) {
+              // A lane writes 32 bytes of its row, in the widest stores the
+              // row's alignment allows (the row starts at grow * cols bytes;
+              // gc0 is a multiple of 32).
+              int8_t* o = static_cast<int8_t*>(uf.out) + (int64_t)grow * uf.cols + gc0;
+              uint32_t pk[8];
+#pragma unroll
+              for (int w = 0; w < 8; ++w) {
+                uint32_t x = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x |= (uint32_t)((v[4 * w + j] < 0.f) ? 0xFFu : 0x01u) << (8 * j);
+                pk[w] = x;
+              }
+              if (nvalid == 32 && (uf.cols & 15) == 0) {
+                reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              } else if (nvalid == 32 && (uf.cols & 7) == 0) {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) reinterpret_cast<uint2*>(o)[w] = make_uint2(pk[2 * w], pk[2 * w + 1]);
+              } else if (nvalid == 32 && (uf.cols & 3) == 0) {
+#pragma unroll
+                for (int w = 0; w < 8; ++w) reinterpret_cast<uint32_t*>(o)[w] = pk[w];
               } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                  if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);
+                  if (j < nvalid) o[j] = v[j] < 0.f ? int8_t(-1) : int8_t(1);
+              }
+            } else if (L.out_kind == kOutUF32) {
+              float* o = static_cast<float*>(uf.out) + (int64_t)grow * uf.cols + gc0;
+              if (nvalid == 32 && (uf.cols & 3) == 0) {
+#pragma unroll
+                for (int w = 0; w < 8; ++w)
+                  reinterpret_cast<float4*>(o)[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nvalid) o[j] = v[j];
+              }
+            } else {  // kOutUpdateW: W <- W - eta * U
+              // 16-byte vectors when the row is aligned for them; the loads
+              // are all issued before the stores.
+              const int64_t off = (int64_t)grow * uf.cols + gc0;
+              if (L.w_dtype == SIGNMUON_BF16) {
+                __nv_bfloat16* w = static_cast<__nv_bfloat16*>(uf.out) + off;
+                if (nvalid == 32 && (uf.cols & 7) == 0) {
+                  uint4 raw[4];
+#pragma unroll
+                  for (int q4 = 0; q4 < 4; ++q4) raw[q4] = reinterpret_cast<const uint4*>(w)[q4];
+#pragma unroll
+                  for (int q4 = 0; q4 < 4; ++q4) {
+                    __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&raw[q4]);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                      e[j] = update_bf16(__bfloat162float(e[j]), L.eta, v[8 * q4 + j]);
+                    reinterpret_cast<uint4*>(w)[q4] = raw[q4];
+                  }
+                } else {
+#pragma unroll
+                  for (int j = 0; j < 32; ++j)
+                    if (j < nvalid) w[j] = update_bf16(__bfloat162float(w[j]), L.eta, v[j]);
+                }
+              } else {
+                float* w = static_cast<float*>(uf.out) + off;
+                if (nvalid == 32 && (uf.cols & 3) == 0) {
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {  // two halves of 16 weights (register pressure)
+                    float4 x[4];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) x[q4] = reinterpret_cast<const float4*>(w)[4 * h + q4];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                      const int j = 16 * h + 4 * q4;
+                      x[q4].x = fmaf(-L.eta, v[j + 0], x[q4].x);
+                      x[q4].y = fmaf(-L.eta, v[j + 1], x[q4].y);
+                      x[q4].z = fmaf(-L.eta, v[j + 2], x[q4].z);
+                      x[q4].w = fmaf(-L.eta, v[j + 3], x[q4].w);
+                      reinterpret_cast<float4*>(w)[4 * h + q4] = x[q4];
+                    }
+                  }
+                } else {
+#pragma unroll
+                  for (int j = 0; j < 32; ++j)
+                    if (j < nvalid) w[j] = fmaf(-L.eta, v[j], w[j]);
+                }
               }
             }
           }
         }
+        tc_fence_before();
+        if constexpr (kPair)
+          mbar_arrive_relaxed_cluster(map_to_rank(smem_addr(&tempty_bar[acc]), 0));  // the even CTA's barrier
+        else
+          mbar_arrive_relaxed(smem_addr(&tempty_bar[acc]));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
-      tc_fence_before();
-      if constexpr (kPair)
-        mbar_arrive_relaxed_cluster(map_to_rank(smem_addr(&tempty_bar[acc]), 0));  // the even CTA's barrier
-      else
-        mbar_arrive_relaxed(smem_addr(&tempty_bar[acc]));
-      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (!ep_ok) break;
     }
     // All of this warp's bulk stores must complete before the CTA exits.
     if (lane == 0 && stores_pending) bulk_wait_all();
@@ -955,21 +1082,24 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
     int n = 0;
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ns_gemm_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<false, false>::kSmem);
+    e = cudaFuncSetAttribute(ns_gemm_kernel<false, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<false, false, false>::kSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ns_gemm_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<true, false>::kSmem);
+    e = cudaFuncSetAttribute(ns_gemm_kernel<true, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<true, false, false>::kSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ns_gemm_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<true, true>::kSmem);
+    e = cudaFuncSetAttribute(ns_gemm_kernel<true, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<true, true, false>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(ns_gemm_kernel<true, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<true, true, true>::kSmem);
     if (e != cudaSuccess) return e;
     g_num_sms[dev] = n;
   }
   const int sms = g_num_sms[dev];
   if (!p.pair) {
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-    ns_gemm_kernel<false, false><<<grid, kGemmThreads, GemmCfg<false, false>::kSmem, stream>>>(p);
+    ns_gemm_kernel<false, false, false><<<grid, kGemmThreads, GemmCfg<false, false, false>::kSmem, stream>>>(p);
     return cudaGetLastError();
   }
   // One cluster of two CTAs per pair tile worker.
@@ -977,7 +1107,9 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = p.long_k ? GemmCfg<true, true>::kSmem : GemmCfg<true, false>::kSmem;
+  cfg.dynamicSmemBytes = p.wide     ? GemmCfg<true, true, true>::kSmem
+                         : p.long_k ? GemmCfg<true, true, false>::kSmem
+                                    : GemmCfg<true, false, false>::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -986,8 +1118,9 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (p.long_k) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true, true>, p);
-  return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true, false>, p);
+  if (p.wide) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true, true, true>, p);
+  if (p.long_k) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true, true, false>, p);
+  return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<true, false, false>, p);
 }
 
 }  // namespace signmuon

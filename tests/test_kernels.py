@@ -962,7 +962,7 @@ def test_square4096_batch_full_size_sampled():
 @pytest.mark.parametrize("shapes,M,k", [([(2056, 2100)], 1, 2), ([(300, 2100), (2100, 300)], 2, 1)])
 def test_long_reduction_layout_ragged_edges(shapes, M, k, monkeypatch):
     """Launches whose every tile has a reduction of 2048 or more use the
-    seven-stage layout that stores its 16-bit outputs from registers.  Ragged
+    layout that stores its 16-bit outputs from registers (256x512 tiles).  Ragged
     sizes (2056 x 2100: all three products long; 300 x 2100 and its
     transpose: the Gram product long) put row and column edges inside tiles
     and inside 32-column chunks: U within the Newton-Schulz tolerance of the
@@ -986,6 +986,33 @@ def test_long_reduction_layout_ragged_edges(shapes, M, k, monkeypatch):
         big = np.abs(ref) > 1e-3
         assert np.mean((got[big] < 0) == (ref[big] < 0)) >= SIGN_AGREE
         assert np.array_equal(unpack_words(packed[u].cpu().numpy().view(np.uint32), r, c), O.sign_entries(got))
+
+
+@pytest.mark.parametrize("shapes,M,k", [([(2056, 2100)], 1, 2), ([(300, 2100), (2100, 300)], 2, 1),
+                                        ([(2048, 4096), (4096, 2304)], 1, 1), ([(2560, 2560)], 2, 1)])
+def test_wide_tiles_equal_256_tiles(shapes, M, k, monkeypatch):
+    """The long-reduction launches run 256x512 CTA-pair tiles (two N = 256
+    MMAs per K step into the two halves of one TMEM accumulator, the first and
+    last k-blocks of a tile issuing half 0 ahead of half 1).  Each output
+    entry is accumulated over the same k-blocks in the same order as on
+    256x256 tiles, so U is bit-identical to the 256x256 layout's, on ragged
+    edges, on symmetric outputs whose tile rows start in the second half of a
+    512-column tile, and on tiles whose second half lies past the matrix; and
+    within the oracle tolerance."""
+    monkeypatch.setenv("SIGNMUON_NS_TILE_MODE", "pair")
+    grads, moms = seeded_state(shapes, M, 29)
+    outs = {}
+    for wide in ("0", "1"):
+        monkeypatch.setenv("SIGNMUON_NS_WIDE", wide)
+        xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], 0.9,
+                               torch.float32)
+        us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+        gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, us)
+        outs[wide] = us
+    for u in range(len(grads)):
+        assert torch.equal(outs["0"][u], outs["1"][u]), shapes[u // M]
+        _, ref = oracle_u(moms[u], grads[u], 0.9, k)
+        assert rel_fro(f64(outs["1"][u]), ref) <= NS_TOL, shapes[u // M]
 
 
 @pytest.mark.slow
