@@ -195,11 +195,11 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
  *   rows <= cols:  A = X X^T,  B = b A + c A^2,  X <- a X + B X
  *   rows >  cols:  A = X^T X,  B = b A + c A^2,  X <- a X + X B
  * on the tensor cores (bf16 operands, fp32 accumulation, bf16 between
- * iterations).  The kernels store A and P = b I + c A in fp16, form
- * B' = a I + A P (= a I + b A + c A^2, bf16) and compute X <- B' X (X B'):
- * the same map with the a X term folded into the product.  Of the
- * symmetric A, P and B' only the 256x256 blocks on and above the diagonal
- * are computed and stored in the workspace.
+ * iterations).  The kernels store A in fp16, form B' = a I + b A + c A A
+ * (bf16) and compute X <- B' X (X B'): the same map with the a X term
+ * folded into the product.  Of the symmetric A and B' only the 256x256
+ * blocks on and above the diagonal are computed and stored in the
+ * workspace.
  * The last iteration's epilogue writes, per out_mode:
  *   PACK1:    out[u] = packed sign(U)   (uint32, signmuon_packed_words words)
  *   INT8:     out[u] = int8 sign(U)     ([rows, cols])
@@ -227,8 +227,8 @@ signmuon_status signmuon_newton_schulz_batched(
  * Step 1b-2 split in two: plan once, run every step.
  * Same computation as signmuon_newton_schulz_batched (which is exactly
  * plan followed by run); the split only moves per-call host work off the
- * step: encoding ten TMA tensor maps per unit and uploading the unit table
- * (1408 bytes per unit) happen once, in plan, instead of on every call.
+ * step: encoding eight TMA tensor maps per unit and uploading the unit table
+ * (1152 bytes per unit) happen once, in plan, instead of on every call.
  * An optimizer whose buffers persist from step to step plans once and then
  * calls run each step.
  *

@@ -88,8 +88,8 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, int64_t inner, int64_t o
 }
 
 // ----------------------------------------------------------------- NS planning
-// Per-unit workspace: Gram A and P = bI + cA (s x s fp16), B' = aI + A P
-// (s x s bf16) and the second X iterate (bf16).
+// Per-unit workspace: Gram A (s x s fp16), B' = aI + bA + cA^2 (s x s bf16)
+// and the second X iterate (bf16).
 struct UnitBytes {
   size_t a, xalt, total;
 };
@@ -100,7 +100,7 @@ UnitBytes ns_unit_bytes(signmuon_shape sh) {
   UnitBytes u;
   u.a = align_up((size_t)(s * ld_s * 2), 1024);
   u.xalt = align_up((size_t)sh.rows * x_ld_of(sh.cols) * 2, 1024);
-  u.total = 3 * u.a + u.xalt;
+  u.total = 2 * u.a + u.xalt;
   return u;
 }
 
@@ -427,10 +427,42 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
   uint8_t* arena = ws + tables;
   const size_t arena_bytes = ws_bytes - tables;
 
-  // Plan waves: consecutive units whose buffers fit the arena together.
+  // Plan waves: consecutive units whose buffers fit the arena together.  The
+  // fewest waves are those of a greedy fill; the units are then re-split into
+  // that many waves of about equal bytes (so that the last is no small
+  // remainder), unless a wave of that split would not fit.
+  std::vector<size_t> ubytes(units);
+  size_t total_bytes = 0;
+  for (int i = 0; i < n_mats; ++i)
+    for (int m = 0; m < n_workers; ++m) total_bytes += (ubytes[i * n_workers + m] = ns_unit_bytes(shapes[i]).total);
+  std::vector<int> starts_new(units, 0);
+  int n_greedy = 0;
+  {
+    size_t fill = arena_bytes;  // forces a new wave at unit 0
+    for (int ui = 0; ui < units; ++ui) {
+      if (fill + ubytes[ui] > arena_bytes) { starts_new[ui] = 1; ++n_greedy; fill = 0; }
+      fill += ubytes[ui];
+    }
+  }
+  {
+    std::vector<int> even(units, 0);
+    size_t before = 0, fill = 0;
+    int wave = -1;
+    bool fits = true;
+    for (int ui = 0; ui < units && fits; ++ui) {
+      // Wave of the unit's midpoint on the even split.
+      const int w = (int)std::min<size_t>((size_t)n_greedy - 1,
+                                          (before + ubytes[ui] / 2) * (size_t)n_greedy / std::max<size_t>(total_bytes, 1));
+      if (w != wave) { even[ui] = 1; wave = w; fill = 0; }
+      fill += ubytes[ui];
+      fits = fill <= arena_bytes;
+      before += ubytes[ui];
+    }
+    if (fits) starts_new = even;
+  }
   std::vector<NsUnit> hu(units);
   std::vector<int> wave_begin;
-  size_t used = arena_bytes;  // forces a new wave at unit 0
+  size_t used = 0;
   int64_t max_elems = 0;
   for (int i = 0; i < n_mats; ++i) {
     const UnitBytes ub = ns_unit_bytes(shapes[i]);
@@ -439,7 +471,7 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
     max_elems = std::max(max_elems, (int64_t)rows * cols);
     for (int m = 0; m < n_workers; ++m) {
       const int ui = i * n_workers + m;
-      if (used + ub.total > arena_bytes) {
+      if (starts_new[ui]) {
         wave_begin.push_back(ui);
         used = 0;
       }
@@ -452,8 +484,7 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
       u.x = static_cast<__nv_bfloat16*>(x_bf16[ui]);
       u.a = arena + used;
       u.b = reinterpret_cast<__nv_bfloat16*>(arena + used + ub.a);
-      u.p = arena + used + 2 * ub.a;
-      u.xalt = reinterpret_cast<__nv_bfloat16*>(arena + used + 3 * ub.a);
+      u.xalt = reinterpret_cast<__nv_bfloat16*>(arena + used + 2 * ub.a);
       used += ub.total;
       u.out = out_mode == SIGNMUON_OUT_UPDATE_W ? w[i] : out[ui];
       u.scale = inv_norm + ui;
@@ -461,8 +492,6 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
           !encode_bf16_2d(&u.map_xalt, u.xalt, cols, rows, u.ld_x) ||
           !encode_bf16_2d(&u.map_a, u.a, sdim, sdim, u.ld_s, false, true) ||
           !encode_bf16_2d(&u.map_b, u.b, sdim, sdim, u.ld_s) ||
-          !encode_bf16_2d(&u.map_p, u.p, sdim, sdim, u.ld_s, false, true) ||
-          !encode_bf16_2d(&u.st_p, u.p, sdim, sdim, u.ld_s, true, true) ||
           !encode_bf16_2d(&u.st_x, u.x, cols, rows, u.ld_x, true) ||
           !encode_bf16_2d(&u.st_xalt, u.xalt, cols, rows, u.ld_x, true) ||
           !encode_bf16_2d(&u.st_a, u.a, sdim, sdim, u.ld_s, true, true) ||

@@ -77,18 +77,15 @@ struct alignas(64) NsUnit {
   CUtensorMap map_xalt;  // workspace bf16 X buffer [rows, ld_x]
   CUtensorMap map_a;     // workspace Gram A (fp16)  [s, ld_s]
   CUtensorMap map_b;     // workspace B' = aI + bA + cA^2 (bf16) [s, ld_s]
-  CUtensorMap map_p;     // workspace P = bI + cA (fp16) [s, ld_s]
   // Store maps: 32x32 boxes, 64-byte swizzle (epilogue output blocks).
   CUtensorMap st_x;
   CUtensorMap st_xalt;
   CUtensorMap st_a;
   CUtensorMap st_b;
-  CUtensorMap st_p;
   __nv_bfloat16* x;
   __nv_bfloat16* xalt;
   void* a;               // fp16
   __nv_bfloat16* b;
-  void* p;               // fp16
   void* out;             // final output (packed / int8 / fp32 U / W)
   const float* scale;    // &inv_norm[u]
   int32_t rows, cols, ld_x, ld_s;
@@ -157,7 +154,7 @@ struct VoteMat {
   int32_t pad_;
 };
 
-static_assert(sizeof(NsUnit) == 1408, "descriptor size is part of the launch-count bookkeeping");
+static_assert(sizeof(NsUnit) == 1152, "descriptor size is part of the launch-count bookkeeping");
 static_assert(sizeof(MomUnit) == 56, "descriptor size is part of the launch-count bookkeeping");
 static_assert(sizeof(VoteMat) == 64, "descriptor size is part of the launch-count bookkeeping");
 

@@ -5,14 +5,14 @@
 // item 1: the momentum is orthogonalised toward its polar factor) over every
 // (matrix, worker) unit of a launch:
 //   stage Gram:   A = X X^T            (X^T X for tall X), symmetric output
-//   stage Square: B' = a I + A P           (P = b I + c A written by the Gram
-//                                            stage; A, P symmetric, stored in
-//                                            fp16 for the diagonal's sake)
+//   stage Square: B' = a I + b A + c A A   (A symmetric, stored in fp16 for
+//                                            the diagonal's sake; the epilogue
+//                                            reads A_ij back for the b A term)
 //   stage Apply:  X' = B' X            (X B' for tall X), i.e. a X + (b A + c A^2) X
 // with, in the last iteration, the entrywise sign fused into the epilogue and
 // written as packed bits or int8 (steps 2-3 of the summary's flow), or the
 // update W <- W - eta U (the optional local polar step, step 5).
-// Of the symmetric A, P and B' only the 256x256 blocks on and above the
+// Of the symmetric A and B' only the 256x256 blocks on and above the
 // diagonal are computed and stored; the stages that consume them read a
 // k-block below the diagonal as the transpose of the stored block.
 //
@@ -407,7 +407,7 @@ struct Tile {
   int a_up, b_up;  // operand is a symmetric matrix of which only the upper 256-blocks are stored
 };
 
-// Symmetric products (A, P, B') are stored as their 256x256 blocks (I, J)
+// Symmetric products (A, B') are stored as their 256x256 blocks (I, J)
 // with J >= I only.  An operand that is one of them reads k-block
 // [k0, k0 + 64) of its rows [r0, r0 + 128) -- all in 256-block r0 / 256 --
 // directly when k0 / 256 >= r0 / 256, and otherwise as the transpose of the
@@ -429,7 +429,7 @@ __device__ __forceinline__ Tile tile_of(int stage, int rows, int cols, int li, i
   T.a_up = 0; T.b_up = 0;
   if (stage == kStageGram) {
     T.M = s; T.N = s; T.K = l; T.sym = 1; T.a_mn = tall; T.b_mn = tall;
-  } else if (stage == kStageSquare) {  // A P: both operands symmetric
+  } else if (stage == kStageSquare) {  // A A: both operands the symmetric A
     T.M = s; T.N = s; T.K = s; T.sym = 1; T.a_mn = 0; T.b_mn = 0; T.a_up = 1; T.b_up = 1;
   } else if (!tall) {  // X' = B' X: A-op = B' (symmetric, K-major), B-op = X (MN-major)
     T.M = rows; T.N = cols; T.K = s; T.sym = 0; T.a_mn = 0; T.b_mn = 1; T.a_up = 1;
@@ -467,13 +467,13 @@ __device__ __forceinline__ bool half_ok(const Tile& T, int h) {
   return n0 < T.N && (!T.sym || n0 >= (T.m0 & ~255));
 }
 
-// Pair mode, Gram stage, diagonal block: each CTA's B rows of the half
-// starting at column n0 (n0 + 128 rank ..) are its A rows (m0 + 128 rank ..)
-// of the same operand, so that half of B is read from the A buffer and not
-// loaded.
+// Pair mode, Gram and square stages (the same matrix on both sides),
+// diagonal block: each CTA's B rows of the half starting at column n0
+// (n0 + 128 rank ..) are its A rows (m0 + 128 rank ..), so that half of B is
+// read from the A buffer and not loaded.
 template <bool kPair>
 __device__ __forceinline__ bool diag_b_from_a(const NsLaunch& L, const Tile& T, int n0) {
-  return kPair && L.stage == kStageGram && T.m0 == n0;
+  return kPair && L.stage != kStageApply && T.m0 == n0;
 }
 
 // Tensor maps of the two operands of a unit's tile.
@@ -483,7 +483,7 @@ __device__ __forceinline__ void operand_maps(const NsLaunch& L, const NsUnit* u,
   if (L.stage == kStageGram) {
     ma = xin; mb = xin;
   } else if (L.stage == kStageSquare) {
-    ma = &u->map_a; mb = &u->map_p;  // A P, P = bI + cA symmetric (K-major rows)
+    ma = &u->map_a; mb = &u->map_a;  // A A (symmetric, K-major rows)
   } else if (!tall) {
     ma = &u->map_b; mb = xin;
   } else {
@@ -637,7 +637,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       for (int t = first_tile; t < L.total_tiles && ok; t += tile_stride) {
         const NsTileRec rec = rs.advance(L, t, tile_stride);
         const Tile T = tile_of(L.stage, rec.rows, rec.cols, rec.li, C::kTileM, C::kTileN);
-        // The square stage multiplies the fp16 A and P; all others are bf16.
+        // The square stage multiplies the fp16 A by itself; all others are bf16.
         const bool fp16_ops = L.stage == kStageSquare;
         const int nkb = (T.K + kBK - 1) / kBK;
         if constexpr (kWide) {
@@ -801,13 +801,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     // Their loads are issued before the wait for the accumulator.
     struct {
       const CUtensorMap* st_out;  // store map of this stage's bf16 output
-      const CUtensorMap* st_p;    // Gram stage: store map of P = bI + cA
-      void* out;
+      void* out;                  // the last apply's output; square stage: the stored fp16 A
       int cols;
       uint8_t* o16;               // long layout: this stage's 16-bit output
-      uint8_t* p16;               //   the Gram stage's P
-      int ld;                     //   and their row stride (elements)
-    } uf = {nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0};
+      int ld;                     //   and its row stride (elements; square stage: A's)
+    } uf = {nullptr, nullptr, 0, nullptr, 0};
     float s = 1.f;
     for (int t = first_tile; t < L.total_tiles; t += tile_stride) {
       const NsTileRec rec = rs.advance(L, t, tile_stride);
@@ -817,14 +815,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         uf.st_out = L.stage == kStageGram ? &un->st_a
                   : L.stage == kStageSquare ? &un->st_b
                   : (L.parity ? &un->st_x : &un->st_xalt);
-        uf.st_p = &un->st_p;
-        uf.out = un->out;
+        uf.out = L.stage == kStageSquare ? un->a : un->out;
+        uf.ld = L.stage == kStageApply ? un->ld_x : un->ld_s;
         if constexpr (kLong) {
           uf.o16 = static_cast<uint8_t*>(L.stage == kStageGram     ? un->a
                                          : L.stage == kStageSquare ? static_cast<void*>(un->b)
                                          : static_cast<void*>(L.parity ? un->x : un->xalt));
-          uf.p16 = static_cast<uint8_t*>(un->p);
-          uf.ld = L.stage == kStageApply ? un->ld_x : un->ld_s;
         }
         uf.cols = rec.cols;
         s = L.first ? __ldg(L.scales + rec.unit) : 1.f;
@@ -869,9 +865,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) * s2;
           } else if (L.stage == kStageSquare) {
-            // B' = a I + A P with P = b I + c A, i.e. a I + b A + c A^2.
+            // B' = a I + b A + c A^2: the accumulator holds A A, and A_ij is
+            // read back from the stored fp16 A (this tile's block (I, J),
+            // J >= I, is one of the stored upper blocks).
+            const __half* arow = static_cast<const __half*>(uf.out) + (int64_t)grow * uf.ld + gc0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) + ((gc0 + j == grow) ? L.a : 0.f);
+            for (int k = 0; k < 4; ++k) {
+              uint4 w = make_uint4(0u, 0u, 0u, 0u);
+              if (row_ok && 8 * k < nvalid) w = *reinterpret_cast<const uint4*>(arow + 8 * k);
+              const __half2* h2 = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float2 f = __half22float2(h2[q]);
+                const int j = 8 * k + 2 * q;
+                v[j] = fmaf(L.c, __uint_as_float(raw[j]), fmaf(L.b, f.x, (gc0 + j == grow) ? L.a : 0.f));
+                v[j + 1] = fmaf(L.c, __uint_as_float(raw[j + 1]), fmaf(L.b, f.y, (gc0 + j + 1 == grow) ? L.a : 0.f));
+              }
+            }
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = s * __uint_as_float(raw[j]);
@@ -880,25 +890,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             // Each 32x32 block is staged in shared memory and written by a TMA
             // store.  The tiles of a symmetric output cover its upper
             // 256-blocks only, which is all that is stored of it (its
-            // consumers read the other blocks transposed).  The Gram stage
-            // writes two outputs: A, then P = b I + c A (from the fp32 value
-            // of A).
-            const int n_out = (L.stage == kStageGram) ? 2 : 1;
-            // The Gram stage's A and P are fp16, everything else bf16.
+            // consumers read the other blocks transposed).
+            // The Gram stage's A is fp16, everything else bf16.
             const bool half_out = L.stage == kStageGram;
-            for (int o = 0; o < n_out; ++o) {
-              if (o == 1) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = fmaf(L.c, v[j], (gc0 + j == grow) ? L.b : 0.f);
-              }
+            {
               if constexpr (kLong) {
                 // Straight from registers: each lane writes its row's 32
                 // columns (64 bytes) as four 16-byte stores, those starting
                 // inside the matrix (the row stride is a multiple of 8, so a
                 // store never crosses into the next row).
                 if (row_ok) {
-                  uint4* dst = reinterpret_cast<uint4*>((o == 0 ? uf.o16 : uf.p16) +
-                                                        ((int64_t)grow * uf.ld + gc0) * 2);
+                  uint4* dst = reinterpret_cast<uint4*>(uf.o16 + ((int64_t)grow * uf.ld + gc0) * 2);
 #pragma unroll
                   for (int k = 0; k < 4; ++k) {
                     uint32_t w[4];
@@ -907,9 +909,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                     if (8 * k < nvalid) dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
                   }
                 }
-                continue;
-              }
-              const CUtensorMap* map = o == 0 ? uf.st_out : uf.st_p;
+              } else {
+              const CUtensorMap* map = uf.st_out;
               // Stores alternate between the two staging blocks, so only the
               // store before last must have finished reading.
               uint8_t* dst = stg0;
@@ -933,6 +934,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                 bulk_commit();
               }
               stores_pending = true;
+              }
             }
           } else if (row_ok) {
             if (L.out_kind == kOutPack1) {

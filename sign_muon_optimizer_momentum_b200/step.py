@@ -271,13 +271,13 @@ class SignMuonStep:
     @staticmethod
     def _waves(shapes, M, ws_bytes) -> int:
         """Waves the library splits the units into for this workspace size
-        (its buffers per unit: A, P, B' and an X copy, 1 KB aligned)."""
+        (its buffers per unit: A, B' and an X copy, 1 KB aligned)."""
         def al(x, a):
             return (x + a - 1) // a * a
 
         def unit_bytes(r, c):
             s = min(r, c)
-            return 3 * al(s * al(s, 8) * 2, 1024) + al(r * al(c, 8) * 2, 1024)
+            return 2 * al(s * al(s, 8) * 2, 1024) + al(r * al(c, 8) * 2, 1024)
         # The minimal workspace is the tables plus the largest unit's buffers.
         tables = (L.signmuon_newton_schulz_workspace_bytes(shapes, M, minimal=True)
                   - max(unit_bytes(r, c) for r, c in shapes))

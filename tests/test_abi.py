@@ -61,8 +61,8 @@ def test_workspace_sizes(lib):
     full = L.signmuon_newton_schulz_workspace_bytes(shapes, 8)
     minimal = L.signmuon_newton_schulz_workspace_bytes(shapes, 8, minimal=True)
     assert minimal < full
-    # One unit of the largest buffers: A, P and B' (768^2 bf16 each) + an X copy.
-    assert minimal >= 256 + 16 * 1408 + 3 * 768 * 768 * 2 + 3072 * 768 * 2
+    # One unit of the largest buffers: A and B' (768^2 16-bit each) + an X copy.
+    assert minimal >= 256 + 16 * 1152 + 2 * 768 * 768 * 2 + 3072 * 768 * 2
     assert L.signmuon_vote_workspace_bytes(shapes, 8) >= 256 + 2 * 64 + 16 * 8
     assert L.signmuon_momentum_workspace_bytes([], 8) == 0
     assert L.signmuon_momentum_workspace_bytes([(0, 3)], 8) == 0
