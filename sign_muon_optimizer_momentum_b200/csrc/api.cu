@@ -540,10 +540,7 @@ signmuon_status ns_make_plan(const signmuon_shape* shapes, int n_mats, int n_wor
         min_k = std::min(min_k, kr);
       }
       W.long_k[stg] = pair && min_k >= kLongK ? 1 : 0;
-      // The Gram product stays on 256x256 tiles: its epilogue writes two
-      // outputs (A and P), which the double-buffered accumulator hides
-      // better than the two halves of a 256x512 tile do.
-      W.wide[stg] = W.long_k[stg] && wide_ok && stg != kStageGram ? 1 : 0;
+      W.wide[stg] = W.long_k[stg] && wide_ok ? 1 : 0;
       const int wide = W.wide[stg];
       int pre = 0;
       W.rec0[stg] = (int64_t)recs.size();

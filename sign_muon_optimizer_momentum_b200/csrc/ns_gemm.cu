@@ -29,10 +29,10 @@
 //           barrier, and one multicast commit frees a stage in both CTAs.
 //           Launches whose every reduction is at least kLongK long use a
 //           seventh stage instead of the epilogue's staging memory and store
-//           their 16-bit outputs from registers (the long-reduction layout);
-//           their square and apply products run 256x512 tiles (two N = 256
-//           MMAs per K step into the two halves of TMEM, 48 KB stages, 4
-//           stages), a quarter less operand data per FLOP.
+//           their 16-bit outputs from registers (the long-reduction layout),
+//           on 256x512 tiles (two N = 256 MMAs per K step into the two
+//           halves of TMEM, 48 KB stages, 4 stages): a quarter less operand
+//           data per FLOP.
 // Roles (320 threads per CTA):
 //   warp 0     TMA producer: 64x64 bf16 boxes, 128-byte swizzle
 //   warp 1     MMA issuer (even CTA of a pair): kind::f16, N=256, K=16,
