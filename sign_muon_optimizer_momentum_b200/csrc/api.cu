@@ -638,6 +638,9 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
       L.a = a;
       L.b = b;
       L.c = c;
+      L.shift = c != 0.f;
+      L.beta = L.shift ? (float)((double)b / (2.0 * (double)c)) : 0.f;
+      L.a2 = L.shift ? (float)((double)a - (double)b * (double)b / (4.0 * (double)c)) : a;
       L.eta = eta;
       L.w_dtype = hdr->w_dtype;
       L.err = reinterpret_cast<uint32_t*>(hdr->workspace);

@@ -118,6 +118,11 @@ struct NsLaunch {
   int total_tiles;
   int pair;         // 1: CTA-pair (cta_group::2) 256x256 tiles; 0: one CTA, 128x256
   float a, b, c, eta;
+  // c != 0: the Gram stage stores Q = A + beta I (beta = b / 2c) in place of
+  // A, and the square stage forms B' = c Q Q + a2 I (a2 = a - b^2 / 4c),
+  // which equals a I + b A + c A^2; c == 0: A itself, B' = a I + b A.
+  int shift;
+  float beta, a2;
   uint32_t* err;
   uint64_t wait_limit_ns;  // every bounded wait gives up after this long
   // Fault injection for testing the bounded waits: the producer arms no

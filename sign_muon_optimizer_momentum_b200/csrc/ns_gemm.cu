@@ -4,10 +4,12 @@
 // a Newton-Schulz iteration (SignMuon summary, section 2 "Core mechanism"
 // item 1: the momentum is orthogonalised toward its polar factor) over every
 // (matrix, worker) unit of a launch:
-//   stage Gram:   A = X X^T            (X^T X for tall X), symmetric output
-//   stage Square: B' = a I + b A + c A A   (A symmetric, stored in fp16 for
-//                                            the diagonal's sake; the epilogue
-//                                            reads A_ij back for the b A term)
+//   stage Gram:   A = X X^T            (X^T X for tall X), symmetric output,
+//                                       stored as Q = A + b/(2c) I (c != 0)
+//   stage Square: B' = c Q Q + a2 I        (Q = A + b/(2c) I, symmetric, stored
+//                                            by the Gram stage in fp16 for the
+//                                            diagonal's sake; a2 = a - b^2/(4c):
+//                                            the same a I + b A + c A^2)
 //   stage Apply:  X' = B' X            (X B' for tall X), i.e. a X + (b A + c A^2) X
 // with, in the last iteration, the entrywise sign fused into the epilogue and
 // written as packed bits or int8 (steps 2-3 of the summary's flow), or the
@@ -861,13 +863,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           const int nvalid = min(32, T.N - gc0);
           float v[32];
           if (L.stage == kStageGram) {
+            // A, or Q = A + beta I (see NsLaunch::shift).
             const float s2 = s * s;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(raw[j]) * s2;
+            for (int j = 0; j < 32; ++j) v[j] = fmaf(__uint_as_float(raw[j]), s2, (gc0 + j == grow) ? L.beta : 0.f);
+          } else if (L.stage == kStageSquare && L.shift) {
+            // B' = c Q Q + a2 I = a I + b A + c A^2 (the accumulator holds Q Q).
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = fmaf(L.c, __uint_as_float(raw[j]), (gc0 + j == grow) ? L.a2 : 0.f);
           } else if (L.stage == kStageSquare) {
-            // B' = a I + b A + c A^2: the accumulator holds A A, and A_ij is
-            // read back from the stored fp16 A (this tile's block (I, J),
-            // J >= I, is one of the stored upper blocks).
+            // c == 0, B' = a I + b A (+ c A A): A_ij is read back from the
+            // stored fp16 A (this tile's block (I, J), J >= I, is one of the
+            // stored upper blocks).
             const __half* arow = static_cast<const __half*>(uf.out) + (int64_t)grow * uf.ld + gc0;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {

@@ -65,10 +65,10 @@ def gpu_momentum(shapes, M, grads, moms, beta, grad_dtype):
 
 
 def gpu_ns(shapes, M, xs, inv, k, out_mode, outs=None, w_dtype=L.SIGNMUON_F32, weights=None, eta=0.0,
-           minimal_ws=False):
+           minimal_ws=False, coeffs=(A, B, C)):
     nbytes = L.signmuon_newton_schulz_workspace_bytes(shapes, M, minimal=minimal_ws)
     w = ws(nbytes)
-    L.signmuon_newton_schulz_batched(shapes, M, [x.data_ptr() for x in xs], inv.data_ptr(), k, A, B, C,
+    L.signmuon_newton_schulz_batched(shapes, M, [x.data_ptr() for x in xs], inv.data_ptr(), k, *coeffs,
                                      out_mode, None if outs is None else [o.data_ptr() for o in outs],
                                      w_dtype, None if weights is None else [x.data_ptr() for x in weights],
                                      eta, w.data_ptr(), w.numel(), stream())
@@ -310,6 +310,25 @@ def test_newton_schulz_matches_oracle(shapes, M, k):
         if big.sum() > 0:
             agree = np.mean(np.sign(got[big]) == np.sign(ref[big]))
             assert agree >= SIGN_AGREE, (shapes[u // M], agree)
+
+
+@pytest.mark.parametrize("coeffs", [(1.5, -0.5, 0.0), (2.0, -1.5, 0.5)])
+@pytest.mark.parametrize("shapes,M,k", [([(256, 384), (300, 700)], 2, 3), ([(2056, 2100)], 1, 2)])
+def test_newton_schulz_other_coefficients(coeffs, shapes, M, k):
+    """Coefficients other than the quintic: c = 0 (the cubic iteration,
+    B' = a I + b A, the square stage reading A back), and c != 0 with another
+    diagonal shift (the Gram stage stores A + b/(2c) I and the square forms
+    c Q Q + (a - b^2/(4c)) I); short and long-reduction launches."""
+    grads, moms = seeded_state(shapes, M, 31)
+    xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], 0.9,
+                           torch.float32)
+    us = [torch.empty(shapes[u // M], dtype=torch.float32, device="cuda") for u in range(len(xs))]
+    gpu_ns(shapes, M, xs, inv, k, L.SIGNMUON_OUT_U_F32, us, coeffs=coeffs)
+    a, b, c = coeffs
+    for u in range(len(grads)):
+        mom = O.momentum_update(f64(moms[u]), f64(grads[u]), float(np.float32(0.9)))
+        ref = O.newton_schulz(O.frobenius_normalize(mom), k, a, b, c)
+        assert rel_fro(f64(us[u]), ref) <= NS_TOL, (coeffs, shapes[u // M])
 
 
 def test_newton_schulz_fused_outputs_are_signs_of_u():
