@@ -195,10 +195,11 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
  *   rows <= cols:  A = X X^T,  B = b A + c A^2,  X <- a X + B X
  *   rows >  cols:  A = X^T X,  B = b A + c A^2,  X <- a X + X B
  * on the tensor cores (bf16 operands, fp32 accumulation, bf16 between
- * iterations).  The kernels store Q = A + b/(2c) I in fp16 (A itself when
- * c == 0), form B' = c Q Q + (a - b^2/(4c)) I = a I + b A + c A^2 (bf16;
- * a I + b A when c == 0) and compute X <- B' X (X B'): the same map with the
- * a X term folded into the product.  Of the symmetric Q and B' only the
+ * iterations).  The kernels store Q = A + b/(2c) I in fp16 and form
+ * B' = c Q Q + (a - b^2/(4c)) I = a I + b A + c A^2 (bf16) when c != 0 and
+ * |b/(2c)| <= 4 (otherwise they store A and form a I + b A + c A A), and
+ * compute X <- B' X (X B'): the same map with the a X term folded into the
+ * product.  Of the symmetric Q and B' only the
  * 256x256 blocks on and above the diagonal are computed and stored in the
  * workspace.
  * The last iteration's epilogue writes, per out_mode:

@@ -3,6 +3,7 @@
 // and their contracts are in include/signmuon.h.
 #include <algorithm>
 #include <climits>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -638,7 +639,9 @@ signmuon_status ns_run_plan(const void* plan, int k, float a, float b, float c, 
       L.a = a;
       L.b = b;
       L.c = c;
-      L.shift = c != 0.f;
+      // The shifted form when the shift is moderate (Q's diagonal keeps fp16's
+      // absolute precision near that of A): |b / 2c| <= 4.
+      L.shift = c != 0.f && std::fabs((double)b) <= 8.0 * std::fabs((double)c);
       L.beta = L.shift ? (float)((double)b / (2.0 * (double)c)) : 0.f;
       L.a2 = L.shift ? (float)((double)a - (double)b * (double)b / (4.0 * (double)c)) : a;
       L.eta = eta;

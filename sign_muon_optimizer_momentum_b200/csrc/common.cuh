@@ -118,9 +118,10 @@ struct NsLaunch {
   int total_tiles;
   int pair;         // 1: CTA-pair (cta_group::2) 256x256 tiles; 0: one CTA, 128x256
   float a, b, c, eta;
-  // c != 0: the Gram stage stores Q = A + beta I (beta = b / 2c) in place of
-  // A, and the square stage forms B' = c Q Q + a2 I (a2 = a - b^2 / 4c),
-  // which equals a I + b A + c A^2; c == 0: A itself, B' = a I + b A.
+  // shift (c != 0 and |b / 2c| <= 4): the Gram stage stores Q = A + beta I
+  // (beta = b / 2c) in place of A, and the square stage forms
+  // B' = c Q Q + a2 I (a2 = a - b^2 / 4c), which equals a I + b A + c A^2;
+  // otherwise A itself, and the square's epilogue reads A back for b A.
   int shift;
   float beta, a2;
   uint32_t* err;

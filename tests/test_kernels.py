@@ -312,13 +312,15 @@ def test_newton_schulz_matches_oracle(shapes, M, k):
             assert agree >= SIGN_AGREE, (shapes[u // M], agree)
 
 
-@pytest.mark.parametrize("coeffs", [(1.5, -0.5, 0.0), (2.0, -1.5, 0.5)])
+@pytest.mark.parametrize("coeffs", [(1.5, -0.5, 0.0), (2.0, -1.5, 0.5), (1.0, -1.0, 0.01)])
 @pytest.mark.parametrize("shapes,M,k", [([(256, 384), (300, 700)], 2, 3), ([(2056, 2100)], 1, 2)])
 def test_newton_schulz_other_coefficients(coeffs, shapes, M, k):
     """Coefficients other than the quintic: c = 0 (the cubic iteration,
-    B' = a I + b A, the square stage reading A back), and c != 0 with another
-    diagonal shift (the Gram stage stores A + b/(2c) I and the square forms
-    c Q Q + (a - b^2/(4c)) I); short and long-reduction launches."""
+    B' = a I + b A, the square stage reading A back), c != 0 with another
+    moderate diagonal shift (the Gram stage stores A + b/(2c) I and the square
+    forms c Q Q + (a - b^2/(4c)) I), and a shift too large for fp16's
+    precision (b/(2c) = -50: the unshifted form); short and long-reduction
+    launches."""
     grads, moms = seeded_state(shapes, M, 31)
     xs, inv = gpu_momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], 0.9,
                            torch.float32)
