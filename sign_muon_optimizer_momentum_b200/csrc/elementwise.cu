@@ -810,6 +810,19 @@ __global__ void spectral_init_kernel(const SpecUnit* __restrict__ units, float* 
   for (int j = threadIdx.x; j < u.cols; j += blockDim.x) vecs[u.v_off + j] = v0;
 }
 
+// Packed fp32 pair helpers (sm_100 fma.rn.f32x2): the low half of the
+// 64-bit value is the even column, the high half the odd one.
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// Two bf16 (low half: the even column) widened to two fp32: a bf16 is the
+// high 16 bits of the fp32 of the same value.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint64_t)(w << 16);
+}
+
 // One block per 32 rows of one unit: y_r = x_r . v for its rows, then the
 // partial z_j = sum_r y_r x_rj of the block (rows re-read from L1/L2).
 __global__ void __launch_bounds__(256, 4)
@@ -837,20 +850,20 @@ spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const f
       const __nv_bfloat16* xr = u.x + (int64_t)(r0 + rr) * u.ld_x;
       if (vec) {
         // Unrolled so that several 16-byte loads of the row are in flight.
+        // Even and odd columns accumulate in the two halves of a packed
+        // f32x2 (one FMA instruction per pair of columns).
+        uint64_t acc2 = 0;
 #pragma unroll 4
         for (int j = lane * 8; j < u.cols; j += 256) {
           const uint4 raw = *reinterpret_cast<const uint4*>(xr + j);
-          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-          const float4 va = *reinterpret_cast<const float4*>(v + j);
-          const float4 vb = *reinterpret_cast<const float4*>(v + j + 4);
-          const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = __bfloat1622float2(h[q]);
-            acc = fmaf(f.x, vv[2 * q], acc);
-            acc = fmaf(f.y, vv[2 * q + 1], acc);
-          }
+          const ulonglong2 va = *reinterpret_cast<const ulonglong2*>(v + j);
+          const ulonglong2 vb = *reinterpret_cast<const ulonglong2*>(v + j + 4);
+          acc2 = fma_f32x2(bf16x2_to_f32x2(raw.x), va.x, acc2);
+          acc2 = fma_f32x2(bf16x2_to_f32x2(raw.y), va.y, acc2);
+          acc2 = fma_f32x2(bf16x2_to_f32x2(raw.z), vb.x, acc2);
+          acc2 = fma_f32x2(bf16x2_to_f32x2(raw.w), vb.y, acc2);
         }
+        acc = __uint_as_float((uint32_t)acc2) + __uint_as_float((uint32_t)(acc2 >> 32));
       } else {
         for (int j = lane; j < u.cols; j += 32) acc = fmaf(__bfloat162float(xr[j]), v[j], acc);
       }
@@ -863,21 +876,19 @@ spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const f
   float* part = parts + u.part_off + (int64_t)rb * u.cols;
   if (vec) {
     for (int j = threadIdx.x * 8; j < u.cols; j += 256 * 8) {
-      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint64_t z2[4] = {0, 0, 0, 0};  // columns j .. j + 7 as four packed f32x2
 #pragma unroll 4
       for (int rr = 0; rr < nrows; ++rr) {
         const uint4 raw = *reinterpret_cast<const uint4*>(u.x + (int64_t)(r0 + rr) * u.ld_x + j);
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        const float y = ys[rr];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h[q]);
-          z[2 * q] = fmaf(y, f.x, z[2 * q]);
-          z[2 * q + 1] = fmaf(y, f.y, z[2 * q + 1]);
-        }
+        const uint32_t yb = __float_as_uint(ys[rr]);
+        const uint64_t y2 = ((uint64_t)yb << 32) | yb;
+        z2[0] = fma_f32x2(bf16x2_to_f32x2(raw.x), y2, z2[0]);
+        z2[1] = fma_f32x2(bf16x2_to_f32x2(raw.y), y2, z2[1]);
+        z2[2] = fma_f32x2(bf16x2_to_f32x2(raw.z), y2, z2[2]);
+        z2[3] = fma_f32x2(bf16x2_to_f32x2(raw.w), y2, z2[3]);
       }
-      *reinterpret_cast<float4*>(part + j) = make_float4(z[0], z[1], z[2], z[3]);
-      *reinterpret_cast<float4*>(part + j + 4) = make_float4(z[4], z[5], z[6], z[7]);
+      *reinterpret_cast<ulonglong2*>(part + j) = make_ulonglong2(z2[0], z2[1]);
+      *reinterpret_cast<ulonglong2*>(part + j + 4) = make_ulonglong2(z2[2], z2[3]);
     }
   } else {
     for (int j = threadIdx.x; j < u.cols; j += 256) {
