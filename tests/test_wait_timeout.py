@@ -8,8 +8,10 @@ operand load, so the MMA issuer's and the epilogue's waits can only run out,
 and shortens the limit to a few milliseconds.  The test checks that the call
 returns, that signmuon_device_error reports a wait-timeout code (and clears
 it), and that the next normal call on the same context and workspace gives
-the oracle's result.  One-CTA tiles: each CTA gives up on its own, nothing
-waits across CTAs.
+the oracle's result.  Both tile modes: one-CTA tiles, where each CTA gives
+up on its own, and CTA pairs on a long-reduction launch (256x512 tiles),
+where the even CTA's MMA issuer and the odd CTA's producer and epilogue each
+give up on their own bounded waits before the pair's exit barrier.
 """
 import time
 
@@ -43,14 +45,16 @@ def _momentum(shapes, M, grads, moms, stream):
     return xs, inv
 
 
-def test_injected_wait_timeout_is_reported_and_the_context_stays_usable(cuda_lib, monkeypatch):
-    shapes, M, k = [(256, 256), (96, 300)], 2, 2
+@pytest.mark.parametrize("shapes,M,k,mode", [([(256, 256), (96, 300)], 2, 2, "single"),
+                                             ([(2048, 2048)], 1, 1, "pair")])
+def test_injected_wait_timeout_is_reported_and_the_context_stays_usable(cuda_lib, monkeypatch, shapes, M, k,
+                                                                         mode):
     stream = torch.cuda.current_stream().cuda_stream
     grads, moms = _inputs(shapes, M)
     nbytes = L.signmuon_newton_schulz_workspace_bytes(shapes, M)
     wk = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     us = [torch.full(shapes[u // M], 7.0, dtype=torch.float32, device="cuda") for u in range(len(grads))]
-    monkeypatch.setenv("SIGNMUON_NS_TILE_MODE", "single")
+    monkeypatch.setenv("SIGNMUON_NS_TILE_MODE", mode)
 
     # 1. Loads withheld, 20 ms limit: 3k launches, each gives up on its own.
     xs, inv = _momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], stream)
@@ -64,7 +68,7 @@ def test_injected_wait_timeout_is_reported_and_the_context_stays_usable(cuda_lib
     elapsed = time.perf_counter() - t0
     code = L.signmuon_device_error(wk.data_ptr(), stream)
     assert code in WAIT_TIMEOUT_CODES, hex(code)
-    assert elapsed < 1.5, elapsed                  # 6 launches x ~20 ms, far below the 2 s default limit
+    assert elapsed < 1.5, elapsed                  # 3k launches x a few 20 ms waits, far below the 2 s default
     assert L.signmuon_device_error(wk.data_ptr(), stream) == 0     # read and cleared
     assert all(bool((u == 7.0).all()) for u in us)                 # the outputs were not written
 
