@@ -516,11 +516,13 @@ def time_workload(ctx, wl, args, *, norm, steps, warmup, graph=False, exchange=F
         updated, read_back = torch.cuda.Event(), torch.cuda.Event()
 
         def e2e_steps(n):
-            h2d_into(0)
+            # Steady state: step t copies step t + 1's gradients while it
+            # computes (the copy for the step after the last one included),
+            # so n steps make n H2D copies and n D2H read-backs; the first
+            # step's gradients were copied before.
             for t in range(n):
                 buf = t % 2
-                if t + 1 < n:
-                    h2d_into(1 - buf)
+                h2d_into(1 - buf)
                 stream.wait_event(copied[buf])
                 opt.momentum_norm(grad_sets[buf], s_ptr)
                 consumed[buf].record(stream)
@@ -534,8 +536,11 @@ def time_workload(ctx, wl, args, *, norm, steps, warmup, graph=False, exchange=F
                     for hw, w in zip(host_w, weights):
                         hw.copy_(w, non_blocking=True)
                     read_back.record(d2h_stream)
-            stream.wait_event(read_back)   # the last step's weights are on the host
+            stream.wait_event(read_back)       # the last step's weights are on the host
+            stream.wait_event(copied[n % 2])   # and the next step's gradients on the device
 
+        h2d_into(0)
+        stream.wait_event(copied[0])
         e2e_steps(2)
         ctx.barrier()
         e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -549,7 +554,9 @@ def time_workload(ctx, wl, args, *, norm, steps, warmup, graph=False, exchange=F
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                       "ms_per_step": e_ms / n_e2e,
                       "note": "gradients H2D from pinned host memory and weights D2H to pinned host memory, every "
-                              "step, each on its own copy stream overlapped with the neighbouring step's compute"}
+                              "step, each on its own copy stream overlapped with the neighbouring step's compute "
+                              "(steady state: each step copies the next step's gradients; the timed region holds "
+                              "one H2D and one D2H per step)"}
         del host_g, host_w
     if graphs:
         del graphs
