@@ -87,6 +87,7 @@ KERNEL_SOURCES = {
     "momentum_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
     "vote_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
     "spectral_rowpass_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
+    "spectral_segment_kernel": (_CSRC + "elementwise.cu", _CSRC + "common.cuh"),
 }
 
 
@@ -574,26 +575,47 @@ def extra_signum(ctx, args, pk):
             "roofline": momentum_roofline(wl, r["opt"], r["phases_ms"]["momentum"], pk)}
 
 
+def spectral_bytes_per_iteration(shapes, n_workers):
+    """Algorithmic bytes of one power iteration: each unit's bf16 copy of M
+    read once, and its partial sums of z written and read back (one per
+    (128-row segment, row subset) for widths that are multiples of 8 up to
+    4096, else one per 32-row block), 4 B per column each."""
+    total = 0
+    for r, c in shapes:
+        if c % 8 == 0 and c <= 4096:
+            nch = c // 8
+            g = min(24576 // (2 * c), 32)
+            rs = 1 if nch > 128 else min(256 // nch, g)
+            parts = -(-r // 128) * rs
+        else:
+            parts = -(-r // 32)
+        total += r * c * 2 + 2 * parts * c * 4
+    return total * n_workers
+
+
 def extra_spectral(ctx, args, pk):
     """The nanoGPT-small step with spectral scaling of the Newton-Schulz input
-    (5 power iterations per unit); roofline of the power-iteration kernels:
-    per iteration each unit's bf16 copy of M is read once (2 B/param), its
-    row-block partial sums written and read back (1/8 + 1/8 B/param)."""
+    (5 power iterations per unit); roofline of the power-iteration pass: per
+    iteration each unit's bf16 copy of M is read once (2 B/param) and its
+    partial sums of z written and read back."""
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
     wl = syn.WORKLOADS["nanogpt_small"]
     r = time_workload(ctx, wl, args, norm="spectral", steps=20, warmup=3)
     iters = r["opt"].spectral_iters
-    gbytes = iters * wl.params * wl.n_workers * 2.25
+    per_iter = spectral_bytes_per_iteration(wl.shapes, wl.n_workers)
+    gbytes = iters * per_iter
     achieved = gbytes / (r["spectral_ms"] / 1e3) / 1e9
+    kernel = "spectral_segment_kernel"
     return {"workload": wl.name, "config": dict(workload_config(wl), norm="spectral", spectral_iters=iters),
             "metric": METRIC, "value": r["value"], "unit": UNIT, "ms_per_step": r["ms_per_step"], "steps": 20,
             "warmup": 3, "phases_ms": dict(r["phases_ms"], spectral_alone=r["spectral_ms"]),
-            "roofline": {"bound": "hbm", "kernel": "spectral_rowpass_kernel", "achieved": achieved,
+            "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                         "traffic": captured_traffic("spectral_rowpass_kernel", wl.name)
-                         if "spectral_rowpass_kernel" in KERNEL_SOURCES else None,
-                         "note": f"{iters} power iterations: {gbytes / 1e9:.3f} GB algorithmic (2.25 B per "
-                                 f"param*worker and iteration) over {r['spectral_ms']:.3f} ms, timed alone"}}
+                         "traffic": captured_traffic(kernel, wl.name),
+                         "note": f"{iters} power iterations: {gbytes / 1e9:.3f} GB algorithmic "
+                                 f"({per_iter / (wl.params * wl.n_workers):.3f} B per param*worker and iteration: "
+                                 f"the bf16 copy of M once, partial sums of z written and read back) over "
+                                 f"{r['spectral_ms']:.3f} ms, timed alone"}}
 
 
 def run_gpu(args, wl):

@@ -277,25 +277,46 @@ signmuon_status signmuon_momentum_sign(const signmuon_shape* shapes, int n_mats,
 }
 
 // ------------------------------------------------------------ spectral scaling
-static size_t spec_layout(const signmuon_shape* shapes, int n_mats, int n_workers, size_t* v_floats,
-                          size_t* part_floats) {
+// Spectral workspace: header | units | seg_unit | blk_seg | v | partials.
+struct SpecLayout {
+  size_t units, seg_unit, blk_seg, vecs, parts, total;  // byte offsets (total = size)
+  int segs;
+};
+// Partials of z per unit: one per row block, or per (segment, row subset).
+static int spec_parts(signmuon_shape sh, int* segs) {
+  if (spec_segmented(sh.cols)) {
+    *segs = (sh.rows + kSpecSegRows - 1) / kSpecSegRows;
+    return *segs * spec_zsplit(sh.cols);
+  }
+  *segs = 0;
+  return (sh.rows + kSpecRows - 1) / kSpecRows;
+}
+static SpecLayout spec_layout(const signmuon_shape* shapes, int n_mats, int n_workers) {
   size_t vf = 0, pf = 0;
+  int segs = 0;
   for (int i = 0; i < n_mats; ++i) {
     const size_t cols4 = align_up((size_t)shapes[i].cols, 4);
-    const size_t n_rb = ((size_t)shapes[i].rows + kSpecRows - 1) / kSpecRows;
+    int ns = 0;
+    const size_t n_parts = (size_t)spec_parts(shapes[i], &ns);
     vf += cols4 * n_workers;
-    pf += n_rb * cols4 * n_workers;
+    pf += n_parts * cols4 * n_workers;
+    segs += ns * n_workers;
   }
-  *v_floats = vf;
-  *part_floats = pf;
   const size_t units = (size_t)n_mats * n_workers;
-  return kWsHeaderBytes + align_up(units * sizeof(SpecUnit), 256) + align_up(vf * 4, 256) + align_up(pf * 4, 256);
+  SpecLayout L;
+  L.segs = segs;
+  L.units = kWsHeaderBytes;
+  L.seg_unit = L.units + align_up(units * sizeof(SpecUnit), 256);
+  L.blk_seg = L.seg_unit + align_up((size_t)segs * 4, 256);
+  L.vecs = L.blk_seg + align_up((size_t)(kSpecMaxGrid + 1) * 4, 256);
+  L.parts = L.vecs + align_up(vf * 4, 256);
+  L.total = L.parts + align_up(pf * 4, 256);
+  return L;
 }
 
 size_t signmuon_spectral_workspace_bytes(const signmuon_shape* shapes, int n_mats, int n_workers) {
   if (validate_shapes(shapes, n_mats) != SIGNMUON_OK || n_workers <= 0) return 0;
-  size_t vf, pf;
-  return spec_layout(shapes, n_mats, n_workers, &vf, &pf);
+  return spec_layout(shapes, n_mats, n_workers).total;
 }
 
 signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats, int n_workers,
@@ -309,38 +330,71 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
   if ((st = validate_ptrs(x_bf16, units))) return st;
   if (!inv_norm) return SIGNMUON_ERR_INVALID_ARG;
   if (!aligned16(inv_norm)) return SIGNMUON_ERR_ALIGNMENT;
-  size_t vf, pf;
-  const size_t need = spec_layout(shapes, n_mats, n_workers, &vf, &pf);
-  if ((st = check_workspace(workspace, ws_bytes, need))) return st;
+  const SpecLayout lay = spec_layout(shapes, n_mats, n_workers);
+  if ((st = check_workspace(workspace, ws_bytes, lay.total))) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  std::vector<SpecUnit> hu(units);
+  // One host blob for the unit table and the segment tables (one upload).
+  std::vector<uint8_t> blob(lay.vecs - lay.units, 0);
+  SpecUnit* hu = reinterpret_cast<SpecUnit*>(blob.data());
+  int32_t* seg_unit = reinterpret_cast<int32_t*>(blob.data() + (lay.seg_unit - lay.units));
+  int32_t* blk_seg = reinterpret_cast<int32_t*>(blob.data() + (lay.blk_seg - lay.units));
+  std::vector<int64_t> seg_bytes;
+  seg_bytes.reserve(lay.segs);
   int64_t voff = 0, poff = 0;
-  int blocks = 0;
+  int blocks = 0, segs = 0;
   for (int i = 0; i < n_mats; ++i) {
     const int64_t cols4 = (int64_t)align_up((size_t)shapes[i].cols, 4);
-    const int n_rb = (shapes[i].rows + kSpecRows - 1) / kSpecRows;
+    int n_seg = 0;
+    const int n_parts = spec_parts(shapes[i], &n_seg);
     for (int m = 0; m < n_workers; ++m) {
-      SpecUnit& u = hu[i * n_workers + m];
+      const int ui = i * n_workers + m;
+      SpecUnit& u = hu[ui];
       memset(&u, 0, sizeof(u));
-      u.x = static_cast<const __nv_bfloat16*>(x_bf16[i * n_workers + m]);
+      u.x = static_cast<const __nv_bfloat16*>(x_bf16[ui]);
       u.rows = shapes[i].rows;
       u.cols = shapes[i].cols;
       u.ld_x = x_ld_of(u.cols);
-      u.n_rb = n_rb;
+      u.n_parts = n_parts;
       u.v_off = voff;
       u.part_off = poff;
+      // Each pass numbers only its own units' work (the others own an empty range).
       u.block_begin = blocks;
+      u.seg_begin = segs;
       voff += cols4;
-      poff += (int64_t)n_rb * cols4;
-      blocks += n_rb;
+      poff += (int64_t)n_parts * cols4;
+      if (n_seg > 0) {
+        for (int k = 0; k < n_seg; ++k) {
+          seg_unit[segs + k] = ui;
+          seg_bytes.push_back((int64_t)std::min(kSpecSegRows, u.rows - k * kSpecSegRows) * u.cols * 2);
+        }
+        segs += n_seg;
+      } else {
+        blocks += n_parts;
+      }
     }
   }
+  // Segment-pass blocks (two per SM) take contiguous ranges of segments
+  // holding about equal shares of the bytes.
+  const int seg_grid = std::min(std::min(segs, 2 * sm_count()), kSpecMaxGrid);
+  int64_t total = 0;
+  for (int64_t b : seg_bytes) total += b;
+  int sgi = 0;
+  int64_t before = 0;
+  blk_seg[0] = 0;
+  for (int b = 1; b < seg_grid; ++b) {
+    const int64_t target = total * b / seg_grid;
+    while (sgi < segs && before + seg_bytes[sgi] / 2 < target) before += seg_bytes[sgi++];
+    blk_seg[b] = sgi;
+  }
+  if (seg_grid > 0) blk_seg[seg_grid] = segs;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  SpecUnit* d_units = reinterpret_cast<SpecUnit*>(ws + kWsHeaderBytes);
-  float* vecs = reinterpret_cast<float*>(ws + kWsHeaderBytes + align_up(units * sizeof(SpecUnit), 256));
-  float* parts = vecs + align_up(vf * 4, 256) / 4;
-  cudaError_t e = upload_bytes(d_units, hu.data(), hu.size() * sizeof(SpecUnit), s);
-  if (e == cudaSuccess) e = launch_spectral(d_units, units, blocks, vecs, parts, iters, inv_norm, s);
+  cudaError_t e = upload_bytes(ws + lay.units, blob.data(), blob.size(), s);
+  if (e == cudaSuccess)
+    e = launch_spectral(reinterpret_cast<const SpecUnit*>(ws + lay.units), units, blocks,
+                        reinterpret_cast<const int32_t*>(ws + lay.seg_unit),
+                        reinterpret_cast<const int32_t*>(ws + lay.blk_seg), seg_grid,
+                        reinterpret_cast<float*>(ws + lay.vecs), reinterpret_cast<float*>(ws + lay.parts), iters,
+                        inv_norm, reinterpret_cast<uint32_t*>(ws), s);
   return cuda_status(e);
 }
 

@@ -20,6 +20,7 @@ enum DeviceError : uint32_t {
   kErrWaitTimeoutMma = 0x102,       // MMA issuer gave up waiting for data / accumulator
   kErrWaitTimeoutEpilogue = 0x103,  // epilogue gave up waiting for an accumulator
   kErrWaitTimeoutDrain = 0x104,     // exit-time wait for in-flight copies ran out
+  kErrWaitTimeoutSpectral = 0x105,  // spectral segment pass gave up waiting for its rows
 };
 
 // Workspace header: error word + padding.  Every workspace starts with it.
@@ -165,18 +166,43 @@ static_assert(sizeof(MomUnit) == 56, "descriptor size is part of the launch-coun
 static_assert(sizeof(VoteMat) == 64, "descriptor size is part of the launch-count bookkeeping");
 
 // Spectral-scaling units (power iteration on X^T X).
+// A unit is passed over either by the segment pass (spec_segmented(cols):
+// rows streamed through shared memory, spec_zsplit(cols) partials of z per
+// kSpecSegRows rows) or by the row-block pass (any other width: one partial
+// of z per kSpecRows rows).
 struct SpecUnit {
   const __nv_bfloat16* x;
   int64_t v_off;        // float offset of this unit's vector v (cols entries)
-  int64_t part_off;     // float offset of its partial sums [n_rb][cols]
+  int64_t part_off;     // float offset of its partial sums [n_parts][cols]
   int32_t rows, cols, ld_x;
-  int32_t n_rb;         // row blocks of kSpecRows rows
-  int32_t block_begin;  // first row block of this unit in the flattened grid
-  int32_t pad_;
+  int32_t n_parts;      // its segment partials, or its row blocks
+  int32_t block_begin;  // first row block of this unit in the row-block pass's grid (none if segmented)
+  int32_t seg_begin;    // first segment of this unit in the segment pass's sequence (none if not)
 };
 static_assert(sizeof(SpecUnit) == 48, "descriptor size");
 constexpr int kSpecRows = 32;
 constexpr int kSpecSmemCols = 8192;  // v is staged in shared memory up to this many columns (32 KB)
+constexpr int kSpecSegRows = 128;       // rows per segment
+constexpr int kSpecSlotBytes = 24576;   // shared-memory ring slot: the rows of one group
+constexpr int kSpecSlots = 4;
+constexpr int kSpecSegMaxCols = 4096;   // at most two 8-column chunks per thread of 256
+constexpr int kSpecMaxGrid = 512;       // segment-pass blocks at most (two per SM)
+__host__ __device__ inline bool spec_segmented(int cols) { return (cols & 7) == 0 && cols <= kSpecSegMaxCols; }
+// Rows per group (ring slot) of a segmented unit: the most rows that fit a
+// slot, at most 32.
+__host__ __device__ inline int spec_group_rows(int cols) {
+  const int g = kSpecSlotBytes / (2 * cols);
+  return g < 32 ? g : 32;
+}
+// Row subsets of a segmented unit's z update: a unit of at most 128 8-column
+// chunks spreads 256 threads over (row subset, chunk) pairs; each subset
+// writes its own partial of z.
+__host__ __device__ inline int spec_zsplit(int cols) {
+  const int nch = cols / 8;
+  if (nch > 128) return 1;
+  const int rs = 256 / nch, g = spec_group_rows(cols);
+  return rs < g ? rs : g;
+}
 
 // ---------------------------------------------------------------------------
 // Launch helpers implemented in the .cu files (all enqueue on `stream`).
@@ -194,8 +220,11 @@ cudaError_t launch_vote(const VoteMat* mats, int n_mats, int total_blocks, const
 cudaError_t launch_vote_inv(const int64_t* nnz, float* inv, int n_mats, cudaStream_t stream);
 int vote_blocks_for(int int8_in, int w_bf16, int vote_out, int cols, int64_t n, int64_t n_words);
 cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream);
-cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, float* vecs, float* parts,
-                            int iters, float* inv_norm, cudaStream_t stream);
+// seg_unit[s]: the unit of segment s (segments in unit order); the segment
+// pass's block b takes segments [blk_seg[b], blk_seg[b + 1]) of seg_grid blocks.
+cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, const int32_t* seg_unit,
+                            const int32_t* blk_seg, int seg_grid, float* vecs, float* parts, int iters,
+                            float* inv_norm, uint32_t* err, cudaStream_t stream);
 cudaError_t launch_ns_identity(const NsUnit* units, int n_units, int64_t max_elems, int out_kind,
                                int w_dtype, float eta, cudaStream_t stream);
 

@@ -899,6 +899,224 @@ spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const f
   }
 }
 
+// Segment pass: blocks of 256 threads, two per SM, each streaming a
+// contiguous range of segments (kSpecSegRows rows of one unit; the ranges
+// split the bytes evenly, so a block rarely changes unit).  The rows go
+// through a ring of kSpecSlots shared-memory slots in groups of
+// G = spec_group_rows(cols) rows, one bulk copy per group (a segmented unit's
+// width is a multiple of 8, so its row stride is its width and a group is one
+// contiguous range) issued by thread 0 up to kSpecSlots groups ahead, across
+// segments: the rows are read from DRAM once, with many bytes in flight.  Per
+// group, warp w forms y_r = x_r . v for rows r = w, w + 8, ... (v staged in
+// shared memory), and after one block barrier every thread adds y_r x_r to
+// its part of z: wide units (more than 128 8-column chunks) by chunk, narrow
+// ones by (row subset, chunk), each row subset keeping a partial of its own.
+// Both products use packed f32x2 FMAs.
+__device__ __forceinline__ void spec_mbar_init(uint32_t bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void spec_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void spec_bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ bool spec_mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of `bar` with this parity; false after kWaitTimeoutNs.
+__device__ __forceinline__ bool spec_mbar_wait(uint32_t bar, uint32_t parity) {
+  if (spec_mbar_test(bar, parity)) return true;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t n = 1;; ++n) {
+    if (spec_mbar_test(bar, parity)) return true;
+    if ((n & 63) == 0) {
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > kWaitTimeoutNs) return false;
+    }
+  }
+}
+// z (8 columns as four f32x2) += y2 * (8 bf16 at p, 16 bytes of shared memory).
+__device__ __forceinline__ void spec_axpy8(const uint8_t* p, uint64_t y2, uint64_t (&z)[4]) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(p);
+  z[0] = fma_f32x2(bf16x2_to_f32x2(raw.x), y2, z[0]);
+  z[1] = fma_f32x2(bf16x2_to_f32x2(raw.y), y2, z[1]);
+  z[2] = fma_f32x2(bf16x2_to_f32x2(raw.z), y2, z[2]);
+  z[3] = fma_f32x2(bf16x2_to_f32x2(raw.w), y2, z[3]);
+}
+
+__global__ void __launch_bounds__(256, 2)
+spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __restrict__ seg_unit,
+                        const int32_t* __restrict__ blk_seg, const float* __restrict__ vecs,
+                        float* __restrict__ parts, uint32_t* __restrict__ err) {
+  // Ring of kSpecSlots slots, then v (kSpecSegMaxCols floats).
+  extern __shared__ __align__(1024) uint8_t spec_ring[];
+  float* vs = reinterpret_cast<float*>(spec_ring + kSpecSlots * kSpecSlotBytes);
+  __shared__ __align__(8) uint64_t full[kSpecSlots];
+  __shared__ float ys[2][32];  // y of the group, double-buffered by group parity
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(spec_ring));
+  const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(full));
+  const int seg_first = __ldg(blk_seg + blockIdx.x), seg_end = __ldg(blk_seg + blockIdx.x + 1);
+  if (tid == 0) {
+    for (int i = 0; i < kSpecSlots; ++i) spec_mbar_init(bar0 + 8 * i);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  // Producer cursor (thread 0): the next group to load.  The unit of the
+  // segment after the current one is fetched a segment ahead.
+  int p_seg = seg_first, p_row = 0, p_idx = 0, p_unit = -1;
+  int p_next = seg_first < seg_end ? __ldg(seg_unit + seg_first) : -1;
+  const __nv_bfloat16* p_x = nullptr;
+  int p_cols = 8, p_g = 1, p_row0 = 0, p_nrows = 0;
+  auto p_open = [&]() {
+    if (p_seg >= seg_end) return;
+    const int ui = p_next;
+    p_next = p_seg + 1 < seg_end ? __ldg(seg_unit + p_seg + 1) : -1;
+    if (ui != p_unit) {
+      p_unit = ui;
+      p_x = units[ui].x;
+      p_cols = __ldg(&units[ui].cols);
+      p_g = spec_group_rows(p_cols);
+    }
+    p_row0 = (p_seg - __ldg(&units[ui].seg_begin)) * kSpecSegRows;
+    p_nrows = min(kSpecSegRows, __ldg(&units[ui].rows) - p_row0);
+  };
+  // Loads the next group into its slot, which no thread still reads.
+  auto p_issue = [&]() {
+    if (p_seg >= seg_end) return;
+    const int gn = min(p_g, p_nrows - p_row);
+    const int slot = p_idx % kSpecSlots;
+    const uint32_t bytes = (uint32_t)gn * (uint32_t)p_cols * 2u;
+    // The slot's earlier rows were read through the generic proxy.
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    spec_expect_tx(bar0 + 8 * slot, bytes);
+    spec_bulk_load(ring + slot * kSpecSlotBytes, p_x + (int64_t)(p_row0 + p_row) * p_cols, bytes, bar0 + 8 * slot);
+    ++p_idx;
+    p_row += gn;
+    if (p_row >= p_nrows) {
+      ++p_seg;
+      p_row = 0;
+      p_open();
+    }
+  };
+  if (tid == 0) {
+    p_open();
+    for (int i = 0; i < kSpecSlots; ++i) p_issue();
+  }
+
+  int g = 0;  // groups consumed by this block
+  bool failed = false;
+  int c_unit = -1, c_next = seg_first < seg_end ? __ldg(seg_unit + seg_first) : -1;
+  int cols = 8, G = 1, rows = 0, seg_begin = 0, nch = 1, rs = 1, q = 0, c0 = 0;
+  int64_t part_off = 0;
+  bool own0 = false, own1 = false;
+  for (int seg = seg_first; seg < seg_end && !failed; ++seg) {
+    const int ui = c_next;
+    c_next = seg + 1 < seg_end ? __ldg(seg_unit + seg + 1) : -1;
+    if (ui != c_unit) {
+      // Every thread is past the last dot phase of the previous unit (its
+      // group's barrier), so v can be replaced.
+      c_unit = ui;
+      cols = __ldg(&units[ui].cols);
+      rows = __ldg(&units[ui].rows);
+      seg_begin = __ldg(&units[ui].seg_begin);
+      part_off = __ldg(&units[ui].part_off);
+      G = spec_group_rows(cols);
+      nch = cols >> 3;
+      rs = spec_zsplit(cols);
+      if (nch > 128) {
+        q = 0; c0 = tid; own0 = tid < nch; own1 = tid + 256 < nch;
+      } else {
+        q = tid / nch; c0 = tid - q * nch; own0 = q < rs; own1 = false;
+      }
+      const float* vg = vecs + __ldg(&units[ui].v_off);
+      for (int j = tid; j < cols; j += 256) vs[j] = vg[j];
+      __syncthreads();
+    }
+    const int row0 = (seg - seg_begin) * kSpecSegRows;
+    const int nrows = min(kSpecSegRows, rows - row0);
+    const int row_bytes = 2 * cols;
+    uint64_t z0[4] = {0, 0, 0, 0}, z1[4] = {0, 0, 0, 0};
+    for (int gr0 = 0; gr0 < nrows; gr0 += G, ++g) {
+      const int gn = min(G, nrows - gr0);
+      const int slot = g % kSpecSlots;
+      const bool ok = spec_mbar_wait(bar0 + 8 * slot, (uint32_t)((g / kSpecSlots) & 1));
+      const uint8_t* base = spec_ring + slot * kSpecSlotBytes;
+      float* yb = ys[g & 1];
+      if (ok) {
+        for (int r = warp; r < gn; r += 8) {
+          const uint8_t* row = base + r * row_bytes;
+          uint64_t acc2 = 0;
+          for (int c = lane; c < nch; c += 32) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(row + 16 * c);
+            const ulonglong2 va = *reinterpret_cast<const ulonglong2*>(vs + 8 * c);
+            const ulonglong2 vb = *reinterpret_cast<const ulonglong2*>(vs + 8 * c + 4);
+            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.x), va.x, acc2);
+            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.y), va.y, acc2);
+            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.z), vb.x, acc2);
+            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.w), vb.y, acc2);
+          }
+          float acc = __uint_as_float((uint32_t)acc2) + __uint_as_float((uint32_t)(acc2 >> 32));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == 0) yb[r] = acc;
+        }
+      }
+      // Every thread is past the previous group here: its slot is free.
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      if (tid == 0 && g > 0) p_issue();
+      if (nch > 128) {
+        for (int r = 0; r < gn; ++r) {
+          const uint32_t yu = __float_as_uint(yb[r]);
+          const uint64_t y2 = ((uint64_t)yu << 32) | yu;
+          const uint8_t* row = base + r * row_bytes;
+          if (own0) spec_axpy8(row + 16 * c0, y2, z0);
+          if (own1) spec_axpy8(row + 16 * (c0 + 256), y2, z1);
+        }
+      } else if (own0) {
+        for (int r = q; r < gn; r += rs) {
+          const uint32_t yu = __float_as_uint(yb[r]);
+          spec_axpy8(base + r * row_bytes + 16 * c0, ((uint64_t)yu << 32) | yu, z0);
+        }
+      }
+    }
+    if (failed) break;
+    // This segment's partial of z (one per row subset for narrow units).
+    float* part = parts + part_off + ((int64_t)(seg - seg_begin) * rs + q) * cols;
+    if (own0) {
+      *reinterpret_cast<ulonglong2*>(part + 8 * c0) = make_ulonglong2(z0[0], z0[1]);
+      *reinterpret_cast<ulonglong2*>(part + 8 * c0 + 4) = make_ulonglong2(z0[2], z0[3]);
+    }
+    if (own1) {
+      *reinterpret_cast<ulonglong2*>(part + 8 * (c0 + 256)) = make_ulonglong2(z1[0], z1[1]);
+      *reinterpret_cast<ulonglong2*>(part + 8 * (c0 + 256) + 4) = make_ulonglong2(z1[2], z1[3]);
+    }
+  }
+  if (failed && tid == 0) {
+    // Record the error, then wait (bounded) for every copy still in flight
+    // before the block's shared memory is released.
+    atomicCAS(err, 0u, (uint32_t)kErrWaitTimeoutSpectral);
+    for (int i = g; i < p_idx; ++i) (void)spec_mbar_wait(bar0 + 8 * (i % kSpecSlots), (uint32_t)((i / kSpecSlots) & 1));
+  }
+}
+
 // One block per unit: z = sum of the row-block partials (fixed order),
 // v <- z / ||z||; after the last iteration inv_norm = 1 / (sqrt(||z||) + eps).
 __global__ void __launch_bounds__(256)
@@ -910,7 +1128,7 @@ spectral_reduce_kernel(const SpecUnit* __restrict__ units, float* __restrict__ v
   double ss = 0.0;
   for (int j = threadIdx.x; j < u.cols; j += blockDim.x) {
     float z = 0.f;
-    for (int rb = 0; rb < u.n_rb; ++rb) z += part[(int64_t)rb * u.cols + j];
+    for (int rb = 0; rb < u.n_parts; ++rb) z += part[(int64_t)rb * u.cols + j];
     v[j] = z;
     ss += (double)z * (double)z;
   }
@@ -927,15 +1145,33 @@ spectral_reduce_kernel(const SpecUnit* __restrict__ units, float* __restrict__ v
   if (last && threadIdx.x == 0) inv_norm[blockIdx.x] = (float)(1.0 / (sqrt(zn) + 1e-7));
 }
 
-cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, float* vecs, float* parts,
-                            int iters, float* inv_norm, cudaStream_t stream) {
+cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, const int32_t* seg_unit,
+                            const int32_t* blk_seg, int seg_grid, float* vecs, float* parts, int iters,
+                            float* inv_norm, uint32_t* err, cudaStream_t stream) {
+  constexpr int kSegSmem = kSpecSlots * kSpecSlotBytes + kSpecSegMaxCols * 4;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    if ((e = cudaFuncSetAttribute(spectral_segment_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSegSmem)) !=
+        cudaSuccess)
+      return e;
+    attr_set[dev] = true;
+  }
   spectral_init_kernel<<<n_units, 256, 0, stream>>>(units, vecs);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
-    spectral_rowpass_kernel<<<total_row_blocks, 256, kSpecSmemCols * sizeof(float), stream>>>(units, n_units,
-                                                                                             vecs, parts);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) break;
+    if (seg_grid > 0) {
+      spectral_segment_kernel<<<seg_grid, 256, kSegSmem, stream>>>(units, seg_unit, blk_seg, vecs, parts, err);
+      if ((e = cudaGetLastError()) != cudaSuccess) break;
+    }
+    if (total_row_blocks > 0) {
+      spectral_rowpass_kernel<<<total_row_blocks, 256, kSpecSmemCols * sizeof(float), stream>>>(units, n_units,
+                                                                                               vecs, parts);
+      if ((e = cudaGetLastError()) != cudaSuccess) break;
+    }
     spectral_reduce_kernel<<<n_units, 256, 0, stream>>>(units, vecs, parts, it == iters - 1, inv_norm);
     e = cudaGetLastError();
   }

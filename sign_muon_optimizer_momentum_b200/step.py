@@ -258,7 +258,15 @@ class SignMuonStep:
         n_mats = len(self.shapes)
         mom = uploads(self.units * 56) + 2
         if self.norm == "spectral":
-            mom += uploads(self.units * 48) + 1 + 2 * self.spectral_iters
+            # Unit table + segment tables in one upload; per iteration the
+            # segment pass (widths that are multiples of 8 up to 4096), the
+            # row-block pass (other widths) and the reduction.
+            def al(x):
+                return -(-x // 256) * 256
+            seg_w = [(-(-r // 128)) * M for (r, c) in self.shapes if c % 8 == 0 and c <= 4096]
+            n_seg, has_rb = sum(seg_w), len(seg_w) < n_mats
+            mom += uploads(al(self.units * 48) + al(n_seg * 4) + al(513 * 4)) + 1
+            mom += self.spectral_iters * (int(n_seg > 0) + int(has_rb) + 1)
         ns_waves = 0 if self.fused_sign else self._waves(self.shapes, M, self.ws_ns.numel())
         ns = 0 if self.fused_sign else (3 * self.k if self.k > 0 else 1) * ns_waves
         vote = uploads(-(-n_mats * 64 // 256) * 256 + self.units * 8) + 1
