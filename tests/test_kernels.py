@@ -830,7 +830,10 @@ def test_signum_majority_vote_step_bit_exact(variant, w_dtype, M):
 # spectral scaling (power iteration)
 # ---------------------------------------------------------------------------
 SPEC_CASES = [([(256, 256)], 2, 5), ([(128, 384), (384, 128)], 2, 3), ([(64, 147), (33, 20)], 3, 1),
-              ([(768, 2304), (3072, 768)], 1, 5), ([(1, 1), (1, 40), (40, 1)], 2, 2)]
+              ([(768, 2304), (3072, 768)], 1, 5), ([(1, 1), (1, 40), (40, 1)], 2, 2),
+              # 4096 columns (two chunks per thread, 3-row groups, ragged last segment) and
+              # 768 columns over 8 segments whose last group is ragged (two row subsets).
+              ([(300, 4096), (1000, 768)], 2, 3)]
 
 
 def gpu_spectral(shapes, M, xs, inv, iters):
