@@ -577,15 +577,13 @@ def extra_signum(ctx, args, pk):
 
 def spectral_bytes_per_iteration(shapes, n_workers):
     """Algorithmic bytes of one power iteration: each unit's bf16 copy of M
-    read once, and its partial sums of z written and read back (one per
-    (128-row segment, row subset) for widths that are multiples of 8 up to
-    4096, else one per 32-row block), 4 B per column each."""
+    read once, and its partial sums of z written and read back (for widths
+    that are multiples of 8 up to 4096 two per 128-row segment up to 1536
+    columns and one beyond, else one per 32-row block), 4 B per column each."""
     total = 0
     for r, c in shapes:
         if c % 8 == 0 and c <= 4096:
-            nch = c // 8
-            g = min(24576 // (2 * c), 32)
-            rs = 1 if nch > 128 else min(256 // nch, g)
+            rs = 2 if c <= 1536 else 1
             parts = -(-r // 128) * rs
         else:
             parts = -(-r // 32)

@@ -185,24 +185,31 @@ constexpr int kSpecSmemCols = 8192;  // v is staged in shared memory up to this 
 constexpr int kSpecSegRows = 128;       // rows per segment
 constexpr int kSpecSlotBytes = 24576;   // shared-memory ring slot: the rows of one group
 constexpr int kSpecSlots = 4;
-constexpr int kSpecSegMaxCols = 4096;   // at most two 8-column chunks per thread of 256
+constexpr int kSpecSegMaxCols = 4096;   // at most six warps per row (below)
+constexpr int kSpecScratchBytes = 16384;  // shared memory for the end-of-segment sums of z
 constexpr int kSpecMaxGrid = 512;       // segment-pass blocks at most (two per SM)
+// The segment pass takes each row with a team of T warps, lane l of the
+// team's warp j holding the 8-column chunks 96 j + l + 32 i (i < 3) of v and
+// z in registers; the block's 8 / T teams take the rows of a group round
+// robin.
+constexpr int kSpecLaneChunks = 3;
+constexpr int kSpecTeamRows = 12;  // rows per group at most when T > 1 (15 fit 776 columns; 12 is 4 teams' multiple)
+constexpr int kSpecWarpChunks = 32 * kSpecLaneChunks;  // 96 chunks: 768 columns per warp
 __host__ __device__ inline bool spec_segmented(int cols) { return (cols & 7) == 0 && cols <= kSpecSegMaxCols; }
+__host__ __device__ inline int spec_team_warps(int cols) { return (cols / 8 + kSpecWarpChunks - 1) / kSpecWarpChunks; }
+__host__ __device__ inline int spec_teams(int cols) { return 8 / spec_team_warps(cols); }
 // Rows per group (ring slot) of a segmented unit: the most rows that fit a
-// slot, at most 32.
+// slot, at most 32, rounded down to a multiple of the teams.
 __host__ __device__ inline int spec_group_rows(int cols) {
-  const int g = kSpecSlotBytes / (2 * cols);
-  return g < 32 ? g : 32;
+  int g = kSpecSlotBytes / (2 * cols);
+  if (g > 32) g = 32;
+  const int t = spec_teams(cols);
+  return g / t * t;
 }
-// Row subsets of a segmented unit's z update: a unit of at most 128 8-column
-// chunks spreads 256 threads over (row subset, chunk) pairs; each subset
-// writes its own partial of z.
-__host__ __device__ inline int spec_zsplit(int cols) {
-  const int nch = cols / 8;
-  if (nch > 128) return 1;
-  const int rs = 256 / nch, g = spec_group_rows(cols);
-  return rs < g ? rs : g;
-}
+// Partials of z per segment of a segmented unit: each team sums z over its
+// own rows, and the block adds the teams' sums in shared memory down to two
+// (eight or four teams) or one.
+__host__ __device__ inline int spec_zsplit(int cols) { return spec_teams(cols) >= 4 ? 2 : 1; }
 
 // ---------------------------------------------------------------------------
 // Launch helpers implemented in the .cu files (all enqueue on `stream`).

@@ -818,9 +818,17 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
   return d;
 }
 // Two bf16 (low half: the even column) widened to two fp32: a bf16 is the
-// high 16 bits of the fp32 of the same value.
+// high 16 bits of the fp32 of the same value.  The pair is assembled with
+// mov.b64 {lo, hi}, so that the two halves land in a register pair directly.
 __device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
-  return ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint64_t)(w << 16);
+  uint64_t d;
+  asm("{\n\t.reg .b32 lo, hi;\n\t"
+      "shl.b32 lo, %1, 16;\n\t"
+      "and.b32 hi, %1, 0xFFFF0000;\n\t"
+      "mov.b64 %0, {lo, hi};\n\t}"
+      : "=l"(d)
+      : "r"(w));
+  return d;
 }
 
 // One block per 32 rows of one unit: y_r = x_r . v for its rows, then the
@@ -906,12 +914,21 @@ spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const f
 // G = spec_group_rows(cols) rows, one bulk copy per group (a segmented unit's
 // width is a multiple of 8, so its row stride is its width and a group is one
 // contiguous range) issued by thread 0 up to kSpecSlots groups ahead, across
-// segments: the rows are read from DRAM once, with many bytes in flight.  Per
-// group, warp w forms y_r = x_r . v for rows r = w, w + 8, ... (v staged in
-// shared memory), and after one block barrier every thread adds y_r x_r to
-// its part of z: wide units (more than 128 8-column chunks) by chunk, narrow
-// ones by (row subset, chunk), each row subset keeping a partial of its own.
-// Both products use packed f32x2 FMAs.
+// segments: the rows are read from DRAM once, with many bytes in flight.
+// A row is taken by a team of T = spec_team_warps(cols) warps (T = 1 up to
+// 768 columns); lane l of the team's warp j holds the chunks
+// c = 96 j + l + 32 i (i < 3, c < cols / 8) of v and of z in registers for
+// the whole unit, so shared memory carries only the rows, read once.  The
+// block's 8 / T teams take the rows of a group round robin.
+//   T = 1: the warp widens its chunks of the row to fp32 once, sums the dot
+//   y_r = x_r . v over its lanes and adds y_r x_r to its chunks of z at once.
+//   T > 1: each warp sums its part of the dot of each of the team's rows (at
+//   most three) over its lanes and leaves it in shared memory; after the
+//   group's barrier it adds the team's T parts and y_r x_r to its chunks of
+//   z, the rows read from the slot a second time.
+// The barrier after each group frees its slot (T = 1) or the one before.  At the end of a segment the
+// teams' sums of z are added in shared memory down to spec_zsplit(cols)
+// partials.  Both products use packed f32x2 FMAs.
 __device__ __forceinline__ void spec_mbar_init(uint32_t bar) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
 }
@@ -948,24 +965,130 @@ __device__ __forceinline__ bool spec_mbar_wait(uint32_t bar, uint32_t parity) {
     }
   }
 }
-// z (8 columns as four f32x2) += y2 * (8 bf16 at p, 16 bytes of shared memory).
-__device__ __forceinline__ void spec_axpy8(const uint8_t* p, uint64_t y2, uint64_t (&z)[4]) {
-  const uint4 raw = *reinterpret_cast<const uint4*>(p);
-  z[0] = fma_f32x2(bf16x2_to_f32x2(raw.x), y2, z[0]);
-  z[1] = fma_f32x2(bf16x2_to_f32x2(raw.y), y2, z[1]);
-  z[2] = fma_f32x2(bf16x2_to_f32x2(raw.z), y2, z[2]);
-  z[3] = fma_f32x2(bf16x2_to_f32x2(raw.w), y2, z[3]);
+constexpr uint64_t kSpecOne2 = 0x3F8000003F800000ull;  // (1.0f, 1.0f)
+// Eight bf16 (raw) widened to eight floats (four f32x2).
+__device__ __forceinline__ void spec_widen8(const uint4& x, uint64_t (&w)[4]) {
+  w[0] = bf16x2_to_f32x2(x.x);
+  w[1] = bf16x2_to_f32x2(x.y);
+  w[2] = bf16x2_to_f32x2(x.z);
+  w[3] = bf16x2_to_f32x2(x.w);
+}
+// Packed sum of the dot of eight widened values with eight floats of v.
+__device__ __forceinline__ uint64_t spec_dot8(const uint64_t (&w)[4], const uint64_t (&v)[4]) {
+  uint64_t a = fma_f32x2(w[0], v[0], 0ull);
+  uint64_t b = fma_f32x2(w[1], v[1], 0ull);
+  a = fma_f32x2(w[2], v[2], a);
+  b = fma_f32x2(w[3], v[3], b);
+  return fma_f32x2(b, kSpecOne2, a);  // a + b
+}
+// z (8 columns as four f32x2) += y2 * w (eight widened values).
+__device__ __forceinline__ void spec_axpy8(const uint64_t (&w)[4], uint64_t y2, uint64_t (&z)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) z[i] = fma_f32x2(w[i], y2, z[i]);
+}
+__device__ __forceinline__ float spec_hsum(uint64_t a) {
+  return __uint_as_float((uint32_t)a) + __uint_as_float((uint32_t)(a >> 32));
+}
+__device__ __forceinline__ uint64_t spec_splat(float y) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(d) : "f"(y));
+  return d;
+}
+// 8 floats (16-byte aligned) as four f32x2, loaded, stored or added.
+__device__ __forceinline__ void spec_ld8(const float* p, uint64_t (&v)[4]) {
+  const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(p);
+  const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(p + 4);
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = b.x;
+  v[3] = b.y;
+}
+__device__ __forceinline__ void spec_st8(float* p, const uint64_t (&v)[4]) {
+  *reinterpret_cast<ulonglong2*>(p) = make_ulonglong2(v[0], v[1]);
+  *reinterpret_cast<ulonglong2*>(p + 4) = make_ulonglong2(v[2], v[3]);
+}
+__device__ __forceinline__ void spec_add8(const float* p, uint64_t (&z)[4]) {
+  uint64_t t[4];
+  spec_ld8(p, t);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) z[i] = fma_f32x2(t[i], kSpecOne2, z[i]);
+}
+
+// T > 1, before the group barrier: warp j of team `team` sums its part of
+// the dot of each of the team's kRpt rows r = team + teams k over its lanes
+// and lane 0 leaves it in rd[r][j].  In a short last group (kFull false) a
+// missing row reads the group's first row and is not stored.
+template <int kRpt, bool kFull>
+__device__ __forceinline__ void spec_team_dots(const uint8_t* base, int row_bytes, int gn, int team, int teams, int j,
+                                               int lane, const int (&off)[kSpecLaneChunks],
+                                               const uint64_t (&v)[kSpecLaneChunks][4], float (*rd)[8]) {
+  float pd[kRpt];
+#pragma unroll
+  for (int k = 0; k < kRpt; ++k) {
+    const int r = team + teams * k;
+    const bool in = kFull || r < gn;
+    const uint8_t* row = base + (in ? r : 0) * row_bytes;
+    uint64_t s = 0ull;
+#pragma unroll
+    for (int i = 0; i < kSpecLaneChunks; ++i) {
+      uint64_t w[4];
+      spec_widen8(*reinterpret_cast<const uint4*>(row + off[i]), w);
+      s = fma_f32x2(spec_dot8(w, v[i]), kSpecOne2, s);
+    }
+    pd[k] = spec_hsum(s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int k = 0; k < kRpt; ++k) pd[k] += __shfl_xor_sync(0xffffffffu, pd[k], o);
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < kRpt; ++k)
+      if (kFull || team + teams * k < gn) rd[team + teams * k][j] = pd[k];
+  }
+}
+// T > 1, after the group barrier: y_r = the team's T parts (in order), and
+// z += y_r x_r over the lane's chunks, the rows read from the slot again.
+template <int kRpt, bool kFull>
+__device__ __forceinline__ void spec_team_update(const uint8_t* base, int row_bytes, int gn, int team, int teams, int T,
+                                                 const int (&off)[kSpecLaneChunks], const float (*rd)[8],
+                                                 uint64_t (&z)[kSpecLaneChunks][4]) {
+#pragma unroll
+  for (int k = 0; k < kRpt; ++k) {
+    const int r = team + teams * k;
+    const bool in = kFull || r < gn;
+    const int rr = in ? r : 0;
+    const float4 a = *reinterpret_cast<const float4*>(&rd[rr][0]);
+    const float4 b = *reinterpret_cast<const float4*>(&rd[rr][4]);
+    // The unused entries are selected away, not added.
+    float y = a.x + a.y;
+    y += T > 2 ? a.z : 0.f;
+    y += T > 3 ? a.w : 0.f;
+    y += T > 4 ? b.x : 0.f;
+    y += T > 5 ? b.y : 0.f;
+    const uint64_t y2 = spec_splat(in ? y : 0.f);
+    const uint8_t* row = base + rr * row_bytes;
+#pragma unroll
+    for (int i = 0; i < kSpecLaneChunks; ++i) {
+      uint64_t w[4];
+      spec_widen8(*reinterpret_cast<const uint4*>(row + off[i]), w);
+      spec_axpy8(w, y2, z[i]);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(256, 2)
 spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __restrict__ seg_unit,
                         const int32_t* __restrict__ blk_seg, const float* __restrict__ vecs,
                         float* __restrict__ parts, uint32_t* __restrict__ err) {
-  // Ring of kSpecSlots slots, then v (kSpecSegMaxCols floats).
+  constexpr int kLC = kSpecLaneChunks;
+  // Ring of kSpecSlots slots, then the scratch for the sums of z.
   extern __shared__ __align__(1024) uint8_t spec_ring[];
-  float* vs = reinterpret_cast<float*>(spec_ring + kSpecSlots * kSpecSlotBytes);
+  float* scratch = reinterpret_cast<float*>(spec_ring + kSpecSlots * kSpecSlotBytes);
   __shared__ __align__(8) uint64_t full[kSpecSlots];
-  __shared__ float ys[2][32];  // y of the group, double-buffered by group parity
+  // T > 1: the warps' parts of the dots, by group parity.  The static shared
+  // memory stays within 1 KB, so that two blocks fit an SM.
+  __shared__ __align__(16) float red[2][kSpecTeamRows][8];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(spec_ring));
   const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(full));
@@ -997,7 +1120,6 @@ spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __res
   };
   // Loads the next group into its slot, which no thread still reads.
   auto p_issue = [&]() {
-    if (p_seg >= seg_end) return;
     const int gn = min(p_g, p_nrows - p_row);
     const int slot = p_idx % kSpecSlots;
     const uint32_t bytes = (uint32_t)gn * (uint32_t)p_cols * 2u;
@@ -1015,21 +1137,24 @@ spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __res
   };
   if (tid == 0) {
     p_open();
-    for (int i = 0; i < kSpecSlots; ++i) p_issue();
+    for (int i = 0; i < kSpecSlots && p_seg < seg_end; ++i) p_issue();
   }
 
   int g = 0;  // groups consumed by this block
   bool failed = false;
   int c_unit = -1, c_next = seg_first < seg_end ? __ldg(seg_unit + seg_first) : -1;
-  int cols = 8, G = 1, rows = 0, seg_begin = 0, nch = 1, rs = 1, q = 0, c0 = 0;
+  int cols = 8, G = 8, rows = 0, seg_begin = 0, nch = 1, T = 1, teams = 8, team = 0, cb = 0, rpt = 1;
   int64_t part_off = 0;
-  bool own0 = false, own1 = false;
+  bool act = true;  // this warp belongs to a team (8 / T teams of T warps)
+  // The lane's chunks: byte offset in a row and v.  A chunk past the row's
+  // end reads the row's last chunk against v = 0, so that the hot loops take
+  // no branch per chunk; its z is never written.
+  int off[kLC];
+  uint64_t v[kLC][4], z[kLC][4];
   for (int seg = seg_first; seg < seg_end && !failed; ++seg) {
     const int ui = c_next;
     c_next = seg + 1 < seg_end ? __ldg(seg_unit + seg + 1) : -1;
     if (ui != c_unit) {
-      // Every thread is past the last dot phase of the previous unit (its
-      // group's barrier), so v can be replaced.
       c_unit = ui;
       cols = __ldg(&units[ui].cols);
       rows = __ldg(&units[ui].rows);
@@ -1037,76 +1162,152 @@ spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __res
       part_off = __ldg(&units[ui].part_off);
       G = spec_group_rows(cols);
       nch = cols >> 3;
-      rs = spec_zsplit(cols);
-      if (nch > 128) {
-        q = 0; c0 = tid; own0 = tid < nch; own1 = tid + 256 < nch;
-      } else {
-        q = tid / nch; c0 = tid - q * nch; own0 = q < rs; own1 = false;
-      }
+      T = spec_team_warps(cols);
+      teams = 8 / T;
+      team = warp / T;
+      act = warp < teams * T;
+      cb = (warp - team * T) * kSpecWarpChunks + lane;
+      rpt = G / teams;
       const float* vg = vecs + __ldg(&units[ui].v_off);
-      for (int j = tid; j < cols; j += 256) vs[j] = vg[j];
-      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < kLC; ++i) {
+        const int c = cb + 32 * i;
+        const bool in = act && c < nch;
+        off[i] = 16 * (in ? c : nch - 1);
+        if (in) {
+          spec_ld8(vg + 8 * c, v[i]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[i][j] = 0ull;
+        }
+      }
     }
     const int row0 = (seg - seg_begin) * kSpecSegRows;
     const int nrows = min(kSpecSegRows, rows - row0);
     const int row_bytes = 2 * cols;
-    uint64_t z0[4] = {0, 0, 0, 0}, z1[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < kLC; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) z[i][j] = 0ull;
     for (int gr0 = 0; gr0 < nrows; gr0 += G, ++g) {
       const int gn = min(G, nrows - gr0);
       const int slot = g % kSpecSlots;
       const bool ok = spec_mbar_wait(bar0 + 8 * slot, (uint32_t)((g / kSpecSlots) & 1));
       const uint8_t* base = spec_ring + slot * kSpecSlotBytes;
-      float* yb = ys[g & 1];
-      if (ok) {
-        for (int r = warp; r < gn; r += 8) {
-          const uint8_t* row = base + r * row_bytes;
-          uint64_t acc2 = 0;
-          for (int c = lane; c < nch; c += 32) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(row + 16 * c);
-            const ulonglong2 va = *reinterpret_cast<const ulonglong2*>(vs + 8 * c);
-            const ulonglong2 vb = *reinterpret_cast<const ulonglong2*>(vs + 8 * c + 4);
-            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.x), va.x, acc2);
-            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.y), va.y, acc2);
-            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.z), vb.x, acc2);
-            acc2 = fma_f32x2(bf16x2_to_f32x2(raw.w), vb.y, acc2);
-          }
-          float acc = __uint_as_float((uint32_t)acc2) + __uint_as_float((uint32_t)(acc2 >> 32));
+      float (*rd)[8] = red[g & 1];
+      // The group barrier (T is the same for the whole block, so all threads
+      // take the same branch).  Past it every thread is done with the slots of
+      // the groups before `done`, which are refilled.
+      auto release = [&](int done) {
+        if (__syncthreads_or(!ok)) return false;
+        if (tid == 0)
+          while (p_idx < done + kSpecSlots && p_seg < seg_end) p_issue();
+        return true;
+      };
+      if (T == 1) {
+        if (ok) {
+          for (int r = warp; r < gn; r += 8) {
+            const uint8_t* row = base + r * row_bytes;
+            uint64_t xw[kLC][4];
+            spec_widen8(*reinterpret_cast<const uint4*>(row + off[0]), xw[0]);
+            uint64_t s = spec_dot8(xw[0], v[0]);
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          if (lane == 0) yb[r] = acc;
+            for (int i = 1; i < kLC; ++i) {
+              spec_widen8(*reinterpret_cast<const uint4*>(row + off[i]), xw[i]);
+              s = fma_f32x2(spec_dot8(xw[i], v[i]), kSpecOne2, s);
+            }
+            float y = spec_hsum(s);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
+            const uint64_t y2 = spec_splat(y);
+#pragma unroll
+            for (int i = 0; i < kLC; ++i) spec_axpy8(xw[i], y2, z[i]);
+          }
         }
-      }
-      // Every thread is past the previous group here: its slot is free.
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-      if (tid == 0 && g > 0) p_issue();
-      if (nch > 128) {
-        for (int r = 0; r < gn; ++r) {
-          const uint32_t yu = __float_as_uint(yb[r]);
-          const uint64_t y2 = ((uint64_t)yu << 32) | yu;
-          const uint8_t* row = base + r * row_bytes;
-          if (own0) spec_axpy8(row + 16 * c0, y2, z0);
-          if (own1) spec_axpy8(row + 16 * (c0 + 256), y2, z1);
+        if (!release(g + 1)) {  // this group's slot is free too
+          failed = true;
+          break;
         }
-      } else if (own0) {
-        for (int r = q; r < gn; r += rs) {
-          const uint32_t yu = __float_as_uint(yb[r]);
-          spec_axpy8(base + r * row_bytes + 16 * c0, ((uint64_t)yu << 32) | yu, z0);
+      } else {
+        // A team takes rpt = G / teams rows of a group (2 or 3 when T > 1).
+        const bool full = gn == G;
+        const int j = warp - team * T;
+        if (ok && act) {
+          if (rpt == 3) {
+            if (full) spec_team_dots<3, true>(base, row_bytes, gn, team, teams, j, lane, off, v, rd);
+            else spec_team_dots<3, false>(base, row_bytes, gn, team, teams, j, lane, off, v, rd);
+          } else {
+            if (full) spec_team_dots<2, true>(base, row_bytes, gn, team, teams, j, lane, off, v, rd);
+            else spec_team_dots<2, false>(base, row_bytes, gn, team, teams, j, lane, off, v, rd);
+          }
+        }
+        if (!release(g)) {  // the z update below still reads this group's rows
+          failed = true;
+          break;
+        }
+        if (act) {
+          if (rpt == 3) {
+            if (full) spec_team_update<3, true>(base, row_bytes, gn, team, teams, T, off, rd, z);
+            else spec_team_update<3, false>(base, row_bytes, gn, team, teams, T, off, rd, z);
+          } else {
+            if (full) spec_team_update<2, true>(base, row_bytes, gn, team, teams, T, off, rd, z);
+            else spec_team_update<2, false>(base, row_bytes, gn, team, teams, T, off, rd, z);
+          }
         }
       }
     }
     if (failed) break;
-    // This segment's partial of z (one per row subset for narrow units).
-    float* part = parts + part_off + ((int64_t)(seg - seg_begin) * rs + q) * cols;
-    if (own0) {
-      *reinterpret_cast<ulonglong2*>(part + 8 * c0) = make_ulonglong2(z0[0], z0[1]);
-      *reinterpret_cast<ulonglong2*>(part + 8 * c0 + 4) = make_ulonglong2(z0[2], z0[3]);
+    // This segment's partials of z: the teams' sums added pairwise in the
+    // scratch (slot s at scratch + s * cols) down to spec_zsplit(cols).  The
+    // barriers below are reached by every thread (the group loop ends for all
+    // of them together), and the scratch is next written after at least one
+    // more group barrier.
+    const int64_t seg_part = part_off + (int64_t)(seg - seg_begin) * spec_zsplit(cols) * cols;
+    auto put = [&](int s) {
+#pragma unroll
+      for (int i = 0; i < kLC; ++i)
+        if (cb + 32 * i < nch) spec_st8(scratch + s * cols + 8 * (cb + 32 * i), z[i]);
+    };
+    auto take = [&](int s) {
+#pragma unroll
+      for (int i = 0; i < kLC; ++i)
+        if (cb + 32 * i < nch) spec_add8(scratch + s * cols + 8 * (cb + 32 * i), z[i]);
+    };
+    int out = -1;  // the partial this team writes, if any
+    if (teams == 8) {
+      if (team >= 4) put(team - 4);
+      __syncthreads();
+      if (team < 4) {
+        take(team);
+        if (team >= 2) put(team);
+      }
+      __syncthreads();
+      if (team < 2) {
+        take(team + 2);
+        out = team;
+      }
+    } else if (teams == 4) {
+      if (team >= 2) put(team - 2);
+      __syncthreads();
+      if (team < 2) {
+        take(team);
+        out = team;
+      }
+    } else if (teams == 2) {
+      if (act && team == 1) put(0);
+      __syncthreads();
+      if (team == 0) {
+        take(0);
+        out = 0;
+      }
+    } else if (team == 0 && act) {
+      out = 0;
     }
-    if (own1) {
-      *reinterpret_cast<ulonglong2*>(part + 8 * (c0 + 256)) = make_ulonglong2(z1[0], z1[1]);
-      *reinterpret_cast<ulonglong2*>(part + 8 * (c0 + 256) + 4) = make_ulonglong2(z1[2], z1[3]);
+    if (out >= 0) {
+      float* part = parts + seg_part + (int64_t)out * cols;
+#pragma unroll
+      for (int i = 0; i < kLC; ++i)
+        if (cb + 32 * i < nch) spec_st8(part + 8 * (cb + 32 * i), z[i]);
     }
   }
   if (failed && tid == 0) {
@@ -1117,20 +1318,78 @@ spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __res
   }
 }
 
-// One block per unit: z = sum of the row-block partials (fixed order),
-// v <- z / ||z||; after the last iteration inv_norm = 1 / (sqrt(||z||) + eps).
+// One block per unit: z = sum of the partials (a fixed order: partial p
+// goes to accumulator p % 8, the eight added pairwise at the end, so that
+// eight loads are in flight per column), v <- z / ||z||; after the last
+// iteration inv_norm = 1 / (sqrt(||z||) + eps).  Widths that are multiples of
+// 4 are summed four columns per load.
 __global__ void __launch_bounds__(256)
 spectral_reduce_kernel(const SpecUnit* __restrict__ units, float* __restrict__ vecs, const float* __restrict__ parts,
                        int last, float* __restrict__ inv_norm) {
   const SpecUnit u = units[blockIdx.x];
   float* v = vecs + u.v_off;
   const float* part = parts + u.part_off;
+  const int np = u.n_parts;
   double ss = 0.0;
-  for (int j = threadIdx.x; j < u.cols; j += blockDim.x) {
-    float z = 0.f;
-    for (int rb = 0; rb < u.n_parts; ++rb) z += part[(int64_t)rb * u.cols + j];
-    v[j] = z;
-    ss += (double)z * (double)z;
+  if ((u.cols & 3) == 0) {
+    const int c4 = u.cols >> 2;
+    for (int j = threadIdx.x; j < c4; j += blockDim.x) {
+      const float4* p4 = reinterpret_cast<const float4*>(part) + j;
+      float4 acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      int rb = 0;
+      for (; rb + 8 <= np; rb += 8) {
+        float4 t[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) t[q] = __ldg(p4 + (int64_t)(rb + q) * c4);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          acc[q].x += t[q].x;
+          acc[q].y += t[q].y;
+          acc[q].z += t[q].z;
+          acc[q].w += t[q].w;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 7; ++q)
+        if (rb + q < np) {
+          const float4 t = __ldg(p4 + (int64_t)(rb + q) * c4);
+          acc[q].x += t.x;
+          acc[q].y += t.y;
+          acc[q].z += t.z;
+          acc[q].w += t.w;
+        }
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int q = 0; q < w; ++q) {
+          acc[q].x += acc[q + w].x;
+          acc[q].y += acc[q + w].y;
+          acc[q].z += acc[q + w].z;
+          acc[q].w += acc[q + w].w;
+        }
+      reinterpret_cast<float4*>(v)[j] = acc[0];
+      ss += (double)acc[0].x * acc[0].x + (double)acc[0].y * acc[0].y + (double)acc[0].z * acc[0].z +
+            (double)acc[0].w * acc[0].w;
+    }
+  } else {
+    for (int j = threadIdx.x; j < u.cols; j += blockDim.x) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int rb = 0;
+      for (; rb + 8 <= np; rb += 8)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += __ldg(part + (int64_t)(rb + q) * u.cols + j);
+#pragma unroll
+      for (int q = 0; q < 7; ++q)
+        if (rb + q < np) acc[q] += __ldg(part + (int64_t)(rb + q) * u.cols + j);
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int q = 0; q < w; ++q) acc[q] += acc[q + w];
+      v[j] = acc[0];
+      ss += (double)acc[0] * (double)acc[0];
+    }
   }
   __shared__ double red[256];
   red[threadIdx.x] = ss;
@@ -1148,7 +1407,7 @@ spectral_reduce_kernel(const SpecUnit* __restrict__ units, float* __restrict__ v
 cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, const int32_t* seg_unit,
                             const int32_t* blk_seg, int seg_grid, float* vecs, float* parts, int iters,
                             float* inv_norm, uint32_t* err, cudaStream_t stream) {
-  constexpr int kSegSmem = kSpecSlots * kSpecSlotBytes + kSpecSegMaxCols * 4;
+  constexpr int kSegSmem = kSpecSlots * kSpecSlotBytes + kSpecScratchBytes;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

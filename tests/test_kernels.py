@@ -831,9 +831,13 @@ def test_signum_majority_vote_step_bit_exact(variant, w_dtype, M):
 # ---------------------------------------------------------------------------
 SPEC_CASES = [([(256, 256)], 2, 5), ([(128, 384), (384, 128)], 2, 3), ([(64, 147), (33, 20)], 3, 1),
               ([(768, 2304), (3072, 768)], 1, 5), ([(1, 1), (1, 40), (40, 1)], 2, 2),
-              # 4096 columns (two chunks per thread, 3-row groups, ragged last segment) and
-              # 768 columns over 8 segments whose last group is ragged (two row subsets).
-              ([(300, 4096), (1000, 768)], 2, 3)]
+              # 4096 columns (a team of six warps, 3-row groups, ragged last segment) and 768
+              # columns over 8 segments whose last group is ragged (one warp per row).
+              ([(300, 4096), (1000, 768)], 2, 3),
+              # Teams of two (776, 1536), three (2056: 257 chunks, the last one alone in its
+              # warp), four (2568) and five warps (3840); the 65- and 33-row units end in a
+              # group shorter than a team round.
+              ([(200, 1536), (70, 2056), (130, 776), (65, 2568), (33, 3840)], 2, 2)]
 
 
 def gpu_spectral(shapes, M, xs, inv, iters):
