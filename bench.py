@@ -154,6 +154,14 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.skip = 0
+
+    def mark(self):
+        """Samples taken so far (before the timed region) are left out."""
+        try:
+            self.skip = len(open(self.path).read().splitlines())
+        except Exception:
+            self.skip = 0
 
     def start(self):
         try:
@@ -173,7 +181,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        rows = [ln.split(",") for ln in open(self.path).read().splitlines() if ln.strip()]
+        rows = [ln.split(",") for ln in open(self.path).read().splitlines()[self.skip:] if ln.strip()]
         os.unlink(self.path)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -450,6 +458,7 @@ def time_workload(ctx, wl, args, *, norm, steps, warmup, graph=False, exchange=F
     if sampler:
         sampler.start()
         time.sleep(0.3)
+        sampler.mark()
     ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ctx.barrier()
@@ -479,15 +488,27 @@ def time_workload(ctx, wl, args, *, norm, steps, warmup, graph=False, exchange=F
         from sign_muon_optimizer_momentum_b200 import _lib as L
         xp = [x.data_ptr() for x in opt.x]
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 20
-        for r in range(reps + 3):
-            if r == 3:
-                a.record(stream)
+        reps = 200
+
+        def spectral():
             L.signmuon_spectral_norm(opt.shapes, opt.n_workers, xp, opt.spectral_iters, opt.inv_norm.data_ptr(),
                                      opt.ws_spec.data_ptr(), opt.ws_spec.numel(), s_ptr)
+
+        for _ in range(3):
+            spectral()
+        ctx.barrier()
+        sp_sampler = ClockSampler(ctx.local) if (clocks and rank == 0) else None
+        if sp_sampler:
+            sp_sampler.start()
+            time.sleep(0.3)
+            sp_sampler.mark()
+        a.record(stream)
+        for _ in range(reps):
+            spectral()
         b.record(stream)
         ctx.barrier()
         out["spectral_ms"] = ctx.max_over_ranks(a.elapsed_time(b)) / reps
+        out["spectral_clocks"] = sp_sampler.stop() if sp_sampler else None
     if e2e:
         # End to end through the public step with HOST buffers: each step's
         # gradients come from pinned host memory and the updated weights go
@@ -569,10 +590,10 @@ def extra_signum(ctx, args, pk):
     momentum + sign pass, then the vote + update."""
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
     wl = syn.WORKLOADS["signum_nanogpt_small"]
-    r = time_workload(ctx, wl, args, norm="frobenius", steps=50, warmup=5)
+    r = time_workload(ctx, wl, args, norm="frobenius", steps=300, warmup=5, clocks=True)
     return {"workload": wl.name, "config": workload_config(wl), "metric": METRIC, "value": r["value"], "unit": UNIT,
-            "ms_per_step": r["ms_per_step"], "steps": 50, "warmup": 5, "phases_ms": r["phases_ms"],
-            "roofline": momentum_roofline(wl, r["opt"], r["phases_ms"]["momentum"], pk)}
+            "ms_per_step": r["ms_per_step"], "steps": 300, "warmup": 5, "phases_ms": r["phases_ms"],
+            "roofline": momentum_roofline(wl, r["opt"], r["phases_ms"]["momentum"], pk), "clocks": r["clocks"]}
 
 
 def spectral_bytes_per_iteration(shapes, n_workers):
@@ -598,15 +619,16 @@ def extra_spectral(ctx, args, pk):
     partial sums of z written and read back."""
     from sign_muon_optimizer_momentum_b200 import synthetic as syn
     wl = syn.WORKLOADS["nanogpt_small"]
-    r = time_workload(ctx, wl, args, norm="spectral", steps=20, warmup=3)
+    r = time_workload(ctx, wl, args, norm="spectral", steps=30, warmup=3, clocks=True)
     iters = r["opt"].spectral_iters
     per_iter = spectral_bytes_per_iteration(wl.shapes, wl.n_workers)
     gbytes = iters * per_iter
     achieved = gbytes / (r["spectral_ms"] / 1e3) / 1e9
     kernel = "spectral_segment_kernel"
     return {"workload": wl.name, "config": dict(workload_config(wl), norm="spectral", spectral_iters=iters),
-            "metric": METRIC, "value": r["value"], "unit": UNIT, "ms_per_step": r["ms_per_step"], "steps": 20,
+            "metric": METRIC, "value": r["value"], "unit": UNIT, "ms_per_step": r["ms_per_step"], "steps": 30,
             "warmup": 3, "phases_ms": dict(r["phases_ms"], spectral_alone=r["spectral_ms"]),
+            "clocks": r["clocks"], "clocks_spectral_alone": r["spectral_clocks"],
             "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                          "traffic": captured_traffic(kernel, wl.name),
@@ -644,6 +666,18 @@ def run_gpu(args, wl):
     _build.build()
     ctx = Ctx(world, rank, local, torch.device("cuda", torch.cuda.current_device()))
     pk = peaks()
+    extras = {}
+    if wl.name == DEFAULT_CONFIG and not args.no_extras and not args.exchange:
+        # Rows measured beside the headline workload, each with its roofline
+        # and the clocks sampled during its own timed region.  They run first:
+        # after the seconds-long headline run the power-capped clock is lower
+        # for a while, which would slow the short, clock-sensitive rows.
+        extras["vote_sweep"] = time_vote_sweep(ctx, 1 << 30, 16, "f32", steps=200, warmup=5, clocks=True)
+        torch.cuda.empty_cache()
+        extras["signum"] = extra_signum(ctx, args, pk)
+        torch.cuda.empty_cache()
+        extras["spectral"] = extra_spectral(ctx, args, pk)
+        torch.cuda.empty_cache()
     r = time_workload(ctx, wl, args, norm=args.norm, steps=args.steps, warmup=args.warmup, graph=args.graph,
                       exchange=args.exchange, e2e=not args.no_e2e, clocks=True)
     if wl.ns_iters > 0:
@@ -664,14 +698,7 @@ def run_gpu(args, wl):
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl)
-    if wl.name == DEFAULT_CONFIG and not args.no_extras and not args.exchange:
-        # Rows measured beside the headline workload, each with its roofline.
-        result["vote_sweep"] = time_vote_sweep(ctx, 1 << 30, 16, "f32", steps=20, warmup=5)
-        torch.cuda.empty_cache()
-        result["signum"] = extra_signum(ctx, args, pk)
-        torch.cuda.empty_cache()
-        result["spectral"] = extra_spectral(ctx, args, pk)
-        torch.cuda.empty_cache()
+    result.update(extras)
     if pg:
         dist.barrier()
         dist.destroy_process_group()
@@ -717,6 +744,7 @@ def time_vote_sweep(ctx, P, M, w_dtype, steps, warmup, clocks=False):
     if sampler:
         sampler.start()
         time.sleep(0.3)
+        sampler.mark()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(steps):
