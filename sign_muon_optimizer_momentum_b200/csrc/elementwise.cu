@@ -918,17 +918,17 @@ spectral_rowpass_kernel(const SpecUnit* __restrict__ units, int n_units, const f
 // A row is taken by a team of T = spec_team_warps(cols) warps (T = 1 up to
 // 768 columns); lane l of the team's warp j holds the chunks
 // c = 96 j + l + 32 i (i < 3, c < cols / 8) of v and of z in registers for
-// the whole unit, so shared memory carries only the rows, read once.  The
-// block's 8 / T teams take the rows of a group round robin.
+// the whole unit, so shared memory carries only the rows.  The block's
+// 8 / T teams take the rows of a group round robin.
 //   T = 1: the warp widens its chunks of the row to fp32 once, sums the dot
 //   y_r = x_r . v over its lanes and adds y_r x_r to its chunks of z at once.
 //   T > 1: each warp sums its part of the dot of each of the team's rows (at
 //   most three) over its lanes and leaves it in shared memory; after the
 //   group's barrier it adds the team's T parts and y_r x_r to its chunks of
 //   z, the rows read from the slot a second time.
-// The barrier after each group frees its slot (T = 1) or the one before.  At the end of a segment the
-// teams' sums of z are added in shared memory down to spec_zsplit(cols)
-// partials.  Both products use packed f32x2 FMAs.
+// The barrier after each group frees its slot (T = 1) or the one before.
+// At the end of a segment the teams' sums of z are added in shared memory
+// down to spec_zsplit(cols) partials.  Both products use packed f32x2 FMAs.
 __device__ __forceinline__ void spec_mbar_init(uint32_t bar) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
 }

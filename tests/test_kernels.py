@@ -836,8 +836,8 @@ SPEC_CASES = [([(256, 256)], 2, 5), ([(128, 384), (384, 128)], 2, 3), ([(64, 147
               ([(300, 4096), (1000, 768)], 2, 3),
               # Teams of two (776, 1536), three (2056: 257 chunks, the last one alone in its
               # warp), four (2568) and five warps (3840); the 65- and 33-row units end in a
-              # group shorter than a team round.
-              ([(200, 1536), (70, 2056), (130, 776), (65, 2568), (33, 3840)], 2, 2)]
+              # group shorter than a team round.  8 columns: one chunk, lanes 1-31 idle.
+              ([(200, 1536), (70, 2056), (130, 776), (65, 2568), (33, 3840), (9, 8)], 2, 2)]
 
 
 def gpu_spectral(shapes, M, xs, inv, iters):
