@@ -387,6 +387,20 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
     blk_seg[b] = sgi;
   }
   if (seg_grid > 0) blk_seg[seg_grid] = segs;
+  // SIGNMUON_SPECTRAL_INJECT_WAIT_TIMEOUT_US=<n> (1 <= n <= 2000000): fault
+  // injection for testing the bounded waits.  The segment pass loads no rows
+  // and every block gives up waiting for them after n microseconds, recording
+  // a wait-timeout code in the workspace; the estimates are then meaningless.
+  // Unset (the default): full 2 s limit, normal operation.
+  uint64_t wait_limit_ns = kWaitTimeoutNs;
+  int withhold = 0;
+  if (const char* inj = getenv("SIGNMUON_SPECTRAL_INJECT_WAIT_TIMEOUT_US")) {
+    const long us = strtol(inj, nullptr, 10);
+    if (us >= 1 && us <= 2000000) {
+      wait_limit_ns = (uint64_t)us * 1000ull;
+      withhold = 1;
+    }
+  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t e = upload_bytes(ws + lay.units, blob.data(), blob.size(), s);
   if (e == cudaSuccess)
@@ -394,7 +408,7 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
                         reinterpret_cast<const int32_t*>(ws + lay.seg_unit),
                         reinterpret_cast<const int32_t*>(ws + lay.blk_seg), seg_grid,
                         reinterpret_cast<float*>(ws + lay.vecs), reinterpret_cast<float*>(ws + lay.parts), iters,
-                        inv_norm, reinterpret_cast<uint32_t*>(ws), s);
+                        inv_norm, reinterpret_cast<uint32_t*>(ws), wait_limit_ns, withhold, s);
   return cuda_status(e);
 }
 

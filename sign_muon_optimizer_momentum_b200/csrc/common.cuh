@@ -231,7 +231,8 @@ cudaError_t launch_ns_gemm(const NsLaunch& p, cudaStream_t stream);
 // pass's block b takes segments [blk_seg[b], blk_seg[b + 1]) of seg_grid blocks.
 cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, const int32_t* seg_unit,
                             const int32_t* blk_seg, int seg_grid, float* vecs, float* parts, int iters,
-                            float* inv_norm, uint32_t* err, cudaStream_t stream);
+                            float* inv_norm, uint32_t* err, uint64_t wait_limit_ns, int withhold,
+                            cudaStream_t stream);
 cudaError_t launch_ns_identity(const NsUnit* units, int n_units, int64_t max_elems, int out_kind,
                                int w_dtype, float eta, cudaStream_t stream);
 

@@ -951,8 +951,8 @@ __device__ __forceinline__ bool spec_mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits for the phase of `bar` with this parity; false after kWaitTimeoutNs.
-__device__ __forceinline__ bool spec_mbar_wait(uint32_t bar, uint32_t parity) {
+// Waits for the phase of `bar` with this parity; false after limit_ns.
+__device__ __forceinline__ bool spec_mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (spec_mbar_test(bar, parity)) return true;
   uint64_t t0;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
@@ -961,7 +961,7 @@ __device__ __forceinline__ bool spec_mbar_wait(uint32_t bar, uint32_t parity) {
     if ((n & 63) == 0) {
       uint64_t t;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-      if (t - t0 > kWaitTimeoutNs) return false;
+      if (t - t0 > limit_ns) return false;
     }
   }
 }
@@ -1080,7 +1080,10 @@ __device__ __forceinline__ void spec_team_update(const uint8_t* base, int row_by
 __global__ void __launch_bounds__(256, 2)
 spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __restrict__ seg_unit,
                         const int32_t* __restrict__ blk_seg, const float* __restrict__ vecs,
-                        float* __restrict__ parts, uint32_t* __restrict__ err) {
+                        float* __restrict__ parts, uint32_t* __restrict__ err, uint64_t wait_ns, int withhold) {
+  // withhold (fault injection, for testing the bounded waits): no row is
+  // loaded, so every block's first wait runs out after wait_ns and the block
+  // records kErrWaitTimeoutSpectral and returns.
   constexpr int kLC = kSpecLaneChunks;
   // Ring of kSpecSlots slots, then the scratch for the sums of z.
   extern __shared__ __align__(1024) uint8_t spec_ring[];
@@ -1137,6 +1140,7 @@ spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __res
   };
   if (tid == 0) {
     p_open();
+    if (withhold) p_seg = seg_end;  // nothing is ever loaded
     for (int i = 0; i < kSpecSlots && p_seg < seg_end; ++i) p_issue();
   }
 
@@ -1192,7 +1196,7 @@ spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __res
     for (int gr0 = 0; gr0 < nrows; gr0 += G, ++g) {
       const int gn = min(G, nrows - gr0);
       const int slot = g % kSpecSlots;
-      const bool ok = spec_mbar_wait(bar0 + 8 * slot, (uint32_t)((g / kSpecSlots) & 1));
+      const bool ok = spec_mbar_wait(bar0 + 8 * slot, (uint32_t)((g / kSpecSlots) & 1), wait_ns);
       const uint8_t* base = spec_ring + slot * kSpecSlotBytes;
       float (*rd)[8] = red[g & 1];
       // The group barrier (T is the same for the whole block, so all threads
@@ -1314,7 +1318,8 @@ spectral_segment_kernel(const SpecUnit* __restrict__ units, const int32_t* __res
     // Record the error, then wait (bounded) for every copy still in flight
     // before the block's shared memory is released.
     atomicCAS(err, 0u, (uint32_t)kErrWaitTimeoutSpectral);
-    for (int i = g; i < p_idx; ++i) (void)spec_mbar_wait(bar0 + 8 * (i % kSpecSlots), (uint32_t)((i / kSpecSlots) & 1));
+    for (int i = g; i < p_idx; ++i)
+      (void)spec_mbar_wait(bar0 + 8 * (i % kSpecSlots), (uint32_t)((i / kSpecSlots) & 1), wait_ns);
   }
 }
 
@@ -1406,7 +1411,8 @@ spectral_reduce_kernel(const SpecUnit* __restrict__ units, float* __restrict__ v
 
 cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_blocks, const int32_t* seg_unit,
                             const int32_t* blk_seg, int seg_grid, float* vecs, float* parts, int iters,
-                            float* inv_norm, uint32_t* err, cudaStream_t stream) {
+                            float* inv_norm, uint32_t* err, uint64_t wait_limit_ns, int withhold,
+                            cudaStream_t stream) {
   constexpr int kSegSmem = kSpecSlots * kSpecSlotBytes + kSpecScratchBytes;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -1423,7 +1429,8 @@ cudaError_t launch_spectral(const SpecUnit* units, int n_units, int total_row_bl
   e = cudaGetLastError();
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
     if (seg_grid > 0) {
-      spectral_segment_kernel<<<seg_grid, 256, kSegSmem, stream>>>(units, seg_unit, blk_seg, vecs, parts, err);
+      spectral_segment_kernel<<<seg_grid, 256, kSegSmem, stream>>>(units, seg_unit, blk_seg, vecs, parts, err,
+                                                                   wait_limit_ns, withhold);
       if ((e = cudaGetLastError()) != cudaSuccess) break;
     }
     if (total_row_blocks > 0) {

@@ -1,4 +1,5 @@
-"""The bounded waits of the Newton-Schulz kernel, made to run out on purpose.
+"""The bounded waits of the Newton-Schulz kernel and of the spectral segment
+pass, made to run out on purpose.
 
 Every mbarrier wait in the kernel gives up after a time limit, records a
 wait-timeout code in the first word of the workspace and lets the kernel
@@ -85,3 +86,40 @@ def test_injected_wait_timeout_is_reported_and_the_context_stays_usable(cuda_lib
         ref = O.newton_schulz(O.frobenius_normalize(mom), k)
         got = us[u].double().cpu().numpy()
         assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 2e-2
+
+
+def test_injected_spectral_wait_timeout_is_reported_and_the_context_stays_usable(cuda_lib, monkeypatch):
+    """The spectral segment pass's bounded waits: with its row loads withheld
+    (SIGNMUON_SPECTRAL_INJECT_WAIT_TIMEOUT_US) every block gives up after the
+    limit and records the spectral wait-timeout code; the next normal call on
+    the same context and workspace matches the oracle.  One-warp rows (768
+    columns) and three-warp teams (2304 columns)."""
+    shapes, M, iters = [(256, 768), (300, 2304)], 2, 2
+    stream = torch.cuda.current_stream().cuda_stream
+    grads, moms = _inputs(shapes, M)
+    nbytes = L.signmuon_spectral_workspace_bytes(shapes, M)
+    wk = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    xs, inv = _momentum(shapes, M, [g.cuda() for g in grads], [m.clone().cuda() for m in moms], stream)
+    torch.cuda.synchronize()
+
+    # 1. Rows withheld, 20 ms limit: `iters` segment passes, each gives up once.
+    monkeypatch.setenv("SIGNMUON_SPECTRAL_INJECT_WAIT_TIMEOUT_US", "20000")
+    t0 = time.perf_counter()
+    L.signmuon_spectral_norm(shapes, M, [x.data_ptr() for x in xs], iters, inv.data_ptr(), wk.data_ptr(), wk.numel(),
+                             stream)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert L.signmuon_device_error(wk.data_ptr(), stream) == 0x105
+    assert elapsed < 1.5, elapsed                  # far below the 2 s default limit per pass
+    assert L.signmuon_device_error(wk.data_ptr(), stream) == 0     # read and cleared
+
+    # 2. The same context, workspace and stream, normal operation.
+    monkeypatch.delenv("SIGNMUON_SPECTRAL_INJECT_WAIT_TIMEOUT_US")
+    L.signmuon_spectral_norm(shapes, M, [x.data_ptr() for x in xs], iters, inv.data_ptr(), wk.data_ptr(), wk.numel(),
+                             stream)
+    torch.cuda.synchronize()
+    assert L.signmuon_device_error(wk.data_ptr(), stream) == 0
+    for u, (g, m0) in enumerate(zip(grads, moms)):
+        mom = O.momentum_update(m0.double().numpy(), g.double().numpy(), float(np.float32(0.9)))
+        ref = 1.0 / (O.spectral_norm_estimate(O.round_to_bf16(mom), iters) + O.NORM_EPS)
+        assert abs(inv[u].item() - ref) <= 2e-4 * ref, (u, inv[u].item(), ref)
