@@ -277,6 +277,14 @@ signmuon_status signmuon_momentum_sign(const signmuon_shape* shapes, int n_mats,
 }
 
 // ------------------------------------------------------------ spectral scaling
+// Relative cost per byte of a segment in the segment pass: a row's teams of
+// T warps leave 8 - (8 / T) T warps of the block idle (two for three-warp
+// teams), and multi-warp teams read their rows twice from shared memory
+// (3 % slower per byte than one warp per row on nanoGPT-small's shapes).
+static double spec_cost_per_byte(int cols) {
+  const int t = spec_team_warps(cols);
+  return 8.0 / (spec_teams(cols) * t) * (t > 1 ? 1.03 : 1.0);
+}
 // Spectral workspace: header | units | seg_unit | blk_seg | v | partials.
 struct SpecLayout {
   size_t units, seg_unit, blk_seg, vecs, parts, total;  // byte offsets (total = size)
@@ -338,8 +346,8 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
   SpecUnit* hu = reinterpret_cast<SpecUnit*>(blob.data());
   int32_t* seg_unit = reinterpret_cast<int32_t*>(blob.data() + (lay.seg_unit - lay.units));
   int32_t* blk_seg = reinterpret_cast<int32_t*>(blob.data() + (lay.blk_seg - lay.units));
-  std::vector<int64_t> seg_bytes;
-  seg_bytes.reserve(lay.segs);
+  std::vector<double> seg_cost;  // estimated cost of each segment (bytes x cost per byte)
+  seg_cost.reserve(lay.segs);
   int64_t voff = 0, poff = 0;
   int blocks = 0, segs = 0;
   for (int i = 0; i < n_mats; ++i) {
@@ -365,7 +373,8 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
       if (n_seg > 0) {
         for (int k = 0; k < n_seg; ++k) {
           seg_unit[segs + k] = ui;
-          seg_bytes.push_back((int64_t)std::min(kSpecSegRows, u.rows - k * kSpecSegRows) * u.cols * 2);
+          seg_cost.push_back((double)std::min(kSpecSegRows, u.rows - k * kSpecSegRows) * u.cols * 2.0 *
+                             spec_cost_per_byte(u.cols));
         }
         segs += n_seg;
       } else {
@@ -374,16 +383,16 @@ signmuon_status signmuon_spectral_norm(const signmuon_shape* shapes, int n_mats,
     }
   }
   // Segment-pass blocks (two per SM) take contiguous ranges of segments
-  // holding about equal shares of the bytes.
+  // holding about equal shares of the estimated cost.
   const int seg_grid = std::min(std::min(segs, 2 * sm_count()), kSpecMaxGrid);
-  int64_t total = 0;
-  for (int64_t b : seg_bytes) total += b;
+  double total = 0.0;
+  for (double c : seg_cost) total += c;
   int sgi = 0;
-  int64_t before = 0;
+  double before = 0.0;
   blk_seg[0] = 0;
   for (int b = 1; b < seg_grid; ++b) {
-    const int64_t target = total * b / seg_grid;
-    while (sgi < segs && before + seg_bytes[sgi] / 2 < target) before += seg_bytes[sgi++];
+    const double target = total * b / seg_grid;
+    while (sgi < segs && before + seg_cost[sgi] / 2 < target) before += seg_cost[sgi++];
     blk_seg[b] = sgi;
   }
   if (seg_grid > 0) blk_seg[seg_grid] = segs;
